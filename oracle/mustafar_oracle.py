@@ -1,0 +1,237 @@
+"""Plain CPU oracle for Mustafar's hot path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
+import this module.  The product path (the CUDA library and its binding) never
+does; it shares no code, table or helper with this file.
+
+What it computes, and from which passage:
+
+* Per-token magnitude pruning of the Key and Value caches to an unstructured
+  sparsity (MUSTAFAR summary, atlas.scime.ai, "Approach"; Mustafar abstract,
+  catalyzex author page): every (token, kv head) vector of ``d`` channels keeps
+  its ``k`` largest-magnitude elements and zeroes the rest.
+* A bitmap-based compressed format (same two passages): a bitmap marks the kept
+  positions, the kept fp16 values are packed, and per-tile offsets locate them.
+  The pages give no layout; this oracle follows the library's own choices, which
+  are written out in ``keep_count``, ``compress`` and ``compressed_bytes`` below.
+* Decode attention over the pruned caches (the abstract: the kernel computes
+  "directly over compressed caches"): the exact result it must reach is plain
+  softmax attention over the pruned K and V, computed here in float64.
+
+Readings where the pages are silent (each is listed in the design notes):
+keep-count ``k = d - floor(s*d)``; magnitude key = fp16 bits with the sign bit
+cleared; ties go to the lower channel index; kept values are packed in
+ascending channel order; bit ``c % 32`` of 32-bit word ``c // 32`` marks channel
+``c``; tiles are 64 tokens with 32-bit offsets counted in elements; every token,
+including the newest, is pruned; the new decode token attends to itself; q head
+``hq`` reads kv head ``hq // (Hq/Hkv)``.
+
+Arrays of fp16 numbers are passed as their raw bits (``np.uint16``) so that both
+sides see identical inputs and the compressed bytes can be compared exactly.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+TILE_TOKENS = 64
+WORD_BITS = 32
+
+
+# --------------------------------------------------------------------------------------
+# keep count and magnitude key
+# --------------------------------------------------------------------------------------
+def keep_count(d: int, sparsity: float) -> int:
+    """Number of channels a token keeps: ``d - floor(s*d)``.
+
+    Sparsity "s" is the fraction pruned (README, Part II: "50% sparsity is 0.5").
+    ``s`` arrives as a 32-bit float (as it does through the library's C call) and
+    the product is formed in double, so the target sparsity is never exceeded.
+    """
+    s = float(np.float32(sparsity))
+    if not (0.0 <= s < 1.0):
+        raise ValueError("sparsity must lie in [0, 1)")
+    return int(d - math.floor(s * d))
+
+
+def magnitude_key(x_bits: np.ndarray) -> np.ndarray:
+    """|x| ordering key of fp16 bit patterns: the 15 low bits (sign cleared).
+
+    For finite fp16 numbers this integer order equals the order of |x|; +0 and -0
+    share key 0.  Inf and NaN patterns rank above every finite value.
+    """
+    return (np.asarray(x_bits, dtype=np.uint16) & np.uint16(0x7FFF)).astype(np.int32)
+
+
+# --------------------------------------------------------------------------------------
+# selection (per-token magnitude pruning)
+# --------------------------------------------------------------------------------------
+def select_sort(x_bits: np.ndarray, k: int) -> np.ndarray:
+    """Boolean kept-mask over the last axis: the ``k`` largest keys, lower channel first on ties.
+
+    Implemented as a stable sort of the negated keys: equal keys keep their
+    channel order, so the first ``k`` positions of the sorted order are the kept set.
+    """
+    m = magnitude_key(x_bits)
+    d = m.shape[-1]
+    order = np.argsort(0x7FFF - m, axis=-1, kind="stable")
+    keep_idx = order[..., :k]
+    mask = np.zeros(m.shape, dtype=bool)
+    np.put_along_axis(mask, keep_idx, True, axis=-1)
+    assert mask.shape[-1] == d
+    return mask
+
+
+def select_rank_bruteforce(x_bits: np.ndarray, k: int) -> np.ndarray:
+    """Same selection by rank counting, for tiny inputs only.
+
+    rank(c) = #{j : m_j > m_c} + #{j < c : m_j == m_c}; channel c is kept iff rank(c) < k.
+    """
+    m = magnitude_key(x_bits)
+    flat = m.reshape(-1, m.shape[-1])
+    out = np.zeros(flat.shape, dtype=bool)
+    d = flat.shape[1]
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        for c in range(d):
+            rank = 0
+            for j in range(d):
+                if row[j] > row[c] or (row[j] == row[c] and j < c):
+                    rank += 1
+            out[r, c] = rank < k
+    return out.reshape(m.shape)
+
+
+def prune(x_bits: np.ndarray, k: int) -> np.ndarray:
+    """Pruned fp16 bits: kept elements keep their exact bits (sign, -0 included), the rest become +0."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    return np.where(select_sort(x, k), x, np.uint16(0)).astype(np.uint16)
+
+
+# --------------------------------------------------------------------------------------
+# bitmap format
+# --------------------------------------------------------------------------------------
+def bitmap_words(mask: np.ndarray) -> np.ndarray:
+    """Pack a [..., d] kept-mask into [..., d/32] uint32 words, channel c -> bit c%32 of word c//32."""
+    d = mask.shape[-1]
+    assert d % WORD_BITS == 0
+    m = mask.reshape(mask.shape[:-1] + (d // WORD_BITS, WORD_BITS)).astype(np.uint64)
+    weights = (np.uint64(1) << np.arange(WORD_BITS, dtype=np.uint64))
+    return (m * weights).sum(axis=-1).astype(np.uint32)
+
+
+def bitmap_to_mask(words: np.ndarray, d: int) -> np.ndarray:
+    """Inverse of ``bitmap_words``."""
+    w = np.asarray(words, dtype=np.uint32).astype(np.uint64)
+    bits = (w[..., None] >> np.arange(WORD_BITS, dtype=np.uint64)) & np.uint64(1)
+    return bits.reshape(w.shape[:-1] + (d,)).astype(bool)
+
+
+def compress(x_bits: np.ndarray, k: int, capacity: int, L: int | None = None) -> dict:
+    """Compress tokens [0, L) of a dense cache ``[B, H, T, d]`` (fp16 bits) into the bitmap format.
+
+    Output arrays, one stream per (b, h), sized for ``capacity`` tokens:
+
+    * ``bitmap``  uint32 [B, H, capacity, d/32] - kept positions of each token;
+    * ``values``  uint16 [B, H, capacity*k]     - kept fp16 bits, ascending channel,
+      token t's run starting at element t*k;
+    * ``tile_offset`` uint32 [B, H, capacity/64] - element offset of each 64-token
+      tile's first value within its stream (the popcount prefix sum).
+
+    Slots of tokens >= L are left zero here; the library leaves them untouched.
+    """
+    x = np.asarray(x_bits, dtype=np.uint16)
+    B, H, T, d = x.shape
+    L = T if L is None else L
+    assert capacity % TILE_TOKENS == 0 and L <= capacity and L <= T
+    mask = select_sort(x[:, :, :L], k)
+    bitmap = np.zeros((B, H, capacity, d // WORD_BITS), dtype=np.uint32)
+    bitmap[:, :, :L] = bitmap_words(mask)
+    values = np.zeros((B, H, capacity * k), dtype=np.uint16)
+    kept = x[:, :, :L][mask].reshape(B, H, L * k)  # boolean indexing walks channels in ascending order
+    values[:, :, : L * k] = kept
+    counts = np.zeros((B, H, capacity), dtype=np.int64)
+    counts[:, :, :L] = mask.sum(axis=-1)
+    # prefix sums over the tokens before each tile; tokens >= L are counted as full (k) so that the
+    # offsets of not-yet-written tiles equal their final value (the closed form 64*i*k).
+    counts[:, :, L:] = k
+    starts = np.concatenate([np.zeros((B, H, 1), np.int64), np.cumsum(counts, axis=-1)[..., :-1]], axis=-1)
+    tile_offset = starts[:, :, ::TILE_TOKENS].astype(np.uint32)
+    return {"bitmap": bitmap, "values": values, "tile_offset": tile_offset, "k": k, "L": L}
+
+
+def decompress(bitmap: np.ndarray, values: np.ndarray, k: int, L: int, d: int) -> np.ndarray:
+    """Dense fp16 bits [B, H, L, d] rebuilt from the bitmap and packed values (pruned positions are +0)."""
+    mask = bitmap_to_mask(bitmap[:, :, :L], d)
+    B, H = mask.shape[:2]
+    out = np.zeros((B, H, L, d), dtype=np.uint16)
+    out[mask] = np.asarray(values, dtype=np.uint16)[:, :, : L * k].reshape(-1)
+    return out
+
+
+def compressed_bytes(L: int, k: int, capacity: int, d: int = 128) -> int:
+    """Closed-form bytes of one stream: bitmap d/8 B per token, 2k B of values per token, 4 B per tile."""
+    return (d // 8) * L + 2 * k * L + 4 * (capacity // TILE_TOKENS)
+
+
+def append(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
+    """Prune + compress one new token per (b, h) into slot ``pos[b]`` (in place).
+
+    The same per-token pruning as the prefill path, applied to the token the
+    decode step produces (the abstract: pruning and compression at runtime).
+    """
+    k = cache["k"]
+    x = np.asarray(x_new_bits, dtype=np.uint16)  # [B, H, d]
+    B, H, d = x.shape
+    mask = select_sort(x, k)
+    words = bitmap_words(mask)
+    for b in range(B):
+        p = int(pos[b])
+        cache["bitmap"][b, :, p] = words[b]
+        for h in range(H):
+            cache["values"][b, h, p * k:(p + 1) * k] = x[b, h][mask[b, h]]
+
+
+# --------------------------------------------------------------------------------------
+# attention over the pruned caches
+# --------------------------------------------------------------------------------------
+def f16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def attention(q_bits: np.ndarray, kp_bits: np.ndarray, vp_bits: np.ndarray, seq_len, scale: float):
+    """Softmax attention of one decode query per (b, q head) over the pruned caches, in float64.
+
+    q ``[B, Hq, d]``; K~/V~ ``[B, Hkv, >=L_b, d]`` (pruned fp16 bits); ``seq_len[b]`` tokens per row.
+    For q head hq the kv head is g = hq // (Hq/Hkv).  z_t = scale * q . K~_t,
+    p = softmax(z), o = sum_t p_t V~_t, lse = log sum_t exp(z_t).
+    Returns (o [B, Hq, d] float64, lse [B, Hq] float64).
+    """
+    q = f16_to_f64(q_bits)
+    B, Hq, d = q.shape
+    Hkv = kp_bits.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        Lb = int(seq_len[b])
+        K = f16_to_f64(kp_bits[b, :, :Lb])  # [Hkv, L, d]
+        V = f16_to_f64(vp_bits[b, :, :Lb])
+        for hq in range(Hq):
+            g = hq // G
+            z = scale * (K[g] @ q[b, hq])
+            zmax = z.max()
+            e = np.exp(z - zmax)
+            ssum = e.sum()
+            out[b, hq] = (e / ssum) @ V[g]
+            lse[b, hq] = zmax + math.log(ssum)
+    return out, lse
+
+
+def attention_over_compressed(q_bits, kc: dict, vc: dict, seq_len, scale: float, d: int):
+    """Attention read back from the compressed caches (decompress, then ``attention``)."""
+    Lmax = int(max(seq_len))
+    kp = decompress(kc["bitmap"], kc["values"], kc["k"], Lmax, d)
+    vp = decompress(vc["bitmap"], vc["values"], vc["k"], Lmax, d)
+    return attention(q_bits, kp, vp, seq_len, scale)

@@ -1,0 +1,273 @@
+"""Checks that pin the oracle to the pages and to mathematics, not to itself.
+
+Each ``pin_*`` takes an oracle namespace ``O`` (the real ``oracle`` package, or a
+mutant built by ``test_oracle_mutants.py``) and raises ``AssertionError`` when the
+oracle disagrees with the fact it checks.  Facts used:
+
+* hand-derived fixtures under ``tests/golden/`` (selection, bitmap bit order,
+  value order, keep-count rounding, a two-token attention with logits 0 and ln 3);
+* brute-force rank counting on tiny tie-heavy inputs;
+* the threshold invariant of a top-k selection and popcount == k;
+* decompress(compress(x)) == prune(x) and the closed-form compressed size;
+* attention at sparsity 0 against torch's float64 ``scaled_dot_product_attention``;
+* L = 1 gives o = V~_0 exactly; softmax weights sum to 1; token-permutation
+  invariance; a GQA group with equal queries gives equal outputs.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+# fp16 bit patterns with many ties: zeros of both signs, smallest/largest
+# subnormals, 1, 2, the largest finite value, of both signs.
+TIE_HEAVY = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x03FF, 0x3C00, 0xBC00, 0x4000, 0xC000,
+                      0x7BFF, 0xFBFF], dtype=np.uint16)
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _d32_vector():
+    g = _load("select_d32.json")
+    spec = g["x_hex_by_channel"]
+    x = np.zeros(32, dtype=np.uint16)
+    for c in range(32):
+        if str(c) in spec:
+            x[c] = int(spec[str(c)], 16)
+        elif c % 2 == 1:
+            x[c] = int(spec["odd_11_to_31"], 16)
+        else:
+            x[c] = int(spec["even_12_to_30"], 16)
+    return x, g
+
+
+def rand_bits(rng, shape, tie_heavy=False):
+    if tie_heavy:
+        return rng.choice(TIE_HEAVY, size=shape).astype(np.uint16)
+    x = rng.standard_normal(shape).astype(np.float16)
+    return x.view(np.uint16)
+
+
+# ----------------------------------------------------------------------------- selection
+def pin_golden_selection(O):
+    x, g = _d32_vector()
+    for case in g["cases"]:
+        k = case["k"]
+        mask = O.select_sort(x[None, :], k)[0]
+        words = O.bitmap_words(mask[None, :])[0]
+        assert int(words[0]) == int(case["bitmap_hex"], 16), (k, hex(int(words[0])))
+        comp = O.compress(x[None, None, None, :], k, 64)
+        vals = comp["values"][0, 0, :k]
+        if isinstance(case["values_hex"], list):
+            assert [int(v) for v in vals] == [int(h, 16) for h in case["values_hex"]], k
+        else:
+            keep = [c for c in range(32) if (int(case["bitmap_hex"], 16) >> c) & 1]
+            assert [int(v) for v in vals] == [int(x[c]) for c in keep], k
+        assert int(comp["bitmap"][0, 0, 0, 0]) == int(case["bitmap_hex"], 16)
+
+
+def pin_golden_keep_count(O):
+    for case in _load("keep_count.json")["cases"]:
+        assert O.keep_count(case["d"], case["s"]) == case["k"], case
+
+
+def pin_bruteforce_selection(O):
+    rng = np.random.default_rng(11)
+    for d in (32, 128):
+        for tie in (True, False):
+            x = rand_bits(rng, (6, d), tie_heavy=tie)
+            for k in (1, 2, d // 3, d // 2, d - 1, d):
+                a = O.select_sort(x, k)
+                b = O.select_rank_bruteforce(x, k)
+                assert np.array_equal(a, b), (d, tie, k)
+    # exhaustive: every 6-channel pattern over a 3-symbol alphabet {+0, -0, 1.0} padded to 32
+    alphabet = np.array([0x0000, 0x8000, 0x3C00], dtype=np.uint16)
+    idx = np.indices((3,) * 6).reshape(6, -1).T
+    xs = np.zeros((idx.shape[0], 32), dtype=np.uint16)
+    xs[:, :6] = alphabet[idx]
+    xs[:, 6:] = 0x3800  # 0.5 fills the rest
+    for k in (1, 3, 26, 27, 29):
+        assert np.array_equal(O.select_sort(xs, k), O.select_rank_bruteforce(xs, k)), k
+
+
+def pin_threshold_invariant(O):
+    rng = np.random.default_rng(12)
+    for tie in (True, False):
+        x = rand_bits(rng, (64, 128), tie_heavy=tie)
+        m = (x & 0x7FFF).astype(np.int64)
+        for k in (1, 13, 39, 64, 90, 127, 128):
+            mask = O.select_sort(x, k)
+            assert (mask.sum(axis=1) == k).all()
+            for r in range(x.shape[0]):
+                kept, pruned = m[r][mask[r]], m[r][~mask[r]]
+                if pruned.size == 0:
+                    continue
+                assert kept.min() >= pruned.max(), "a pruned element outranks a kept one"
+                edge = kept.min()
+                if pruned.max() == edge:
+                    ki = np.nonzero(mask[r] & (m[r] == edge))[0]
+                    pi = np.nonzero(~mask[r] & (m[r] == edge))[0]
+                    assert ki.max() < pi.min(), "tie not resolved toward the lower channel"
+
+
+# ----------------------------------------------------------------------------- format
+def pin_roundtrip_and_popcount(O):
+    rng = np.random.default_rng(13)
+    B, H, L, d, cap = 2, 3, 150, 128, 192
+    x = rand_bits(rng, (B, H, L, d))
+    x[0, 0, 5] = rand_bits(rng, (d,), tie_heavy=True)
+    for k in (128, 90, 64, 39, 13, 1):
+        comp = O.compress(x, k, cap)
+        words = comp["bitmap"][:, :, :L]
+        pop = np.vectorize(lambda w: bin(int(w)).count("1"))(words).sum(axis=-1)
+        assert (pop == k).all()
+        dec = O.decompress(comp["bitmap"], comp["values"], k, L, d)
+        assert np.array_equal(dec, O.prune(x, k))
+        # pruned positions hold +0, kept positions hold the input bits exactly
+        mask = O.bitmap_to_mask(words, d)
+        assert np.array_equal(dec[mask], x[mask]) and (dec[~mask] == 0).all()
+        # tile offsets = popcount prefix sums at every 64-token boundary = 64*i*k
+        prefix = np.concatenate([[0], np.cumsum(pop[0, 0])])
+        for i in range(cap // 64):
+            expect = prefix[64 * i] if 64 * i <= L else 64 * i * k
+            assert int(comp["tile_offset"][0, 0, i]) == expect == 64 * i * k
+
+
+def pin_compressed_size(O):
+    # closed form per stream: 16 B bitmap + 2k B values per token, 4 B per 64-token tile
+    cases = [(4096, 39, 4160, 4096 * (16 + 78) + 4 * 65), (16384, 90, 16384, 16384 * 196 + 4 * 256),
+             (1024, 64, 1024, 1024 * 144 + 4 * 16), (1, 128, 64, 16 + 256 + 4)]
+    for L, k, cap, expect in cases:
+        assert O.compressed_bytes(L, k, cap, 128) == expect
+    rng = np.random.default_rng(14)
+    x = rand_bits(rng, (1, 1, 130, 128))
+    comp = O.compress(x, 39, 192)
+    used = 130 * 16 + 130 * 39 * 2 + comp["tile_offset"].nbytes
+    assert used == O.compressed_bytes(130, 39, 192, 128)
+    # the pages' ratios (45% of dense at 70% sparsity, 65% at 50%) are upper bounds for this format
+    for s, bound in ((0.7, 0.45), (0.5, 0.65)):
+        k = O.keep_count(128, s)
+        ratio = O.compressed_bytes(16384, k, 16384, 128) / (16384 * 256)
+        assert ratio < bound, (s, ratio)
+
+
+# ----------------------------------------------------------------------------- attention
+def _sdpa_f64(q, K, V, scale, G):
+    # q [B,Hq,d], K/V [B,Hkv,L,d] float64 -> [B,Hq,d]
+    qt = torch.from_numpy(q)[:, :, None, :]
+    Kt = torch.from_numpy(K).repeat_interleave(G, dim=1)
+    Vt = torch.from_numpy(V).repeat_interleave(G, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=scale)
+    return o[:, :, 0, :].numpy()
+
+
+def pin_dense_limit_sdpa(O):
+    rng = np.random.default_rng(15)
+    B, Hq, Hkv, L, d = 2, 8, 2, 77, 128
+    q = rand_bits(rng, (B, Hq, d))
+    K = rand_bits(rng, (B, Hkv, L, d))
+    V = rand_bits(rng, (B, Hkv, L, d))
+    k = O.keep_count(d, 0.0)
+    kc, vc = O.compress(K, k, 128), O.compress(V, k, 128)
+    seq = np.full(B, L)
+    o, lse = O.attention_over_compressed(q, kc, vc, seq, 0.37, d)
+    f = lambda b: b.view(np.float16).astype(np.float64)
+    ref = _sdpa_f64(f(q), f(K), f(V), 0.37, Hq // Hkv)
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
+    z = 0.37 * np.einsum("bgjd,bgld->bgjl", f(q).reshape(B, Hkv, Hq // Hkv, d), f(K))
+    lse_ref = torch.logsumexp(torch.from_numpy(z), dim=-1).numpy().reshape(B, Hq)
+    assert np.allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_golden_attention(O):
+    g = _load("attention_tiny.json")
+    d = 32
+    q = np.zeros((1, 1, d), np.float16); q[0, 0, 0] = 1; q[0, 0, 1] = 1
+    K = np.zeros((1, 1, 2, d), np.float16)
+    K[0, 0, 0, 4:7] = 5
+    K[0, 0, 1, 0], K[0, 0, 1, 1], K[0, 0, 1, 2], K[0, 0, 1, 3] = 1, 0.5, 2, 2
+    V = np.zeros((1, 1, 2, d), np.float16)
+    V[0, 0, 0, :] = 1; V[0, 0, 0, :3] = 4
+    V[0, 0, 1, :] = 0.5; V[0, 0, 1, :3] = 8
+    scale = float(np.float32(math.log(3)))
+    kc = O.compress(K.view(np.uint16), 3, 64)
+    vc = O.compress(V.view(np.uint16), 3, 64)
+    o, lse = O.attention_over_compressed(q.view(np.uint16), kc, vc, [2], scale, d)
+    e = g["expected"]
+    assert np.allclose(o[0, 0, :3], e["o_c0_c2"], atol=e["tol"])
+    assert np.allclose(o[0, 0, 3:], e["o_other"], atol=e["tol"])
+    assert abs(lse[0, 0] - e["lse"]) < e["tol"]
+
+
+def pin_attention_invariants(O):
+    rng = np.random.default_rng(16)
+    B, Hq, Hkv, L, d = 2, 8, 2, 70, 128
+    G = Hq // Hkv
+    K = rand_bits(rng, (B, Hkv, L, d))
+    V = rand_bits(rng, (B, Hkv, L, d))
+    q = rand_bits(rng, (B, Hq, d))
+    k = 39
+    kp, vp = O.prune(K, k), O.prune(V, k)
+    # L = 1: the output is the single pruned value row, exactly
+    o1, lse1 = O.attention(q, kp, vp, [1, 1], 1.0)
+    f = lambda b: b.view(np.float16).astype(np.float64)
+    for b in range(B):
+        for hq in range(Hq):
+            assert np.array_equal(o1[b, hq], f(vp[b, hq // G, 0]))
+    # weights sum to one: with V~ replaced by all-ones rows, o == 1 everywhere
+    ones = np.full_like(vp, 0x3C00)
+    o_ones, _ = O.attention(q, kp, ones, [L, L - 5], 0.8)
+    assert np.allclose(o_ones, 1.0, rtol=0, atol=1e-13)
+    # token permutation invariance
+    perm = rng.permutation(L)
+    oa, la = O.attention(q, kp, vp, [L, L], 0.8)
+    ob, lb = O.attention(q, kp[:, :, perm], vp[:, :, perm], [L, L], 0.8)
+    assert np.allclose(oa, ob, rtol=1e-12, atol=1e-13) and np.allclose(la, lb, rtol=1e-12)
+    # equal queries inside a GQA group give equal outputs; different kv heads differ
+    qg = q.copy()
+    for g_ in range(Hkv):
+        qg[:, g_ * G:(g_ + 1) * G] = q[:, g_ * G][:, None]
+    og, _ = O.attention(qg, kp, vp, [L, L], 0.8)
+    for g_ in range(Hkv):
+        for j in range(1, G):
+            assert np.array_equal(og[:, g_ * G + j], og[:, g_ * G])
+    assert not np.allclose(og[:, 0], og[:, G])
+    # q head hq reads kv head hq // G: zeroing kv head 1's values changes only heads G..2G-1
+    vz = vp.copy(); vz[:, 1] = 0
+    oz, _ = O.attention(q, kp, vz, [L, L], 0.8)
+    assert np.array_equal(oz[:, :G], oa[:, :G]) and np.allclose(oz[:, G:2 * G], 0)
+
+
+def pin_append_equals_compress(O):
+    rng = np.random.default_rng(17)
+    B, H, L, d, cap, k = 2, 2, 70, 128, 128, 39
+    x = rand_bits(rng, (B, H, L + 3, d))
+    full = O.compress(x, k, cap, L + 3)
+    part = O.compress(x, k, cap, L)
+    for s in range(3):
+        O.append(part, x[:, :, L + s], np.full(B, L + s))
+    for key in ("bitmap", "values", "tile_offset"):
+        assert np.array_equal(full[key], part[key]), key
+
+
+ALL_PINS = [pin_golden_selection, pin_golden_keep_count, pin_bruteforce_selection, pin_threshold_invariant,
+            pin_roundtrip_and_popcount, pin_compressed_size, pin_dense_limit_sdpa, pin_golden_attention,
+            pin_attention_invariants, pin_append_equals_compress]
+
+
+def failing_pins(O):
+    bad = []
+    for pin in ALL_PINS:
+        try:
+            pin(O)
+        except Exception:  # a mutant may also crash; that counts as caught
+            bad.append(pin.__name__)
+    return bad

@@ -1,0 +1,155 @@
+"""Plant plausible mistakes in copies of the oracle and check that some pin catches each one.
+
+Mistakes are planted in the oracle only, on the CPU.
+"""
+import types
+
+import numpy as np
+import pytest
+
+import oracle.mustafar_oracle as real
+from tests import oracle_pins as P
+
+
+def _mutant(**overrides):
+    ns = types.SimpleNamespace(**{n: getattr(real, n) for n in dir(real) if not n.startswith("__")})
+    for name, fn in overrides.items():
+        setattr(ns, name, fn)
+    # rebind functions that call each other so they see the overrides
+    def compress(x_bits, k, capacity, L=None):
+        x = np.asarray(x_bits, dtype=np.uint16)
+        B, H, T, d = x.shape
+        L = T if L is None else L
+        mask = ns.select_sort(x[:, :, :L], k)
+        bitmap = np.zeros((B, H, capacity, d // 32), dtype=np.uint32)
+        bitmap[:, :, :L] = ns.bitmap_words(mask)
+        values = np.zeros((B, H, capacity * k), dtype=np.uint16)
+        values[:, :, : L * k] = x[:, :, :L][mask].reshape(B, H, L * k)
+        starts = np.arange(capacity // 64, dtype=np.int64) * 64 * k
+        return {"bitmap": bitmap, "values": values,
+                "tile_offset": np.broadcast_to(starts, (B, H, capacity // 64)).astype(np.uint32), "k": k, "L": L}
+    if "compress" not in overrides:
+        ns.compress = compress
+    def prune(x_bits, k):
+        x = np.asarray(x_bits, dtype=np.uint16)
+        return np.where(ns.select_sort(x, k), x, np.uint16(0)).astype(np.uint16)
+    if "prune" not in overrides:
+        ns.prune = prune
+    def decompress(bitmap, values, k, L, d):
+        mask = ns.bitmap_to_mask(bitmap[:, :, :L], d)
+        out = np.zeros(mask.shape, dtype=np.uint16)
+        out[mask] = np.asarray(values)[:, :, : L * k].reshape(-1)
+        return out
+    if "decompress" not in overrides:
+        ns.decompress = decompress
+    def attention_over_compressed(q_bits, kc, vc, seq_len, scale, d):
+        Lmax = int(max(seq_len))
+        return ns.attention(q_bits, ns.decompress(kc["bitmap"], kc["values"], kc["k"], Lmax, d),
+                            ns.decompress(vc["bitmap"], vc["values"], vc["k"], Lmax, d), seq_len, scale)
+    ns.attention_over_compressed = attention_over_compressed
+    def append(cache, x_new_bits, pos):
+        k = cache["k"]
+        x = np.asarray(x_new_bits, dtype=np.uint16)
+        mask = ns.select_sort(x, k)
+        words = ns.bitmap_words(mask)
+        for b in range(x.shape[0]):
+            p = int(pos[b])
+            cache["bitmap"][b, :, p] = words[b]
+            for h in range(x.shape[1]):
+                cache["values"][b, h, p * k:(p + 1) * k] = x[b, h][mask[b, h]]
+    if "append" not in overrides:
+        ns.append = append
+    return ns
+
+
+def sel_ascending(x_bits, k):           # wrong sign: keeps the smallest magnitudes
+    m = real.magnitude_key(x_bits)
+    order = np.argsort(m, axis=-1, kind="stable")[..., :k]
+    mask = np.zeros(m.shape, bool); np.put_along_axis(mask, order, True, axis=-1); return mask
+
+
+def sel_high_index_ties(x_bits, k):     # wrong tie rule: higher channel wins
+    m = real.magnitude_key(x_bits)[..., ::-1]
+    order = np.argsort(0x7FFF - m, axis=-1, kind="stable")[..., :k]
+    mask = np.zeros(m.shape, bool); np.put_along_axis(mask, order, True, axis=-1); return mask[..., ::-1]
+
+
+def sel_signed(x_bits, k):              # compares signed values instead of magnitudes
+    v = np.asarray(x_bits, np.uint16).view(np.float16).astype(np.float64)
+    order = np.argsort(-v, axis=-1, kind="stable")[..., :k]
+    mask = np.zeros(v.shape, bool); np.put_along_axis(mask, order, True, axis=-1); return mask
+
+
+def words_msb_first(mask):              # wrong bit order inside a word
+    return real.bitmap_words(np.flip(mask.reshape(mask.shape[:-1] + (-1, 32)), -1).reshape(mask.shape))
+
+
+def keep_round(d, s):                   # rounds (1-s)*d instead of d - floor(s*d)
+    return int(round((1 - float(np.float32(s))) * d))
+
+
+def size_no_offsets(L, k, capacity, d=128):
+    return (d // 8) * L + 2 * k * L
+
+
+def size_bits_as_bytes(L, k, capacity, d=128):
+    return d * L + 2 * k * L + 4 * (capacity // 64)
+
+
+def attn_no_scale(q, kp, vp, seq_len, scale):
+    return real.attention(q, kp, vp, seq_len, 1.0)
+
+
+def attn_wrong_group(q_bits, kp_bits, vp_bits, seq_len, scale):   # hq % Hkv instead of hq // G
+    B, Hq, d = q_bits.shape
+    Hkv = kp_bits.shape[1]
+    perm = np.array([(hq % Hkv) * (Hq // Hkv) + hq // Hkv for hq in range(Hq)])
+    inv = np.argsort(perm)
+    o, l = real.attention(q_bits[:, perm], kp_bits, vp_bits, seq_len, scale)
+    return o[:, inv], l[:, inv]
+
+
+def attn_unnormalised(q, kp, vp, seq_len, scale):
+    o, l = real.attention(q, kp, vp, seq_len, scale)
+    return o * np.exp(l)[..., None] / np.exp(l).mean(), l
+
+
+def attn_drop_last(q, kp, vp, seq_len, scale):      # attends over one token too few
+    return real.attention(q, kp, vp, [max(1, int(s) - 1) for s in seq_len], scale)
+
+
+def attn_lse_log2(q, kp, vp, seq_len, scale):
+    o, l = real.attention(q, kp, vp, seq_len, scale)
+    return o, l / np.log(2)
+
+
+def prune_negzero(x_bits, k):           # pruned slots written as -0 instead of +0
+    x = np.asarray(x_bits, np.uint16)
+    return np.where(real.select_sort(x, k), x, np.uint16(0x8000)).astype(np.uint16)
+
+
+MUTANTS = {
+    "select ascending": dict(select_sort=sel_ascending),
+    "ties to higher index": dict(select_sort=sel_high_index_ties),
+    "signed compare": dict(select_sort=sel_signed),
+    "bitmap msb first": dict(bitmap_words=words_msb_first),
+    "keep count rounded": dict(keep_count=keep_round),
+    "size without offsets": dict(compressed_bytes=size_no_offsets),
+    "bitmap counted in bytes": dict(compressed_bytes=size_bits_as_bytes),
+    "scale dropped": dict(attention=attn_no_scale),
+    "wrong gqa mapping": dict(attention=attn_wrong_group),
+    "softmax not normalised": dict(attention=attn_unnormalised),
+    "last token dropped": dict(attention=attn_drop_last),
+    "lse in log2": dict(attention=attn_lse_log2),
+    "pruned slots -0": dict(prune=prune_negzero),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name):
+    caught = P.failing_pins(_mutant(**MUTANTS[name]))
+    assert caught, f"no pin catches the planted mistake '{name}'"
+
+
+def test_unmutated_copy_passes():
+    assert P.failing_pins(_mutant()) == []

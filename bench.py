@@ -1,0 +1,445 @@
+"""Benchmark of the Mustafar hot path on B200.
+
+A step is one decode step of the Llama-3-8B-like GQA workload at batch 8: prune +
+compress the new token's K and V into the compressed caches (two append launches),
+then sparse decode attention over the 4097..4160-token compressed context (one launch).
+The workload is 4096 prefill tokens plus 64 decode steps at K and V sparsity 0.7; timed
+steps cycle through the 64 decode positions.  Inputs are synthetic (seeded; see
+``unstructured_sparse_kv_b200/synth.py``).
+
+Timing: CUDA graphs of 64 steps are replayed; every step reads one of 8 rotating copies
+of the compressed caches (8 x 49.5 MB, over twice the 126 MB L2), so no step finds the
+previous step's cache in L2.  The timed region is bracketed by a barrier and
+``torch.cuda.synchronize()``; the time is the max over ranks.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode-attn µs/step & compressed-KV GB/s (fraction of HBM peak) vs sparsity"
+UNIT = "us/step"
+WORKLOAD = dict(batch=8, q_heads=32, kv_heads=8, head_dim=128, context=4096, decode_steps=64,
+                sparsity_k=0.7, sparsity_v=0.7)
+ROTATE = 8
+GRAPH_STEPS = 64
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------------------------------ helpers
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs the same workload shape on its own seeded batch (weak scaling, no exchange)."""
+    return 1002 + 1000 * rank
+
+
+def aggregate_us_per_step(max_elapsed_ms: float, steps: int, world: int) -> float:
+    """Whole-job time per step: all ranks' steps together took the slowest rank's time."""
+    return max_elapsed_ms * 1000.0 / (steps * world)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_algorithmic_bytes(B, Hq, Hkv, d, lens, kK, kV):
+    """Bytes the decode attention must move: every stored token's bitmaps and kept values
+    of K and V, plus q in and out (fp16).  Split partials are overhead, not credited."""
+    per_tok = 2 * (d // 8) + 2 * (kK + kV)
+    return sum(Hkv * L * per_tok for L in lens) + 2 * (2 * B * Hq * d)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("common.cuh", "decode_attn.cu"):
+        with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on this kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_attn_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        if rec.get("kernel_source_sha256_16") == kernel_source_hash():
+            return float(rec["dram_bytes_per_launch_full_workload"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.dev), "-lms", "200"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.path is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------ workload
+class Workload:
+    def __init__(self, seed: int, device):
+        import torch
+        import unstructured_sparse_kv_b200 as M
+        from unstructured_sparse_kv_b200 import synth
+        w = WORKLOAD
+        self.M, self.torch = M, torch
+        self.B, self.Hq, self.Hkv, self.d = w["batch"], w["q_heads"], w["kv_heads"], w["head_dim"]
+        self.L0, self.steps = w["context"], w["decode_steps"]
+        self.cap = self.L0 + self.steps
+        self.sK, self.sV = w["sparsity_k"], w["sparsity_v"]
+        self.dev = device
+        B, Hq, Hkv, d, cap = self.B, self.Hq, self.Hkv, self.d, self.cap
+        # dense caches hold the prefill and the 64 decode tokens; every copy is fully compressed so that
+        # each append rewrites a slot with identical bits and every copy stays a valid cache
+        self.K = synth.keys(B, Hkv, cap, d, seed, device)
+        self.V = synth.values(B, Hkv, cap, d, seed, device)
+        self.kc, self.vc = [], []
+        for _ in range(ROTATE):
+            kc = M.CompressedCache(B, Hkv, cap, self.sK, device=device)
+            vc = M.CompressedCache(B, Hkv, cap, self.sV, device=device)
+            M.mustafar_compress(self.K, cap, self.sK, kc)
+            M.mustafar_compress(self.V, cap, self.sV, vc)
+            self.kc.append(kc)
+            self.vc.append(vc)
+        self.q = torch.stack([synth.queries(B, Hq, d, seed, device, step=i) for i in range(self.steps)])
+        self.kn = self.K[:, :, self.L0:].permute(2, 0, 1, 3).contiguous()  # [steps, B, Hkv, d]
+        self.vn = self.V[:, :, self.L0:].permute(2, 0, 1, 3).contiguous()
+        self.pos = (self.L0 + torch.arange(self.steps, dtype=torch.int32, device=device))[:, None].repeat(1, B)
+        self.seq = (self.pos + 1).contiguous()
+        self.out = torch.empty(B, Hq, d, dtype=torch.float16, device=device)
+        self.lse = torch.empty(B, Hq, dtype=torch.float32, device=device)
+        self.ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, cap), dtype=torch.uint8, device=device)
+        self.splits = M.mustafar_decode_plan_splits(B, Hkv, cap, self.kc[0].keep, self.vc[0].keep)
+        self.compressed_bytes = self.kc[0].nbytes() + self.vc[0].nbytes()
+
+    def step(self, i: int, attend_only: bool = False):
+        M, r, j = self.M, i % ROTATE, i % self.steps
+        if not attend_only:
+            M.mustafar_append(self.kn[j], self.pos[j], self.kc[r])
+            M.mustafar_append(self.vn[j], self.pos[j], self.vc[r])
+        M.mustafar_decode_attn(self.q[j], self.kc[r], self.vc[r], self.seq[j], self.cap, 1.0, out=self.out,
+                               lse=self.lse, workspace=self.ws)
+
+    def graph(self, attend_only=False, dense=None):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        for i in range(GRAPH_STEPS):  # warm once eagerly (plans, attributes) before capture
+            (dense.step(i) if dense else self.step(i, attend_only))
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for i in range(GRAPH_STEPS):
+                (dense.step(i) if dense else self.step(i, attend_only))
+        return g
+
+
+class DenseBaseline:
+    """Dense fp16 decode attention over the same (unpruned) caches, 3 rotating copies (> 3x L2)."""
+
+    def __init__(self, wl: Workload):
+        import torch
+        self.wl, self.M = wl, wl.M
+        self.copies = [wl.K] + [wl.K.clone() for _ in range(2)]
+        self.vcopies = [wl.V] + [wl.V.clone() for _ in range(2)]
+        self.ws = torch.zeros(wl.M.mustafar_decode_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.cap), dtype=torch.uint8,
+                              device=wl.dev)
+
+    def step(self, i: int):
+        wl, r, j = self.wl, i % 3, i % self.wl.steps
+        self.M.mustafar_dense_decode_attn(wl.q[j], self.copies[r], self.vcopies[r], wl.seq[j], wl.cap, 1.0,
+                                          out=wl.out, lse=wl.lse, workspace=self.ws)
+
+
+def time_graph(g, replays: int, stream) -> float:
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(replays):
+        g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle
+def oracle_decode_sample(budget_s: float = 12.0, seed: int = 1002):
+    """Time the CPU oracle (as it stands) on the same decode workload: append K and V, then
+    attention over the compressed caches, over all 64 (b, kv head) streams, for as many
+    decode steps as fit in ``budget_s``.  BLAS limited to one thread."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    from unstructured_sparse_kv_b200 import synth
+    w = WORKLOAD
+    B, Hq, Hkv, d, L0, steps = w["batch"], w["q_heads"], w["kv_heads"], w["head_dim"], w["context"], w["decode_steps"]
+    cap = L0 + steps
+    to_bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    K = to_bits(synth.keys(B, Hkv, cap, d, seed, "cpu"))
+    V = to_bits(synth.values(B, Hkv, cap, d, seed, "cpu"))
+    kK, kV = oracle.keep_count(d, w["sparsity_k"]), oracle.keep_count(d, w["sparsity_v"])
+    kc = oracle.compress(K, kK, cap, L0)
+    vc = oracle.compress(V, kV, cap, L0)
+    done, t_total = 0, 0.0
+    with threadpool_limits(limits=1):
+        while done < steps:
+            q = to_bits(synth.queries(B, Hq, d, seed, "cpu", step=done))
+            t0 = time.perf_counter()
+            pos = np.full(B, L0 + done)
+            oracle.append(kc, K[:, :, L0 + done], pos)
+            oracle.append(vc, V[:, :, L0 + done], pos)
+            oracle.attention_over_compressed(q, kc, vc, pos + 1, 1.0, d)
+            t_total += time.perf_counter() - t0
+            done += 1
+            if t_total >= budget_s:
+                break
+    return {"value": t_total / done * 1e6, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} of the 64 decode steps (append K, append V, attention over all 64 streams), "
+                      f"float64 NumPy, 1 BLAS thread"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    base = oracle_decode_sample(budget_s=min(20.0, 4.0 + 2.0 * args.steps))
+    line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": base["value"] / 1000.0,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(), "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def config_dict():
+    w = WORKLOAD
+    return {"workload": "Llama-3-8B-like GQA decode (q32/kv8/d128), batch 8, context 4096 + 64 decode steps, "
+                        "K/V sparsity 0.7; step = append K + append V + sparse decode attention",
+            "batch": w["batch"], "context": w["context"], "decode_steps": w["decode_steps"],
+            "sparsity_k": w["sparsity_k"], "sparsity_v": w["sparsity_v"],
+            "l2": f"{ROTATE} rotating compressed-cache copies (> 2x the 126 MB L2)", "timing": "CUDA graphs of 64 steps"}
+
+
+# ------------------------------------------------------------------------------------------ main
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64 * 2000)
+    ap.add_argument("--warmup", type=int, default=64 * 20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import unstructured_sparse_kv_b200 as M
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    M.load()
+    wl = Workload(rank_seed(rank), dev)
+    stream = torch.cuda.current_stream()
+
+    # ---- the timed region: K steps (graphs of 64 steps; a tail of K % 64 eager steps)
+    g_step = wl.graph()
+    reps_w = max(1, math.ceil(args.warmup / GRAPH_STEPS))
+    for _ in range(reps_w):
+        g_step.replay()
+    torch.cuda.synchronize()
+    reps, tail = divmod(args.steps, GRAPH_STEPS)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g_step.replay()
+        for i in range(tail):
+            wl.step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    us_per_step = aggregate_us_per_step(elapsed_ms, args.steps, world)
+    clk = clocks.summary()
+
+    # ---- dominant kernel alone (decode attention), same inputs and rotation
+    g_att = wl.graph(attend_only=True)
+    for _ in range(3):
+        g_att.replay()
+    torch.cuda.synchronize()
+    att_reps = max(20, min(400, reps))
+    att_ms = time_graph(g_att, att_reps, stream)
+    att_us = att_ms * 1000.0 / (att_reps * GRAPH_STEPS)
+    lens = [wl.L0 + 1 + i for i in range(wl.steps)]
+    avg_bytes = sum(decode_algorithmic_bytes(wl.B, wl.Hq, wl.Hkv, wl.d, [L] * wl.B, wl.kc[0].keep, wl.vc[0].keep)
+                    for L in lens) / len(lens)
+    peak, peak_kind = measured_peak()
+    achieved = avg_bytes / (att_us * 1e-6) / 1e9
+
+    # ---- dense fp16 baseline on the same context
+    dense = DenseBaseline(wl)
+    g_dense = wl.graph(dense=dense)
+    for _ in range(3):
+        g_dense.replay()
+    torch.cuda.synchronize()
+    dense_reps = max(10, min(200, reps))
+    dense_us = time_graph(g_dense, dense_reps, stream) * 1000.0 / (dense_reps * GRAPH_STEPS)
+
+    # ---- end to end through the public API with host buffers (eager calls)
+    e2e = None
+    if True:  # end-to-end leg
+        qh = wl.q.cpu().pin_memory()
+        knh, vnh = wl.kn.cpu().pin_memory(), wl.vn.cpu().pin_memory()
+        posh = wl.pos.cpu().pin_memory()
+        outh = torch.empty((wl.steps,) + tuple(wl.out.shape), dtype=torch.float16).pin_memory()
+        qd, knd, vnd = torch.empty_like(wl.q[0]), torch.empty_like(wl.kn[0]), torch.empty_like(wl.vn[0])
+        posd = torch.empty_like(wl.pos[0])
+        seqd = torch.empty_like(wl.pos[0])
+        n_e2e = 64 * 10
+
+        def e2e_step(i):
+            j, r = i % wl.steps, i % ROTATE
+            qd.copy_(qh[j], non_blocking=True)
+            knd.copy_(knh[j], non_blocking=True)
+            vnd.copy_(vnh[j], non_blocking=True)
+            posd.copy_(posh[j], non_blocking=True)
+            M.mustafar_append(knd, posd, wl.kc[r])
+            M.mustafar_append(vnd, posd, wl.vc[r])
+            torch.add(posd, 1, out=seqd)
+            M.mustafar_decode_attn(qd, wl.kc[r], wl.vc[r], seqd, wl.cap, 1.0, out=wl.out, lse=wl.lse,
+                                   workspace=wl.ws)
+            outh[j].copy_(wl.out, non_blocking=True)
+
+        for i in range(64):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(n_e2e):
+            e2e_step(i)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1), dev)
+        bi = (wl.q[0].numel() + wl.kn[0].numel() + wl.vn[0].numel()) * 2 + wl.pos[0].numel() * 4
+        e2e = {"value": aggregate_us_per_step(e2e_ms, n_e2e, world), "unit": UNIT, "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": wl.out.numel() * 2, "steps": n_e2e,
+               "how": "eager public-API calls per step: pinned H2D of q/k_new/v_new/pos, 3 library launches "
+                      "(+1 torch add for seq_len), D2H of out"}
+
+    line = {"metric": METRIC, "value": us_per_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": reps_w * GRAPH_STEPS, "ms_per_step": us_per_step / 1000.0, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config_dict(),
+            "gpu_launches": 3 * args.steps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "traffic": recorded_traffic(), "kernel": "decode_kernel (sparse)",
+                         "algorithmic_bytes_per_launch": avg_bytes, "us_per_launch": att_us,
+                         "splits": wl.splits},
+            "dense_baseline": {"us_per_launch": dense_us, "sparse_speedup": dense_us / att_us,
+                               "bytes_per_launch": sum(4 * wl.B * wl.Hkv * L * wl.d for L in lens) / len(lens)
+                               + 4 * wl.B * wl.Hq * wl.d},
+            "compressed_kv_bytes": wl.compressed_bytes,
+            "clocks": clk, "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_decode_sample()
+    if rank == 0:
+        print(json.dumps(line))
+    del g_step, g_att, g_dense
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * mustafar.h - C ABI of the B200 (sm_100a) Mustafar KV-cache library.
+ *
+ * The method (MUSTAFAR summary, atlas.scime.ai, "Approach"; Mustafar abstract,
+ * catalyzex author page): every (token, kv head) vector of the Key and Value
+ * caches is pruned by magnitude to an unstructured sparsity, compressed into a
+ * bitmap-based sparse format, and decode attention is computed directly over
+ * the compressed caches.  New decode tokens are pruned and compressed at run
+ * time.  K and V take separate sparsities ("k_sparsity / v_sparsity",
+ * Mustafar README, Part II).
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Every data pointer is a DEVICE pointer unless marked "host".  The caller
+ *   owns all memory; the library allocates nothing, never synchronises, and
+ *   enqueues its kernels on `stream` (a cudaStream_t; NULL = legacy stream).
+ * - fp16 tensors are passed as raw 16-bit storage (IEEE binary16).
+ * - head_dim must be 128 for the kernels (the format itself needs a multiple of 32).
+ * - Host-side validation failures return an error status and launch nothing.
+ *   A failed launch returns MUSTAFAR_ERR_CUDA.  mustafar_last_error() gives a
+ *   message for the calling thread's last failure.
+ * - Problems only the device can see (a position or length beyond the cache
+ *   capacity) never trap: the kernel skips that row and ORs a bit into the
+ *   optional device word `d_err` (MUSTAFAR_DEVERR_*).
+ *
+ * Compressed format (one "stream" per (batch row b, kv head h); s = b*H + h)
+ * ---------------------------------------------------------------------------
+ *   keep k   = head_dim - floor(sparsity * head_dim), sparsity rounded to float
+ *              and the product formed in double; 1 <= k <= head_dim.
+ *   selection: the k channels with the largest magnitude key (fp16 bits & 0x7FFF);
+ *              on equal keys the lower channel index wins.
+ *   bitmap   : uint32 [streams][capacity][head_dim/32]; channel c of token t is
+ *              kept iff bit (c % 32) of word (c / 32) is set.  Always popcount k.
+ *   values   : fp16 bits [streams][capacity * k]; token t's k kept values, in
+ *              ascending channel order, start at element t*k of its stream.
+ *   tile_offset: uint32 [streams][capacity/64]; element offset of the first value
+ *              of each 64-token tile (the popcount prefix sum, = 64*i*k).
+ *   Pruned positions read back as +0.  Bytes per stream:
+ *              16*L + 2*k*L + 4*capacity/64 for L stored tokens (head_dim 128).
+ */
+#ifndef MUSTAFAR_H_
+#define MUSTAFAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MUSTAFAR_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MUSTAFAR_API __attribute__((visibility("default")))
+#else
+#define MUSTAFAR_API
+#endif
+
+typedef struct CUstream_st *mustafar_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MUSTAFAR_OK = 0,
+  MUSTAFAR_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad sparsity, keep mismatch   */
+  MUSTAFAR_ERR_UNSUPPORTED = 2, /* valid for the format but not for these kernels (d!=128) */
+  MUSTAFAR_ERR_MISALIGNED = 3,  /* a pointer or stride breaks the 16-byte rule            */
+  MUSTAFAR_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed            */
+  MUSTAFAR_ERR_WORKSPACE = 5    /* workspace missing or smaller than the query returned   */
+} mustafar_status;
+
+/* device-side error bits ORed into *d_err (never a trap) */
+#define MUSTAFAR_DEVERR_POS_RANGE 0x1u /* append: pos[b] < 0 or >= capacity; row skipped     */
+#define MUSTAFAR_DEVERR_LEN_RANGE 0x2u /* decode: seq_len[b] < 0 or > capacity; row clamped  */
+
+/* One compressed cache (K or V).  The three arrays are caller-owned device
+ * memory sized by mustafar_cache_sizes(); bitmap and values 16-byte aligned,
+ * tile_offset 4-byte aligned.  capacity is a multiple of 64. */
+typedef struct {
+  int32_t batch;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t capacity;
+  int32_t keep; /* = mustafar_keep_count(head_dim, sparsity) */
+  uint32_t *bitmap;
+  uint16_t *values;
+  uint32_t *tile_offset;
+} mustafar_cache_t;
+
+/* Keep count for a pruning sparsity s (fraction of channels removed, README
+ * Part II: "50% sparsity is 0.5").  Returns head_dim - floor(s*head_dim), or -1
+ * when head_dim <= 0, head_dim % 32 != 0 or s is outside [0, 1). */
+MUSTAFAR_API int32_t mustafar_keep_count(int32_t head_dim, float sparsity);
+
+/* Bytes of the three arrays of one cache (host outputs, any may be NULL). */
+MUSTAFAR_API mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t capacity, float sparsity, size_t *bitmap_bytes,
+                                     size_t *values_bytes, size_t *offset_bytes);
+
+/* Prune + compress (prefill).  Per-token magnitude pruning followed by the
+ * bitmap compression (MUSTAFAR summary, "Approach"; Mustafar abstract).
+ *   x        : fp16 dense cache; element (b, h, t, c) at
+ *              x[b*stride_b + h*stride_h + t*stride_t + c] (strides in elements,
+ *              channels contiguous; x and every stride a multiple of 8 elements).
+ *   L        : tokens [0, L) are compressed into slots [0, L); 0 <= L <= capacity.
+ *   sparsity : must satisfy c->keep == mustafar_keep_count(c->head_dim, sparsity).
+ *   c        : the destination cache; its whole tile_offset array is written.
+ *   d_err    : optional device word (unused by this call today; may be NULL).
+ * Slots >= L are not touched.  Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */
+MUSTAFAR_API mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t stride_h,
+                                  int64_t stride_t, int32_t L, float sparsity,
+                                  const mustafar_cache_t *c, uint32_t *d_err,
+                                  mustafar_stream_t stream);
+
+/* Append: prune + compress one new decode token per (b, kv head) into slot
+ * pos[b] (the runtime compression the abstract describes).
+ *   x     : fp16 [batch][num_kv_heads][head_dim] with element (b, h, c) at
+ *           x[b*stride_b + h*stride_h + c] (x and strides multiples of 8 elements).
+ *   d_pos : int32 [batch] device array of slots; a slot outside [0, capacity)
+ *           skips that row and sets MUSTAFAR_DEVERR_POS_RANGE in *d_err.
+ * The caller advances its lengths (e.g. seq_len = pos + 1) itself; the library
+ * keeps no state.  Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */
+MUSTAFAR_API mustafar_status mustafar_append(const void *x, int64_t stride_b, int64_t stride_h,
+                                const int32_t *d_pos, const mustafar_cache_t *c, uint32_t *d_err,
+                                mustafar_stream_t stream);
+
+/* Workspace bytes for mustafar_decode_attn / mustafar_dense_decode_attn with
+ * these shapes.  num_splits = 0 asks for the automatic split plan; a positive
+ * value forces that many context splits (clamped to the number of 16-token chunks).
+ * The workspace holds per-split partial softmax states and one ticket counter per
+ * (b, kv head).  It must be zero-filled once when allocated; every completed call
+ * leaves the counters at zero again.  Calls that share a workspace must not overlap. */
+MUSTAFAR_API mustafar_status mustafar_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
+                                                int32_t num_kv_heads, int32_t head_dim,
+                                                int32_t max_len, int32_t num_splits,
+                                                size_t *bytes);
+
+/* Sparse decode attention over the compressed caches (Mustafar abstract: a
+ * custom attention kernel "directly computing over compressed caches").
+ * For q head hq (kv head g = hq / (Hq/Hkv)) of batch row b:
+ *   z_t = scale * q[b,hq] . K~[b,g,t]   for t < seq_len[b]
+ *   out[b,hq] = sum_t softmax(z)_t V~[b,g,t]          (fp16, fp32 accumulation)
+ *   lse[b,hq] = log sum_t exp(z_t)                    (fp32, natural log; optional)
+ *   q, out    : fp16 [batch][num_q_heads][head_dim], 16-byte aligned.
+ *   k, v      : compressed caches with equal batch, num_kv_heads, head_dim; their
+ *               keep counts (sparsities) may differ.
+ *   d_seq_len : int32 [batch]; each in [1, capacity] (longer rows are clamped
+ *               and flagged in d_err; 0 gives out = 0 and lse = -inf).
+ *   max_len   : host upper bound on seq_len, sizes the split plan.
+ *   workspace : see mustafar_decode_workspace_bytes (same max_len and num_splits).
+ *   d_err     : optional device error word.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
+MUSTAFAR_API mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_heads, const mustafar_cache_t *k,
+                                     const mustafar_cache_t *v, const int32_t *d_seq_len,
+                                     int32_t max_len, float scale, void *out, float *lse,
+                                     void *workspace, size_t workspace_bytes, int32_t num_splits,
+                                     uint32_t *d_err, mustafar_stream_t stream);
+
+/* Dense fp16 decode attention over uncompressed caches, the baseline the pages
+ * compare against ("FlashAttention", "cuBLAS dense": MUSTAFAR summary,
+ * "Experimental setup").  Same math and kernel skeleton as mustafar_decode_attn.
+ *   k_dense, v_dense : fp16 [batch][num_kv_heads][capacity][head_dim], 16-byte aligned.
+ * Other arguments as in mustafar_decode_attn. */
+MUSTAFAR_API mustafar_status mustafar_dense_decode_attn(const void *q, int32_t num_q_heads, const void *k_dense,
+                                           const void *v_dense, int32_t batch, int32_t num_kv_heads,
+                                           int32_t head_dim, int32_t capacity,
+                                           const int32_t *d_seq_len, int32_t max_len, float scale,
+                                           void *out, float *lse, void *workspace,
+                                           size_t workspace_bytes, int32_t num_splits,
+                                           uint32_t *d_err, mustafar_stream_t stream);
+
+/* The split count the automatic plan would use for this call (host query, for
+ * benchmarks and tests).  Returns a value >= 1, or -1 on invalid shapes. */
+MUSTAFAR_API int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t max_len, int32_t keep_k, int32_t keep_v, int32_t dense);
+
+MUSTAFAR_API const char *mustafar_status_string(mustafar_status s);
+MUSTAFAR_API const char *mustafar_last_error(void);
+MUSTAFAR_API int32_t mustafar_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUSTAFAR_H_ */

@@ -1,0 +1,125 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, and its
+host-side queries and argument checks behave (no kernel launch, no GPU needed)."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import unstructured_sparse_kv_b200 as M
+from unstructured_sparse_kv_b200 import _lib
+from unstructured_sparse_kv_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return M.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "mustafar.h")).read()
+    return sorted(set(re.findall(r"MUSTAFAR_API[^;(]*?\b(mustafar_\w+)\s*\(", text, flags=re.S)))
+
+
+def test_header_lists_the_binding_symbols():
+    assert declared_symbols() == sorted(_lib.ABI_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.mustafar_abi_version() == 1
+
+
+def test_keep_count_matches_oracle(lib):
+    for d in (32, 64, 128, 256):
+        for s in np.concatenate([np.linspace(0, 0.999, 97), [0.1, 0.3, 0.7, 0.9, 0.995]]):
+            assert M.mustafar_keep_count(d, float(s)) == oracle.keep_count(d, float(s)), (d, s)
+    for bad in (-0.01, 1.0, 2.0, float("nan")):
+        assert lib.mustafar_keep_count(128, bad) == -1
+    assert lib.mustafar_keep_count(100, 0.5) == -1
+
+
+def test_cache_sizes_match_closed_form(lib):
+    for (Bt, H, cap, s) in [(8, 8, 4160, 0.7), (1, 8, 1024, 0.5), (4, 8, 32768, 0.3), (32, 32, 131072, 0.0)]:
+        nb, nv, no = M.mustafar_cache_sizes(Bt, H, 128, cap, s)
+        k = oracle.keep_count(128, s)
+        per_stream = oracle.compressed_bytes(cap, k, cap, 128)
+        assert nb + nv + no == Bt * H * per_stream
+        assert nb == Bt * H * cap * 16 and no == Bt * H * (cap // 64) * 4
+    with pytest.raises(M.MustafarError):
+        M.mustafar_cache_sizes(1, 1, 128, 100, 0.5)  # capacity not a multiple of 64
+
+
+def _cache(batch=2, heads=2, cap=128, keep=39, bitmap=0x1000, values=0x2000, offs=0x3000, d=128):
+    return _lib.CacheT(batch, heads, d, cap, keep, bitmap, values, offs)
+
+
+def _status(lib, fn, *args):
+    st = getattr(lib, fn)(*args)
+    return st, lib.mustafar_last_error().decode()
+
+
+def test_compress_argument_checks(lib):
+    ok = _cache()
+    cases = [
+        (dict(c=None), 1, "NULL"),
+        (dict(c=_cache(keep=40)), 1, "keep"),
+        (dict(c=_cache(cap=100)), 1, "multiple of 64"),
+        (dict(c=_cache(d=64, keep=20)), 2, "128"),
+        (dict(c=_cache(bitmap=0x1004)), 3, "alignment"),
+        (dict(L=129), 1, "capacity"),
+        (dict(s=1.0), 1, "sparsity"),
+        (dict(x=0x5002), 3, "multiples of 8"),
+        (dict(st=12), 3, "multiples of 8"),
+        (dict(x=None), 1, "NULL"),
+    ]
+    for over, want, msg in cases:
+        a = dict(x=0x5000, sb=4096, sh=2048, st=128, L=64, s=0.7, c=ok)
+        a.update(over)
+        cref = C.byref(a["c"]) if a["c"] is not None else None
+        st, err = _status(lib, "mustafar_compress", a["x"], a["sb"], a["sh"], a["st"], a["L"], a["s"], cref, None, None)
+        assert st == want and msg in err, (over, st, err)
+
+
+def test_append_and_decode_argument_checks(lib):
+    c = _cache()
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 128, None, C.byref(c), None, None)
+    assert st == 1 and "pos" in err
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(c), None, None)
+    assert st == 3
+    kc, vc = _cache(), _cache(heads=4)
+    st, err = _status(lib, "mustafar_decode_attn", 0x7000, 8, C.byref(kc), C.byref(vc), 0x6000, 64, 1.0, 0x8000,
+                      None, None, 0, 0, None, None)
+    assert st == 1 and "disagree" in err
+    vc = _cache()
+    st, err = _status(lib, "mustafar_decode_attn", 0x7000, 5, C.byref(kc), C.byref(vc), 0x6000, 64, 1.0, 0x8000,
+                      None, None, 0, 0, None, None)
+    assert st == 1 and "multiple" in err
+    st, err = _status(lib, "mustafar_decode_attn", 0x7000, 2 * 17, C.byref(kc), C.byref(vc), 0x6000, 64, 1.0,
+                      0x8000, None, None, 0, 0, None, None)
+    assert st == 2 and "16" in err
+    st, err = _status(lib, "mustafar_decode_attn", 0x7008, 8, C.byref(kc), C.byref(vc), 0x6000, 64, 1.0, 0x8000,
+                      None, None, 0, 0, None, None)
+    assert st == 3
+    st, err = _status(lib, "mustafar_decode_attn", 0x7000, 8, C.byref(kc), C.byref(vc), 0x6000, 64,
+                      float("inf"), 0x8000, None, None, 0, 0, None, None)
+    assert st == 1 and "scale" in err
+    st, err = _status(lib, "mustafar_dense_decode_attn", 0x7000, 8, 0x9000, 0xA000, 2, 2, 128, 100, 0x6000, 64,
+                      1.0, 0x8000, None, None, 0, 0, None, None)
+    assert st == 1 and "16" in err
+
+
+def test_workspace_query(lib):
+    n1 = M.mustafar_decode_workspace_bytes(8, 32, 8, 4160, num_splits=1)
+    n4 = M.mustafar_decode_workspace_bytes(8, 32, 8, 4160, num_splits=4)
+    assert n1 == 256
+    assert n4 >= 8 * 32 * 4 * (128 + 2) * 4 + 8 * 8 * 4
+    assert M.mustafar_decode_workspace_bytes(8, 32, 8, 4160) >= n1
+    with pytest.raises(M.MustafarError):
+        M.mustafar_decode_workspace_bytes(8, 30, 8, 4160)

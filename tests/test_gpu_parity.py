@@ -1,0 +1,269 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Compressed caches (bitmap, packed values, tile offsets) must be bit-exact; attention
+outputs within max-abs 2e-3 and relative L2 1e-3 of the float64 oracle, lse within 1e-3.
+Sizes span several 16-token chunks and 64-token tiles with ragged tails; the workload
+shapes (batch 1..32, context up to 128k, MHA and GQA, sparsity 0..0.9) are checked at
+full size, with the oracle run on sampled (batch, kv head) streams where the full
+tensor would take it too long.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import unstructured_sparse_kv_b200 as M
+from tests import gpu_util as U
+from unstructured_sparse_kv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+D = 128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    M.load()
+
+
+def _setup(B, Hq, Hkv, L, cap, sK, sV, seed, seq=None):
+    K = synth.keys(B, Hkv, L, D, seed, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L, D, seed, DEV, capacity=cap)
+    q = synth.queries(B, Hq, D, seed, DEV)
+    kc = M.CompressedCache(B, Hkv, cap, sK)
+    vc = M.CompressedCache(B, Hkv, cap, sV)
+    M.mustafar_compress(K, L, sK, kc)
+    M.mustafar_compress(V, L, sV, vc)
+    seq = torch.full((B,), L, dtype=torch.int32) if seq is None else seq
+    return K, V, q, kc, vc, seq
+
+
+def _attend(q, kc, vc, seq, max_len, scale=1.0, splits=0):
+    return M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), max_len, scale, num_splits=splits)
+
+
+# ------------------------------------------------------------------------------------ compress / append
+TIE_ROWS = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x03FF, 0x3C00, 0xBC00, 0x4000, 0xC000, 0x7BFF, 0xFBFF],
+                    dtype=np.uint16)
+
+
+@pytest.mark.parametrize("s", [0.0, 0.1, 0.3, 0.5, 0.7, 0.9, 0.995])
+def test_compress_bit_exact_strided_with_ties(s):
+    B, H, L, cap = 2, 3, 200, 256
+    rng = np.random.default_rng(5)
+    x = synth.keys(B, H, L, D, 42, "cpu").permute(0, 2, 1, 3).contiguous()  # [B, L, H, d] storage
+    xb = x.view(torch.int16).numpy().view(np.uint16).copy()
+    xb[0, 3, 1] = rng.choice(TIE_ROWS, D)
+    xb[1, 77, 2] = 0x3C00                      # all equal
+    xb[1, 78, 0] = 0                           # all +0
+    xb[0, 150, 0, :64] = 0x8000                # -0 and ties with +0
+    xb[0, 151, 1, 5] = 0x7C00                  # +inf / NaN patterns rank by bits
+    xb[0, 151, 1, 9] = 0x7E00
+    xdev = torch.from_numpy(xb.view(np.int16)).view(torch.float16).to(DEV)
+    view = xdev.permute(0, 2, 1, 3)            # [B, H, L, d] strided view
+    c = M.CompressedCache(B, H, cap, s)
+    M.mustafar_compress(view, L, s, c)
+    U.assert_cache_matches(c, np.ascontiguousarray(xb.transpose(0, 2, 1, 3)), L)
+
+
+def test_compress_leaves_slots_beyond_L_untouched():
+    B, H, L, cap = 1, 2, 100, 192
+    x = synth.values(B, H, cap, D, 3, DEV)
+    c = M.CompressedCache(B, H, cap, 0.7)
+    c.bitmap.fill_(-1)
+    c.values.fill_(0x1234)
+    M.mustafar_compress(x, L, 0.7, c)
+    bm, vals, _ = U.cache_np(c)
+    assert (bm[:, :, L:] == 0xFFFFFFFF).all() and (vals[:, :, L * c.keep:] == 0x1234).all()
+    U.assert_cache_matches(c, U.bits(x), L)
+
+
+def test_compress_empty_writes_offsets_only():
+    c = M.CompressedCache(2, 2, 128, 0.5)
+    c.tile_offset.fill_(-1)
+    x = torch.zeros(2, 2, 128, D, dtype=torch.float16, device=DEV)
+    M.mustafar_compress(x, 0, 0.5, c)
+    _, _, offs = U.cache_np(c)
+    assert (offs == np.array([0, 64 * 64], dtype=np.uint32)).all()
+    assert int(c.bitmap.abs().sum()) == 0
+
+
+def test_append_across_tile_boundaries_matches_oracle():
+    B, H, cap, k_s = 3, 2, 256, 0.7
+    L0 = 60
+    full = synth.keys(B, H, 140, D, 9, DEV, capacity=cap)
+    c = M.CompressedCache(B, H, cap, k_s)
+    M.mustafar_compress(full, L0, k_s, c)
+    for t in range(L0, 140):
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        M.mustafar_append(full[:, :, t], pos, c)  # strided [B, H, d] slice
+    U.assert_cache_matches(c, U.bits(full), 140)
+
+
+def test_append_rows_at_different_positions_and_out_of_range():
+    B, H, cap = 4, 2, 128
+    c = M.CompressedCache(B, H, cap, 0.5)
+    x = synth.step_tokens(B, H, D, 11, 0, DEV)[0]
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pos = torch.tensor([0, 63, 64, cap], dtype=torch.int32, device=DEV)  # the last row is out of range
+    M.mustafar_append(x, pos, c, err=err)
+    assert int(err.item()) & M.DEVERR_POS_RANGE
+    bm, vals, _ = U.cache_np(c)
+    xb = U.bits(x)
+    k = c.keep
+    for b, p in enumerate([0, 63, 64]):
+        ref = oracle.compress(xb[b][:, None, :], k, 64)
+        assert np.array_equal(bm[b, :, p], ref["bitmap"][:, 0, 0])
+        assert np.array_equal(vals[b, :, p * k:(p + 1) * k], ref["values"][:, 0, :k])
+    assert (bm[3] == 0).all() and (vals[3] == 0).all()
+
+
+# ------------------------------------------------------------------------------------ decode attention
+@pytest.mark.parametrize("B,Hq,Hkv,L,sK,sV,splits,ragged", [
+    (2, 8, 2, 200, 0.7, 0.7, 0, True),
+    (2, 8, 2, 200, 0.7, 0.5, 3, True),
+    (3, 4, 4, 77, 0.5, 0.9, 1, True),      # MHA (G = 1)
+    (1, 32, 2, 300, 0.3, 0.7, 0, False),   # G = 16
+    (2, 8, 1, 1, 0.7, 0.7, 0, False),      # one token
+    (2, 12, 4, 129, 0.0, 0.0, 2, True),    # sparsity 0: plain attention
+    (1, 8, 8, 1000, 0.995, 0.995, 0, False),  # keep = 1
+])
+def test_decode_small_cases(B, Hq, Hkv, L, sK, sV, splits, ragged):
+    cap = ((L + 63) // 64) * 64
+    seq = synth.seq_lens(B, L, ragged, 1)
+    K, V, q, kc, vc, seq = _setup(B, Hq, Hkv, L, cap, sK, sV, 100 + B + L, seq)
+    scale = 1.0 / math.sqrt(D) if sK == 0 else 1.0
+    out, lse = _attend(q, kc, vc, seq, L, scale, splits)
+    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, seq.numpy(), scale)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"B{B} Hq{Hq} Hkv{Hkv} L{L}")
+
+
+def test_split_count_invariance():
+    B, Hq, Hkv, L = 2, 32, 8, 2000
+    K, V, q, kc, vc, seq = _setup(B, Hq, Hkv, L, 2048, 0.7, 0.7, 7)
+    outs = [_attend(q, kc, vc, seq, L, 1.0, s) for s in (1, 2, 5, 31, 0)]
+    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, seq.numpy(), 1.0)
+    for o, l in outs:
+        U.assert_attn_close(o, o_ref, l, l_ref, tag="splits")
+        assert float((o.float() - outs[0][0].float()).abs().max()) <= 2e-3
+
+
+def test_seq_len_zero_and_beyond_capacity():
+    B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 21)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    seq = torch.tensor([0, 64, 500], dtype=torch.int32, device=DEV)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq, 500, 1.0, err=err)
+    assert int(err.item()) & M.DEVERR_LEN_RANGE
+    assert float(out[0].abs().max()) == 0.0 and torch.isinf(lse[0]).all() and (lse[0] < 0).all()
+    o_ref, l_ref = U.oracle_attention(q[1:], U.bits(K)[1:], U.bits(V)[1:], kc.keep, vc.keep, [64, 64], 1.0)
+    U.assert_attn_close(out[1:], o_ref, lse[1:], l_ref, tag="clamped")
+
+
+def test_dense_baseline_matches_oracle_and_sdpa():
+    B, Hq, Hkv, L, cap = 2, 32, 8, 700, 704
+    K = synth.keys(B, Hkv, L, D, 5, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L, D, 5, DEV, capacity=cap)
+    q = synth.queries(B, Hq, D, 5, DEV)
+    seq = torch.tensor([L, 333], dtype=torch.int32)
+    for splits in (1, 0):
+        out, lse = M.mustafar_dense_decode_attn(q, K, V, seq.to(DEV), L, 1.0, num_splits=splits)
+        o_ref, l_ref = oracle.attention(U.bits(q), U.bits(K), U.bits(V), seq.numpy(), 1.0)
+        U.assert_attn_close(out, o_ref, lse, l_ref, tag="dense")
+    Kr = K[:1, :, :L].repeat_interleave(Hq // Hkv, dim=1).float()
+    Vr = V[:1, :, :L].repeat_interleave(Hq // Hkv, dim=1).float()
+    sd = torch.nn.functional.scaled_dot_product_attention(q[:1, :, None].float(), Kr, Vr, scale=1.0)[:, :, 0]
+    assert float((sd - out[:1].float()).abs().max()) < 2e-3
+
+
+# ------------------------------------------------------------------------------------ the workload shapes
+def test_llama3_gqa_b1_ctx1024_s05():
+    B, Hq, Hkv, L = 1, 32, 8, 1024
+    K, V, q, kc, vc, seq = _setup(B, Hq, Hkv, L, L, 0.5, 0.5, 1001)
+    U.assert_cache_matches(kc, U.bits(K), L)
+    U.assert_cache_matches(vc, U.bits(V), L)
+    out, lse = _attend(q, kc, vc, seq, L)
+    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, seq.numpy(), 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag="b1 ctx1024")
+
+
+def test_llama3_gqa_b8_ctx4096_s07_64_decode_steps():
+    B, Hq, Hkv, L0, steps = 8, 32, 8, 4096, 64
+    cap = L0 + steps
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L0, cap, 0.7, 0.7, 1002)
+    saved = {}
+    for st in range(steps):
+        kn, vn = synth.step_tokens(B, Hkv, D, 1002, st, DEV)
+        K[:, :, L0 + st] = kn
+        V[:, :, L0 + st] = vn
+        pos = torch.full((B,), L0 + st, dtype=torch.int32, device=DEV)
+        M.mustafar_append(kn, pos, kc)
+        M.mustafar_append(vn, pos, vc)
+        qs = synth.queries(B, Hq, D, 1002, DEV, step=st)
+        out, lse = M.mustafar_decode_attn(qs, kc, vc, pos + 1, cap, 1.0)
+        if st in (0, 1, 31, 63):
+            saved[st] = (qs.clone(), out.clone(), lse.clone())
+    Kb, Vb = U.bits(K), U.bits(V)
+    U.assert_cache_matches(kc, Kb, cap)
+    U.assert_cache_matches(vc, Vb, cap)
+    kp, vp = oracle.prune(Kb, kc.keep), oracle.prune(Vb, vc.keep)
+    for st, (qs, out, lse) in saved.items():
+        o_ref, l_ref = oracle.attention(U.bits(qs), kp, vp, [L0 + st + 1] * B, 1.0)
+        U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"decode step {st}")
+
+
+def test_mistral_gqa_b4_ctx32k_sk07_sv05():
+    B, Hq, Hkv, L = 4, 32, 8, 32768
+    K, V, q, kc, vc, seq = _setup(B, Hq, Hkv, L, L, 0.7, 0.5, 1003)
+    streams = [(0, 0), (1, 3), (2, 7), (3, 5)]
+    Kb, Vb = U.bits(K), U.bits(V)
+    U.assert_cache_matches(kc, np.stack([Kb[b, h] for b, h in streams]), L, streams)
+    U.assert_cache_matches(vc, np.stack([Vb[b, h] for b, h in streams]), L, streams)
+    out, lse = _attend(q, kc, vc, seq, L)
+    o_ref, l_ref = U.oracle_attention(q, Kb, Vb, kc.keep, vc.keep, seq.numpy(), 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag="b4 ctx32k")
+
+
+@pytest.mark.parametrize("s", [0.3, 0.5, 0.7])
+def test_prefill_compress_b8_16k_h8(s):
+    B, L, H = 8, 16384, 8
+    g = torch.Generator(device=DEV)
+    g.manual_seed(1004)
+    x = torch.randn(B, L, H, D, generator=g, device=DEV).to(torch.float16)  # [B, L, H, d] storage
+    c = M.CompressedCache(B, H, L, s)
+    M.mustafar_compress(x.permute(0, 2, 1, 3), L, s, c)
+    streams = [(0, 0), (3, 4), (7, 7)]
+    xb = U.bits(x)
+    U.assert_cache_matches(c, np.stack([xb[b, :, h] for b, h in streams]), L, streams)
+    assert c.nbytes() == B * H * oracle.compressed_bytes(L, c.keep, L, D)
+
+
+SWEEP_POINTS = [  # (Hq, Hkv, B, L, s)
+    (32, 8, 1, 4096, 0.0), (32, 32, 8, 4096, 0.3), (32, 8, 32, 4096, 0.5), (32, 32, 1, 32768, 0.7),
+    (32, 8, 8, 32768, 0.9), (32, 32, 1, 131072, 0.5), (32, 8, 32, 131072, 0.7), (32, 32, 32, 131072, 0.7),
+]
+
+
+@pytest.mark.parametrize("Hq,Hkv,B,L,s", SWEEP_POINTS)
+def test_sweep_points_sampled(Hq, Hkv, B, L, s):
+    """Full-size sweep points; the oracle checks sampled (b, kv head) streams and their q heads."""
+    K, V, q, kc, vc, seq = _setup(B, Hq, Hkv, L, L, s, s, 2000 + B + Hkv + int(10 * s))
+    out, lse = _attend(q, kc, vc, seq, L)
+    dense, _ = M.mustafar_dense_decode_attn(q, K, V, seq.to(DEV), L, 1.0)
+    rng = np.random.default_rng(B * L)
+    picks = sorted({(0, 0), (B - 1, Hkv - 1)} | {(int(rng.integers(B)), int(rng.integers(Hkv))) for _ in range(2)})
+    G = Hq // Hkv
+    for b, h in picks:
+        Kb, Vb = U.bits(K[b, h]), U.bits(V[b, h])
+        U.assert_cache_matches(kc, Kb[None], L, [(b, h)])
+        U.assert_cache_matches(vc, Vb[None], L, [(b, h)])
+        qb = U.bits(q[b:b + 1, h * G:(h + 1) * G])
+        o_ref, l_ref = U.oracle_attention(qb, Kb[None, None], Vb[None, None], kc.keep, vc.keep, [L], 1.0)
+        U.assert_attn_close(out[b:b + 1, h * G:(h + 1) * G], o_ref, lse[b:b + 1, h * G:(h + 1) * G], l_ref,
+                            tag=f"sweep b{b} h{h}")
+        d_ref, _ = oracle.attention(qb, Kb[None, None], Vb[None, None], [L], 1.0)
+        U.assert_attn_close(dense[b:b + 1, h * G:(h + 1) * G], d_ref, tag=f"dense b{b} h{h}")
+    del K, V, kc, vc
+    torch.cuda.empty_cache()

@@ -1,0 +1,223 @@
+"""ctypes binding of libmustafar.so: argument marshalling only.
+
+Every step of the path runs inside the library's CUDA kernels; these wrappers
+turn torch tensors into pointers, shapes and a stream handle, call the C entry
+point of the same name, and raise on a non-OK status.  There is no fallback:
+if the library is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmustafar.so")
+
+MUSTAFAR_OK = 0
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4: "CUDA", 5: "WORKSPACE"}
+DEVERR_POS_RANGE = 0x1
+DEVERR_LEN_RANGE = 0x2
+HEAD_DIM = 128
+
+# every symbol include/mustafar.h declares
+ABI_SYMBOLS = (
+    "mustafar_keep_count", "mustafar_cache_sizes", "mustafar_compress", "mustafar_append",
+    "mustafar_decode_workspace_bytes", "mustafar_decode_attn", "mustafar_dense_decode_attn",
+    "mustafar_decode_plan_splits", "mustafar_status_string", "mustafar_last_error", "mustafar_abi_version",
+)
+
+
+class MustafarError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class CacheT(C.Structure):
+    """Mirror of mustafar_cache_t."""
+    _fields_ = [("batch", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
+                ("capacity", C.c_int32), ("keep", C.c_int32), ("bitmap", C.c_void_p),
+                ("values", C.c_void_p), ("tile_offset", C.c_void_p)]
+
+
+_lib = None
+
+
+def load() -> C.CDLL:
+    """Load libmustafar.so (built in-tree by ``unstructured_sparse_kv_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libmustafar.so is not built ({LIB_PATH}); run `python -m unstructured_sparse_kv_b200.build`")
+    lib = C.CDLL(LIB_PATH)
+    i32, i64, f32, vp, sz = C.c_int32, C.c_int64, C.c_float, C.c_void_p, C.c_size_t
+    P = C.POINTER
+    sig = {
+        "mustafar_keep_count": (i32, [i32, f32]),
+        "mustafar_cache_sizes": (i32, [i32, i32, i32, i32, f32, P(sz), P(sz), P(sz)]),
+        "mustafar_compress": (i32, [vp, i64, i64, i64, i32, f32, P(CacheT), vp, vp]),
+        "mustafar_append": (i32, [vp, i64, i64, vp, P(CacheT), vp, vp]),
+        "mustafar_decode_workspace_bytes": (i32, [i32, i32, i32, i32, i32, i32, P(sz)]),
+        "mustafar_decode_attn": (i32, [vp, i32, P(CacheT), P(CacheT), vp, i32, f32, vp, vp, vp, sz, i32, vp, vp]),
+        "mustafar_dense_decode_attn": (i32, [vp, i32, vp, vp, i32, i32, i32, i32, vp, i32, f32, vp, vp, vp, sz,
+                                             i32, vp, vp]),
+        "mustafar_decode_plan_splits": (i32, [i32, i32, i32, i32, i32, i32, i32]),
+        "mustafar_status_string": (C.c_char_p, [i32]),
+        "mustafar_last_error": (C.c_char_p, []),
+        "mustafar_abi_version": (i32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != MUSTAFAR_OK:
+        raise MustafarError(status, load().mustafar_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _cuda_f16(t: torch.Tensor, name: str):
+    if not (t.is_cuda and t.dtype == torch.float16):
+        raise TypeError(f"{name} must be a CUDA float16 tensor")
+
+
+# ------------------------------------------------------------------------------------------- queries
+def mustafar_keep_count(head_dim: int, sparsity: float) -> int:
+    k = load().mustafar_keep_count(head_dim, sparsity)
+    if k < 0:
+        raise ValueError("head_dim must be a positive multiple of 32 and sparsity in [0, 1)")
+    return k
+
+
+def mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity):
+    a, b, c = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    _check(load().mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity,
+                                       C.byref(a), C.byref(b), C.byref(c)))
+    return a.value, b.value, c.value
+
+
+def mustafar_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, max_len, num_splits=0, head_dim=HEAD_DIM):
+    n = C.c_size_t()
+    _check(load().mustafar_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_len,
+                                                  num_splits, C.byref(n)))
+    return n.value
+
+
+def mustafar_decode_plan_splits(batch, num_kv_heads, max_len, keep_k, keep_v, dense=False, head_dim=HEAD_DIM):
+    s = load().mustafar_decode_plan_splits(batch, num_kv_heads, head_dim, max_len, keep_k, keep_v, int(dense))
+    if s < 1:
+        raise MustafarError(1, "invalid shapes for the split plan")
+    return s
+
+
+# ------------------------------------------------------------------------------------------- caches
+class CompressedCache:
+    """Caller-owned device arrays of one compressed cache (K or V) plus its C descriptor."""
+
+    def __init__(self, batch: int, num_kv_heads: int, capacity: int, sparsity: float, head_dim: int = HEAD_DIM,
+                 device="cuda"):
+        self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
+        self.sparsity = float(sparsity)
+        self.keep = mustafar_keep_count(head_dim, sparsity)
+        nb, nv, no = mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity)
+        self.bitmap = torch.zeros(nb // 4, dtype=torch.int32, device=device)
+        self.values = torch.zeros(nv // 2, dtype=torch.int16, device=device)
+        self.tile_offset = torch.zeros(no // 4, dtype=torch.int32, device=device)
+        self._struct = CacheT(batch, num_kv_heads, head_dim, capacity, self.keep, self.bitmap.data_ptr(),
+                              self.values.data_ptr(), self.tile_offset.data_ptr())
+
+    @property
+    def struct(self) -> CacheT:
+        return self._struct
+
+    def nbytes(self) -> int:
+        return self.bitmap.numel() * 4 + self.values.numel() * 2 + self.tile_offset.numel() * 4
+
+    def views(self):
+        """(bitmap [B,H,cap,d/32] int32, values [B,H,cap*k] int16, tile_offset [B,H,cap/64] int32)."""
+        B, H, cap, d = self.batch, self.num_kv_heads, self.capacity, self.head_dim
+        return (self.bitmap.view(B, H, cap, d // 32), self.values.view(B, H, cap * self.keep),
+                self.tile_offset.view(B, H, cap // 64))
+
+
+# ------------------------------------------------------------------------------------------- calls
+def mustafar_compress(x: torch.Tensor, L: int, sparsity: float, cache: CompressedCache, err=None, stream=None):
+    """Prune + compress tokens [0, L) of ``x`` ([B, H, T, d] fp16, d contiguous) into ``cache``."""
+    _cuda_f16(x, "x")
+    if x.dim() != 4 or x.stride(3) != 1:
+        raise ValueError("x must be [B, H, T, d] with contiguous channels")
+    if tuple(x.shape[:2]) != (cache.batch, cache.num_kv_heads) or x.shape[3] != cache.head_dim or x.shape[2] < L:
+        raise ValueError("x shape does not match the cache")
+    _check(load().mustafar_compress(_ptr(x), x.stride(0), x.stride(1), x.stride(2), L, sparsity,
+                                    C.byref(cache.struct), _ptr(err), _stream(stream)))
+
+
+def mustafar_append(x: torch.Tensor, pos: torch.Tensor, cache: CompressedCache, err=None, stream=None):
+    """Prune + compress one token per (b, kv head) (``x`` [B, H, d] fp16) into slot ``pos[b]``."""
+    _cuda_f16(x, "x")
+    if x.dim() != 3 or x.stride(2) != 1 or tuple(x.shape) != (cache.batch, cache.num_kv_heads, cache.head_dim):
+        raise ValueError("x must be [B, H, d] with contiguous channels, matching the cache")
+    if not (pos.is_cuda and pos.dtype == torch.int32 and pos.numel() == cache.batch):
+        raise ValueError("pos must be a CUDA int32 tensor of length batch")
+    _check(load().mustafar_append(_ptr(x), x.stride(0), x.stride(1), _ptr(pos), C.byref(cache.struct), _ptr(err),
+                                  _stream(stream)))
+
+
+def _decode_outputs(q, out, lse, want_lse):
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def mustafar_decode_attn(q: torch.Tensor, k: CompressedCache, v: CompressedCache, seq_len: torch.Tensor,
+                         max_len: int, scale: float, out=None, lse=None, workspace=None, num_splits: int = 0,
+                         err=None, stream=None, want_lse: bool = True):
+    """Sparse decode attention over compressed caches; returns (out [B,Hq,d] fp16, lse [B,Hq] fp32)."""
+    _cuda_f16(q, "q")
+    if not q.is_contiguous() or q.dim() != 3:
+        raise ValueError("q must be a contiguous [B, Hq, d] tensor")
+    out, lse = _decode_outputs(q, out, lse, want_lse)
+    if workspace is None:
+        workspace = torch.zeros(mustafar_decode_workspace_bytes(q.shape[0], q.shape[1], k.num_kv_heads, max_len,
+                                                                num_splits), dtype=torch.uint8, device=q.device)
+    _check(load().mustafar_decode_attn(_ptr(q), q.shape[1], C.byref(k.struct), C.byref(v.struct), _ptr(seq_len),
+                                       max_len, scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                       num_splits, _ptr(err), _stream(stream)))
+    return out, lse
+
+
+def mustafar_dense_decode_attn(q: torch.Tensor, k_dense: torch.Tensor, v_dense: torch.Tensor, seq_len: torch.Tensor,
+                               max_len: int, scale: float, out=None, lse=None, workspace=None, num_splits: int = 0,
+                               err=None, stream=None, want_lse: bool = True):
+    """Dense fp16 decode attention (baseline) over [B, Hkv, cap, d] caches."""
+    for t, n in ((q, "q"), (k_dense, "k_dense"), (v_dense, "v_dense")):
+        _cuda_f16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, Hkv, cap, d = k_dense.shape
+    out, lse = _decode_outputs(q, out, lse, want_lse)
+    if workspace is None:
+        workspace = torch.zeros(mustafar_decode_workspace_bytes(B, q.shape[1], Hkv, max_len, num_splits),
+                                dtype=torch.uint8, device=q.device)
+    _check(load().mustafar_dense_decode_attn(_ptr(q), q.shape[1], _ptr(k_dense), _ptr(v_dense), B, Hkv, d, cap,
+                                             _ptr(seq_len), max_len, scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                                             workspace.numel(), num_splits, _ptr(err), _stream(stream)))
+    return out, lse

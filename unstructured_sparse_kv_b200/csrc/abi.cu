@@ -1,0 +1,298 @@
+// abi.cu - the extern "C" entry points declared in include/mustafar.h: argument
+// validation, split planning and kernel launches.  No allocation, no synchronisation.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mustafar {
+namespace {
+
+thread_local std::string g_last_error;
+
+mustafar_status fail(mustafar_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+mustafar_status fail(mustafar_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+mustafar_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(MUSTAFAR_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int32_t keep_count(int32_t d, float s) {
+  if (d <= 0 || d % 32 != 0) return -1;
+  if (!(s >= 0.0f && s < 1.0f)) return -1;  // also rejects NaN
+  const double pruned = std::floor(static_cast<double>(s) * static_cast<double>(d));
+  return d - static_cast<int32_t>(pruned);
+}
+
+mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
+  if (c == nullptr) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: cache descriptor is NULL", name);
+  if (c->batch <= 0 || c->num_kv_heads <= 0 || c->capacity <= 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: batch, num_kv_heads and capacity must be positive", name);
+  if (c->head_dim <= 0 || c->head_dim % 32 != 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: head_dim must be a positive multiple of 32", name);
+  if (c->head_dim != kHeadDim)
+    return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: kernels are built for head_dim 128 (got %d)", name, c->head_dim);
+  if (c->capacity % kTileTokens != 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: capacity must be a multiple of 64 (got %d)", name, c->capacity);
+  if (c->keep < 1 || c->keep > c->head_dim)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: keep must lie in [1, head_dim] (got %d)", name, c->keep);
+  if (static_cast<int64_t>(c->capacity) * c->keep >= (int64_t(1) << 32))
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: capacity*keep must stay below 2^32 (32-bit tile offsets)", name);
+  if (c->bitmap == nullptr || c->values == nullptr || c->tile_offset == nullptr)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: bitmap, values and tile_offset must be non-NULL", name);
+  if (!aligned(c->bitmap, 16) || !aligned(c->values, 16) || !aligned(c->tile_offset, 4))
+    return fail(MUSTAFAR_ERR_MISALIGNED, "%s: bitmap/values need 16-byte, tile_offset 4-byte alignment", name);
+  return MUSTAFAR_OK;
+}
+
+}  // namespace
+
+cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes) {
+  static int done[64][32];  // bytes already granted per (device, kernel slot)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || slot < 0 || slot >= 32)
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (done[dev][slot] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev][slot] = bytes;
+  return e;
+}
+
+}  // namespace mustafar
+
+using namespace mustafar;
+
+extern "C" {
+
+int32_t mustafar_abi_version(void) { return MUSTAFAR_ABI_VERSION; }
+
+const char *mustafar_status_string(mustafar_status s) {
+  switch (s) {
+    case MUSTAFAR_OK: return "ok";
+    case MUSTAFAR_ERR_INVALID_ARG: return "invalid argument";
+    case MUSTAFAR_ERR_UNSUPPORTED: return "unsupported";
+    case MUSTAFAR_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case MUSTAFAR_ERR_CUDA: return "CUDA error";
+    case MUSTAFAR_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char *mustafar_last_error(void) { return g_last_error.c_str(); }
+
+int32_t mustafar_keep_count(int32_t head_dim, float sparsity) { return keep_count(head_dim, sparsity); }
+
+mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity,
+                                     float sparsity, size_t *bitmap_bytes, size_t *values_bytes,
+                                     size_t *offset_bytes) {
+  const int32_t k = keep_count(head_dim, sparsity);
+  if (k < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes: head_dim %% 32 != 0 or sparsity outside [0,1)");
+  if (batch <= 0 || num_kv_heads <= 0 || capacity <= 0 || capacity % kTileTokens != 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes: positive shapes and capacity %% 64 == 0 required");
+  const size_t streams = static_cast<size_t>(batch) * num_kv_heads;
+  if (bitmap_bytes) *bitmap_bytes = streams * capacity * (head_dim / 8);
+  if (values_bytes) *values_bytes = streams * capacity * static_cast<size_t>(k) * 2;
+  if (offset_bytes) *offset_bytes = streams * (capacity / kTileTokens) * 4;
+  return MUSTAFAR_OK;
+}
+
+mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t stride_h, int64_t stride_t, int32_t L,
+                                  float sparsity, const mustafar_cache_t *c, uint32_t *d_err,
+                                  mustafar_stream_t stream) {
+  (void)d_err;
+  mustafar_status s = check_cache(c, "compress");
+  if (s != MUSTAFAR_OK) return s;
+  const int32_t k = keep_count(c->head_dim, sparsity);
+  if (k < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: sparsity must lie in [0, 1)");
+  if (k != c->keep)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: cache keep %d != keep_count(%d, %g) = %d", c->keep,
+                c->head_dim, static_cast<double>(sparsity), k);
+  if (L < 0 || L > c->capacity) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: L must lie in [0, capacity]");
+  if (x == nullptr && L > 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: x is NULL");
+  if (L > 0) {
+    if (!aligned(x, 16) || stride_b % 8 != 0 || stride_h % 8 != 0 || stride_t % 8 != 0)
+      return fail(MUSTAFAR_ERR_MISALIGNED, "compress: x and its strides must be multiples of 8 elements");
+    if (stride_b < 0 || stride_h < 0 || stride_t < 0)
+      return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: negative strides are not supported");
+  }
+  cudaError_t e = launch_compress(static_cast<const uint16_t *>(x), stride_b, stride_h, stride_t, L, c->batch,
+                                  c->num_kv_heads, c->keep, c->capacity, c->bitmap, c->values, c->tile_offset,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "compress launch");
+}
+
+mustafar_status mustafar_append(const void *x, int64_t stride_b, int64_t stride_h, const int32_t *d_pos,
+                                const mustafar_cache_t *c, uint32_t *d_err, mustafar_stream_t stream) {
+  mustafar_status s = check_cache(c, "append");
+  if (s != MUSTAFAR_OK) return s;
+  if (x == nullptr || d_pos == nullptr) return fail(MUSTAFAR_ERR_INVALID_ARG, "append: x and pos must be non-NULL");
+  if (!aligned(x, 16) || stride_b % 8 != 0 || stride_h % 8 != 0)
+    return fail(MUSTAFAR_ERR_MISALIGNED, "append: x and its strides must be multiples of 8 elements");
+  if (stride_b < 0 || stride_h < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "append: negative strides");
+  if (!aligned(d_pos, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "append: pos must be 4-byte aligned");
+  cudaError_t e = launch_append(static_cast<const uint16_t *>(x), stride_b, stride_h, d_pos, c->batch,
+                                c->num_kv_heads, c->keep, c->capacity, c->bitmap, c->values, d_err,
+                                reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "append launch");
+}
+
+mustafar_status mustafar_decode_workspace_bytes(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                                int32_t head_dim, int32_t max_len, int32_t num_splits,
+                                                size_t *bytes) {
+  if (bytes == nullptr) return fail(MUSTAFAR_ERR_INVALID_ARG, "workspace_bytes: bytes is NULL");
+  if (batch <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_len <= 0 || num_splits < 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "workspace_bytes: shapes must be positive, num_splits >= 0");
+  if (num_q_heads % num_kv_heads != 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "workspace_bytes: Hq %% Hkv != 0");
+  if (head_dim != kHeadDim) return fail(MUSTAFAR_ERR_UNSUPPORTED, "workspace_bytes: head_dim must be 128");
+  const int nch = (max_len + kChunk - 1) / kChunk;
+  int splits = num_splits > 0 ? (num_splits < nch ? num_splits : nch) : decode_split_bound(batch, num_kv_heads, max_len);
+  *bytes = decode_workspace_bytes(batch, num_q_heads, num_kv_heads, splits);
+  return MUSTAFAR_OK;
+}
+
+int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t max_len,
+                                    int32_t keep_k, int32_t keep_v, int32_t dense) {
+  if (batch <= 0 || num_kv_heads <= 0 || head_dim != kHeadDim || max_len <= 0) return -1;
+  if (!dense && (keep_k < 1 || keep_k > kHeadDim || keep_v < 1 || keep_v > kHeadDim)) return -1;
+  DecodePlan plan;
+  if (plan_decode(!dense, batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, &plan) != cudaSuccess) return -1;
+  return plan.splits;
+}
+
+namespace {
+
+mustafar_status run_decode(bool sparse, DecodeParams &p, int max_len, int num_splits, void *workspace,
+                           size_t workspace_bytes, const char *name, cudaStream_t stream) {
+  DecodePlan plan;
+  cudaError_t e = plan_decode(sparse, p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, &plan);
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  p.num_splits = plan.splits;
+  p.chunks_per_split = plan.chunks_per_split;
+  p.stage_bytes = plan.stage_bytes;
+  p.warp_bytes = plan.warp_bytes;
+  if (plan.splits > 1) {
+    const size_t need = decode_workspace_bytes(p.B, p.Hq, p.Hkv, plan.splits);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(MUSTAFAR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed (%d splits), got %zu", name, need,
+                  plan.splits, workspace == nullptr ? size_t(0) : workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned", name);
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    const size_t cnt = ((static_cast<size_t>(p.B) * p.Hkv * 4 + 255) / 256) * 256;
+    const size_t ml = ((static_cast<size_t>(p.B) * p.Hq * plan.splits * 2 * 4 + 255) / 256) * 256;
+    p.ws_cnt = reinterpret_cast<uint32_t *>(w);
+    p.ws_ml = reinterpret_cast<float *>(w + cnt);
+    p.ws_o = reinterpret_cast<float *>(w + cnt + ml);
+  }
+  e = launch_decode(sparse, p, plan, stream);
+  return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, name);
+}
+
+mustafar_status check_decode_common(const void *q, int32_t Hq, int32_t B, int32_t Hkv, const int32_t *d_seq_len,
+                                    int32_t max_len, float scale, const void *out, const float *lse,
+                                    const char *name) {
+  if (q == nullptr || out == nullptr || d_seq_len == nullptr)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: q, out and seq_len must be non-NULL", name);
+  if (Hq <= 0 || Hq % Hkv != 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: num_q_heads must be a multiple of num_kv_heads", name);
+  if (Hq / Hkv > 16) return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: at most 16 q heads per kv head", name);
+  if (max_len <= 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: max_len must be positive", name);
+  if (!std::isfinite(scale)) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: scale must be finite", name);
+  if (!aligned(q, 16) || !aligned(out, 16)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: q and out need 16-byte alignment", name);
+  if (lse != nullptr && !aligned(lse, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: lse needs 4-byte alignment", name);
+  if (!aligned(d_seq_len, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: seq_len needs 4-byte alignment", name);
+  (void)B;
+  return MUSTAFAR_OK;
+}
+
+}  // namespace
+
+mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_heads, const mustafar_cache_t *k,
+                                     const mustafar_cache_t *v, const int32_t *d_seq_len, int32_t max_len,
+                                     float scale, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                     int32_t num_splits, uint32_t *d_err, mustafar_stream_t stream) {
+  mustafar_status s = check_cache(k, "decode_attn(k)");
+  if (s != MUSTAFAR_OK) return s;
+  s = check_cache(v, "decode_attn(v)");
+  if (s != MUSTAFAR_OK) return s;
+  if (k->batch != v->batch || k->num_kv_heads != v->num_kv_heads || k->head_dim != v->head_dim)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "decode_attn: K and V caches disagree on batch/heads/head_dim");
+  s = check_decode_common(q, num_q_heads, k->batch, k->num_kv_heads, d_seq_len, max_len, scale, out, lse,
+                          "decode_attn");
+  if (s != MUSTAFAR_OK) return s;
+  if (num_splits < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "decode_attn: num_splits must be >= 0");
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t *>(q);
+  p.kbm = k->bitmap;
+  p.kval = k->values;
+  p.vbm = v->bitmap;
+  p.vval = v->values;
+  p.keep_k = k->keep;
+  p.keep_v = v->keep;
+  p.cap_k = k->capacity;
+  p.cap_v = v->capacity;
+  p.seq_len = d_seq_len;
+  p.B = k->batch;
+  p.Hq = num_q_heads;
+  p.Hkv = k->num_kv_heads;
+  p.G = num_q_heads / k->num_kv_heads;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.out = static_cast<uint16_t *>(out);
+  p.lse = lse;
+  p.err = d_err;
+  return run_decode(true, p, max_len, num_splits, workspace, workspace_bytes, "decode_attn",
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+mustafar_status mustafar_dense_decode_attn(const void *q, int32_t num_q_heads, const void *k_dense,
+                                           const void *v_dense, int32_t batch, int32_t num_kv_heads,
+                                           int32_t head_dim, int32_t capacity, const int32_t *d_seq_len,
+                                           int32_t max_len, float scale, void *out, float *lse, void *workspace,
+                                           size_t workspace_bytes, int32_t num_splits, uint32_t *d_err,
+                                           mustafar_stream_t stream) {
+  if (k_dense == nullptr || v_dense == nullptr)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "dense_decode_attn: k_dense and v_dense must be non-NULL");
+  if (batch <= 0 || num_kv_heads <= 0 || capacity <= 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "dense_decode_attn: shapes must be positive");
+  if (head_dim != kHeadDim) return fail(MUSTAFAR_ERR_UNSUPPORTED, "dense_decode_attn: head_dim must be 128");
+  if (capacity % kChunk != 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "dense_decode_attn: capacity must be a multiple of 16");
+  if (!aligned(k_dense, 16) || !aligned(v_dense, 16))
+    return fail(MUSTAFAR_ERR_MISALIGNED, "dense_decode_attn: caches need 16-byte alignment");
+  mustafar_status s = check_decode_common(q, num_q_heads, batch, num_kv_heads, d_seq_len, max_len, scale, out, lse,
+                                          "dense_decode_attn");
+  if (s != MUSTAFAR_OK) return s;
+  if (num_splits < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "dense_decode_attn: num_splits must be >= 0");
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t *>(q);
+  p.kd = static_cast<const uint16_t *>(k_dense);
+  p.vd = static_cast<const uint16_t *>(v_dense);
+  p.cap_k = p.cap_v = capacity;
+  p.keep_k = p.keep_v = kHeadDim;
+  p.seq_len = d_seq_len;
+  p.B = batch;
+  p.Hq = num_q_heads;
+  p.Hkv = num_kv_heads;
+  p.G = num_q_heads / num_kv_heads;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.out = static_cast<uint16_t *>(out);
+  p.lse = lse;
+  p.err = d_err;
+  return run_decode(false, p, max_len, num_splits, workspace, workspace_bytes, "dense_decode_attn",
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,155 @@
+// compress.cu - prune + compress (prefill) and append (decode) kernels.
+//
+// Per-token magnitude pruning and the bitmap-based sparse format (MUSTAFAR summary,
+// atlas.scime.ai, "Approach"; Mustafar abstract, catalyzex author page).  Layout of
+// the format: see include/mustafar.h.
+//
+// compress: one CTA = 128 consecutive tokens of one (b, kv head) stream, one thread per
+//   token.  The CTA stages its 32 KB of dense rows in shared memory with coalesced
+//   16-byte cp.async (16 threads per 256-byte row), each thread runs the top-k on its
+//   own row, writes its 16-byte bitmap, packs its kept values into a shared staging
+//   run, and the CTA writes the 128*k packed values with coalesced 16-byte stores.
+// append: one thread per (b, kv head) vector of the new token.
+#include "internal.h"
+#include "select.cuh"
+
+namespace mustafar {
+
+constexpr int kCompressThreads = 128;
+constexpr int kRowBytesDense = kHeadDim * 2;  // 256
+
+// byte offset of 16-byte chunk j of staged row `tok` (XOR swizzle: conflict-free row reads)
+__device__ __forceinline__ int stage_off(int tok, int j) { return tok * kRowBytesDense + ((j ^ (tok & 15)) << 4); }
+
+__global__ void __launch_bounds__(kCompressThreads)
+compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, int k,
+                int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
+                uint32_t *__restrict__ tile_offset) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t *in_stage = smem;
+  uint16_t *out_stage = reinterpret_cast<uint16_t *>(smem + kCompressThreads * kRowBytesDense);
+
+  const int tid = threadIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t stream = static_cast<int64_t>(b) * H + h;
+
+  // tile offsets of the whole stream: the closed form 64*i*k (= popcount prefix sums, every
+  // token keeps exactly k channels)
+  const int ntiles = cap / kTileTokens;
+  for (int i = blockIdx.x * kCompressThreads + tid; i < ntiles; i += gridDim.x * kCompressThreads)
+    tile_offset[stream * ntiles + i] = static_cast<uint32_t>(i) * kTileTokens * static_cast<uint32_t>(k);
+
+  const int t0 = blockIdx.x * kCompressThreads;
+  const int ntok = min(kCompressThreads, L - t0);
+  if (ntok <= 0) return;
+
+  const uint16_t *xs = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
+  for (int idx = tid; idx < ntok * 16; idx += kCompressThreads) {
+    const int tok = idx >> 4, j = idx & 15;
+    cp_async16(smem_addr(in_stage + stage_off(tok, j)), xs + static_cast<int64_t>(t0 + tok) * st + j * 8);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  if (tid < ntok) {
+    uint32_t raw[64];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(in_stage + stage_off(tid, j));
+      raw[4 * j + 0] = v.x;
+      raw[4 * j + 1] = v.y;
+      raw[4 * j + 2] = v.z;
+      raw[4 * j + 3] = v.w;
+    }
+    uint32_t bm[kWords];
+    topk_bitmap(raw, k, bm);
+    reinterpret_cast<uint4 *>(bitmap)[stream * cap + t0 + tid] = make_uint4(bm[0], bm[1], bm[2], bm[3]);
+    // pack the kept values in ascending channel order
+    uint16_t *dst = out_stage + tid * k;
+    int jj = 0;
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) {
+      uint32_t m = bm[w];
+      while (m && jj < k) {
+        const int ch = 32 * w + __ffs(m) - 1;
+        m &= m - 1;
+        dst[jj++] = *reinterpret_cast<const uint16_t *>(in_stage + stage_off(tid, ch >> 3) + ((ch & 7) << 1));
+      }
+    }
+  }
+  __syncthreads();
+
+  // coalesced write-out of the CTA's packed run; its start (stream*cap + t0)*k*2 bytes is
+  // 16-byte aligned because cap % 64 == 0 and t0 % 128 == 0
+  uint16_t *vdst = values + (stream * cap + t0) * static_cast<int64_t>(k);
+  const int n = ntok * k;
+  const int nvec = n >> 3;
+  for (int i = tid; i < nvec; i += kCompressThreads)
+    reinterpret_cast<uint4 *>(vdst)[i] = reinterpret_cast<const uint4 *>(out_stage)[i];
+  for (int i = (nvec << 3) + tid; i < n; i += kCompressThreads) vdst[i] = out_stage[i];
+}
+
+__global__ void __launch_bounds__(64)
+append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int32_t *__restrict__ pos, int B,
+              int H, int k, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
+              uint32_t *__restrict__ err) {
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v >= B * H) return;
+  const int b = v / H, h = v - b * H;
+  const int p = pos[b];
+  if (p < 0 || p >= cap) {
+    if (err != nullptr) atomicOr(err, MUSTAFAR_DEVERR_POS_RANGE);
+    return;
+  }
+  const uint16_t *src = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
+  uint32_t raw[64];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src) + j);
+    raw[4 * j + 0] = q.x;
+    raw[4 * j + 1] = q.y;
+    raw[4 * j + 2] = q.z;
+    raw[4 * j + 3] = q.w;
+  }
+  uint32_t bm[kWords];
+  topk_bitmap(raw, k, bm);
+  const int64_t stream = static_cast<int64_t>(b) * H + h;
+  reinterpret_cast<uint4 *>(bitmap)[stream * cap + p] = make_uint4(bm[0], bm[1], bm[2], bm[3]);
+  uint16_t *dst = values + (stream * cap + p) * static_cast<int64_t>(k);
+  int jj = 0;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    uint32_t m = bm[w];
+    while (m && jj < k) {
+      const int ch = 32 * w + __ffs(m) - 1;
+      m &= m - 1;
+      dst[jj++] = __ldg(src + ch);
+    }
+  }
+}
+
+cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H, int k,
+                            int cap, uint32_t *bitmap, uint16_t *values, uint32_t *tile_offset,
+                            cudaStream_t stream) {
+  const size_t smem = kCompressThreads * kRowBytesDense + static_cast<size_t>(kCompressThreads) * k * 2;
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(compress_kernel), 0,
+                                    kCompressThreads * kRowBytesDense + kCompressThreads * kHeadDim * 2);
+  if (e != cudaSuccess) return e;
+  const int nbx = L > 0 ? (L + kCompressThreads - 1) / kCompressThreads : 1;
+  dim3 grid(nbx, H, B);
+  compress_kernel<<<grid, kCompressThreads, smem, stream>>>(x, sb, sh, st, L, H, k, cap, bitmap, values,
+                                                            tile_offset);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H, int k,
+                          int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err, cudaStream_t stream) {
+  const int n = B * H;
+  const int threads = 64;
+  append_kernel<<<(n + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, k, cap, bitmap,
+                                                                     values, err);
+  return cudaGetLastError();
+}
+
+}  // namespace mustafar

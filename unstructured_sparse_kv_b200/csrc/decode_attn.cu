@@ -1,0 +1,496 @@
+// decode_attn.cu - split-K decode attention over the bitmap-compressed caches, and the
+// dense fp16 baseline built on the same skeleton.
+//
+// Computes, for each batch row b and q head hq (kv head g = hq / G):
+//   out = softmax(scale * q K~^T) V~  over the pruned caches K~, V~
+// directly from the compressed format (Mustafar abstract, catalyzex author page: a custom
+// attention kernel that computes directly over the compressed caches; MUSTAFAR summary,
+// atlas.scime.ai, "Approach": an SpMV-style attention kernel over the bitmap format).
+//
+// Work decomposition (B200-first, not the pages' design):
+// * grid = (splits, Hkv, B); a CTA owns a contiguous range of 16-token chunks of one
+//   (b, kv head) stream and the whole GQA group of that kv head.
+// * each of the CTA's 4 warps is an independent pipeline over every 4th chunk of the
+//   range: a cp.async ring (NSTAGE deep) stages the chunk's compressed bytes (16 bitmap
+//   rows + 16*k packed values, for K and for V) in the warp's own shared memory, so the
+//   loop needs no CTA barrier.
+// * expansion: lanes 0-15 rebuild the 16 K rows and lanes 16-31 the 16 V rows of the chunk
+//   as dense fp16 rows in shared memory, walking each row's set bits (__ffs) and scattering
+//   its packed values in order.
+// * the group's logits S = Q K~^T (G q heads padded to 16 rows x 16 tokens x 128 channels)
+//   and O += P V~ run as mma.sync m16n8k16 (fp16 in, fp32 accumulate) fed by ldmatrix;
+//   softmax is online (running max / sum per row in the log2 domain).
+// * warps merge in shared memory; with splits > 1 each CTA writes its (m, l, o) partial to
+//   the workspace and the last CTA of the stream (atomic ticket, no spin-wait) merges all
+//   splits in a fixed order and writes out / lse.
+#include <cfloat>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace mustafar {
+
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeThreads = 32 * kDecodeWarps;
+constexpr float kNegInf = -INFINITY;
+
+template <bool SPARSE>
+__device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t stream, int c, uint8_t *stage,
+                                            int lane) {
+  if constexpr (SPARSE) {
+    const int64_t tk = stream * P.cap_k + static_cast<int64_t>(c) * kChunk;
+    const int64_t tv = stream * P.cap_v + static_cast<int64_t>(c) * kChunk;
+    const uint8_t *src_kb = reinterpret_cast<const uint8_t *>(P.kbm + tk * kWords);
+    const uint8_t *src_vb = reinterpret_cast<const uint8_t *>(P.vbm + tv * kWords);
+    const uint8_t *src_kv = reinterpret_cast<const uint8_t *>(P.kval + tk * P.keep_k);
+    const uint8_t *src_vv = reinterpret_cast<const uint8_t *>(P.vval + tv * P.keep_v);
+    const uint32_t dst = smem_addr(stage);
+    // bitmaps: 16 rows x 16 B for K then V (32 units of 16 B: one per lane)
+    {
+      const uint8_t *src = lane < 16 ? src_kb + lane * 16 : src_vb + (lane - 16) * 16;
+      cp_async16(dst + lane * 16, src);
+    }
+    const int uk = 2 * P.keep_k, uv = 2 * P.keep_v;  // 16-byte units of packed values (16*k*2/16)
+    for (int u = lane; u < uk; u += 32) cp_async16(dst + 512 + u * 16, src_kv + u * 16);
+    for (int u = lane; u < uv; u += 32) cp_async16(dst + 512 + uk * 16 + u * 16, src_vv + u * 16);
+  } else {
+    const int64_t row0 = (stream * P.cap_k + static_cast<int64_t>(c) * kChunk) * kHeadDim;
+    const uint8_t *src_k = reinterpret_cast<const uint8_t *>(P.kd + row0);
+    const uint8_t *src_v = reinterpret_cast<const uint8_t *>(P.vd + row0);
+    const uint32_t dst = smem_addr(stage);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // 256 units of 16 B per tile, 8 per lane
+      const int u = lane + 32 * i;
+      const int r = u >> 4, j = u & 15;
+      cp_async16(dst + r * kRowBytes + j * 16, src_k + u * 16);
+      cp_async16(dst + kTileBytes + r * kRowBytes + j * 16, src_v + u * 16);
+    }
+  }
+}
+
+// Rebuild the chunk's 16 K rows (lanes 0-15) and 16 V rows (lanes 16-31) as dense fp16.
+__device__ __forceinline__ void expand_chunk(const DecodeParams &P, const uint8_t *stage, uint8_t *dense, int lane,
+                                             int t0, int L) {
+  const int side = lane >> 4, r = lane & 15;
+  uint8_t *row = dense + side * kTileBytes + r * kRowBytes;
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) reinterpret_cast<uint4 *>(row)[j] = z;
+  if (t0 + r < L) {
+    const uint4 bm = *reinterpret_cast<const uint4 *>(stage + side * 256 + r * 16);
+    const int kk = side ? P.keep_v : P.keep_k;
+    const uint16_t *vals = reinterpret_cast<const uint16_t *>(stage + 512 + side * 32 * P.keep_k) + r * kk;
+    uint16_t *drow = reinterpret_cast<uint16_t *>(row);
+    const uint32_t words[4] = {bm.x, bm.y, bm.z, bm.w};
+    int j = 0;
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) {
+      uint32_t m = words[w];
+      while (m && j < kk) {  // a bitmap never holds more than k bits; the bound only guards the buffer
+        const int ch = 32 * w + __ffs(m) - 1;
+        m &= m - 1;
+        drow[ch] = vals[j++];
+      }
+    }
+  }
+}
+
+template <bool SPARSE, int NSTAGE, bool HIROWS>
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeParams P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int G = P.G;
+  const int cap = SPARSE ? min(P.cap_k, P.cap_v) : P.cap_k;
+  int L = P.seq_len[b];
+  if (L < 0 || L > cap) {
+    if (threadIdx.x == 0 && split == 0 && g == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_LEN_RANGE);
+    L = L < 0 ? 0 : cap;
+  }
+  const int nch = (L + kChunk - 1) / kChunk;
+  const int c_begin = split * P.chunks_per_split;
+  const int c_end = min(nch, c_begin + P.chunks_per_split);
+  const int my_n = (c_end - c_begin > warp) ? (c_end - c_begin - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+  const int64_t stream = static_cast<int64_t>(b) * P.Hkv + g;
+
+  uint8_t *wbase = smem + warp * P.warp_bytes;
+  uint8_t *dense = wbase + NSTAGE * P.stage_bytes;  // sparse only
+
+  // Q A-fragments (rows = q heads of the group, zero beyond G), 8 k-steps of 16 channels
+  const int gq = lane >> 2, qq = lane & 3;
+  uint32_t qa[8][4];
+  {
+    const uint16_t *qb = P.q + (static_cast<int64_t>(b) * P.Hq + static_cast<int64_t>(g) * G) * kHeadDim;
+    const bool r0 = gq < G, r1 = HIROWS && (gq + 8 < G);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int col = ks * 16 + 2 * qq;
+      qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + col) : 0u;
+      qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + col) : 0u;
+      qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + col + 8) : 0u;
+      qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + col + 8) : 0u;
+    }
+  }
+
+  float o[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run[2] = {kNegInf, kNegInf};
+  float l_run[2] = {0.f, 0.f};
+
+#pragma unroll
+  for (int i = 0; i < NSTAGE - 1; ++i) {
+    if (i < my_n) issue_chunk<SPARSE>(P, stream, c_begin + warp + kDecodeWarps * i, wbase + i * P.stage_bytes, lane);
+    cp_async_commit();
+  }
+
+  // per-lane ldmatrix address offsets
+  const int mat = lane >> 3;
+  const uint32_t k_off = (((mat >> 1) << 3) + (lane & 7)) * kRowBytes + ((mat & 1) << 4);
+  const uint32_t v_off = (((mat & 1) << 3) + (lane & 7)) * kRowBytes + ((mat >> 1) << 4);
+
+#pragma unroll 1
+  for (int i = 0; i < my_n; ++i) {
+    {
+      const int ni = i + NSTAGE - 1;
+      if (ni < my_n)
+        issue_chunk<SPARSE>(P, stream, c_begin + warp + kDecodeWarps * ni, wbase + (ni % NSTAGE) * P.stage_bytes,
+                            lane);
+      cp_async_commit();
+    }
+    cp_async_wait<NSTAGE - 1>();
+    __syncwarp();
+    const uint8_t *stage = wbase + (i % NSTAGE) * P.stage_bytes;
+    const int t0 = (c_begin + warp + kDecodeWarps * i) * kChunk;
+    const uint8_t *ktile;
+    const uint8_t *vtile;
+    if constexpr (SPARSE) {
+      expand_chunk(P, stage, dense, lane, t0, L);
+      __syncwarp();
+      ktile = dense;
+      vtile = dense + kTileBytes;
+    } else {
+      ktile = stage;
+      vtile = stage + kTileBytes;
+    }
+
+    // S = Q K~^T for the chunk's 16 tokens (two n-tiles of 8)
+    float s[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    const uint32_t kaddr = smem_addr(ktile) + k_off;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * 32);
+      mma_f16_16816(s[0], qa[ks], b0, b1);
+      mma_f16_16816(s[1], qa[ks], b2, b3);
+    }
+
+    // scale into the log2 domain, mask tokens >= L, online softmax per row
+    float mx[2] = {kNegInf, kNegInf};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = t0 + nt * 8 + 2 * qq + (e & 1);
+        const float x = tok < L ? s[nt][e] * P.scale_log2 : kNegInf;
+        s[nt][e] = x;
+        mx[e >> 1] = fmaxf(mx[e >> 1], x);
+      }
+    }
+    float alpha[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+      mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+      const float m_new = fmaxf(m_run[h], mx[h]);
+      const float base = m_new == kNegInf ? 0.f : m_new;
+      alpha[h] = fast_exp2(m_run[h] - base);
+      m_run[h] = m_new;
+      mx[h] = base;
+    }
+    float psum[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p = fast_exp2(s[nt][e] - mx[e >> 1]);
+        s[nt][e] = p;
+        psum[e >> 1] += p;
+      }
+    }
+    l_run[0] = l_run[0] * alpha[0] + psum[0];
+    l_run[1] = l_run[1] * alpha[1] + psum[1];
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        o[nt][0] *= alpha[0];
+        o[nt][1] *= alpha[0];
+        o[nt][2] *= alpha[1];
+        o[nt][3] *= alpha[1];
+      }
+    }
+    uint32_t pa[4];
+    pa[0] = pack_half2(s[0][0], s[0][1]);
+    pa[1] = pack_half2(s[0][2], s[0][3]);
+    pa[2] = pack_half2(s[1][0], s[1][1]);
+    pa[3] = pack_half2(s[1][2], s[1][3]);
+
+    // O += P V~ : 16 n-tiles of 8 channels
+    const uint32_t vaddr = smem_addr(vtile) + v_off;
+#pragma unroll
+    for (int ntp = 0; ntp < 8; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(b0, b1, b2, b3, vaddr + ntp * 32);
+      mma_f16_16816(o[2 * ntp], pa, b0, b1);
+      mma_f16_16816(o[2 * ntp + 1], pa, b2, b3);
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+  }
+
+  // ---- merge the 4 warps (shared memory reused after everyone is done)
+  __syncthreads();
+  float *sm_m = reinterpret_cast<float *>(smem);             // [4][16]
+  float *sm_l = sm_m + kDecodeWarps * 16;                     // [4][16]
+  float *sm_o = sm_l + kDecodeWarps * 16;                     // [4][G][128]
+  if (qq == 0) {
+    if (gq < G) {
+      sm_m[warp * 16 + gq] = m_run[0];
+      sm_l[warp * 16 + gq] = l_run[0];
+    }
+    if (HIROWS && gq + 8 < G) {
+      sm_m[warp * 16 + gq + 8] = m_run[1];
+      sm_l[warp * 16 + gq + 8] = l_run[1];
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) {
+    const int ch = nt * 8 + 2 * qq;
+    if (gq < G)
+      *reinterpret_cast<float2 *>(sm_o + (warp * G + gq) * kHeadDim + ch) = make_float2(o[nt][0], o[nt][1]);
+    if (HIROWS && gq + 8 < G)
+      *reinterpret_cast<float2 *>(sm_o + (warp * G + gq + 8) * kHeadDim + ch) = make_float2(o[nt][2], o[nt][3]);
+  }
+  __syncthreads();
+
+  const int c = threadIdx.x;  // output channel
+  const int S = P.num_splits;
+  for (int r = 0; r < G; ++r) {
+    float M = kNegInf;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
+    float lsum = 0.f, acc = 0.f;
+    if (M != kNegInf) {
+#pragma unroll
+      for (int w = 0; w < kDecodeWarps; ++w) {
+        const float wt = fast_exp2(sm_m[w * 16 + r] - M);
+        lsum += sm_l[w * 16 + r] * wt;
+        acc += sm_o[(w * G + r) * kHeadDim + c] * wt;
+      }
+    }
+    const int64_t hq = static_cast<int64_t>(b) * P.Hq + static_cast<int64_t>(g) * G + r;
+    if (S == 1) {
+      P.out[hq * kHeadDim + c] = __float2half_rn(lsum > 0.f ? acc / lsum : 0.f);
+      if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
+    } else {
+      P.ws_o[(hq * S + split) * kHeadDim + c] = acc;
+      if (c == 0) *reinterpret_cast<float2 *>(P.ws_ml + (hq * S + split) * 2) = make_float2(M, lsum);
+    }
+  }
+  if (S == 1) return;
+
+  // ---- last CTA of this stream merges every split (no waiting: an atomic ticket)
+  __threadfence();
+  __syncthreads();
+  __shared__ int is_last;
+  if (threadIdx.x == 0) {
+    const uint32_t ticket = atomicAdd(P.ws_cnt + stream, 1u);
+    is_last = (ticket == static_cast<uint32_t>(S - 1));
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  for (int r = 0; r < G; ++r) {
+    const int64_t hq = static_cast<int64_t>(b) * P.Hq + static_cast<int64_t>(g) * G + r;
+    const float *ml = P.ws_ml + hq * S * 2;
+    float M = kNegInf;
+    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(ml + 2 * sp));
+    float lsum = 0.f, acc = 0.f;
+    if (M != kNegInf) {
+      for (int sp = 0; sp < S; ++sp) {
+        const float wt = fast_exp2(__ldcg(ml + 2 * sp) - M);
+        lsum += __ldcg(ml + 2 * sp + 1) * wt;
+        acc += __ldcg(P.ws_o + (hq * S + sp) * kHeadDim + c) * wt;
+      }
+    }
+    P.out[hq * kHeadDim + c] = __float2half_rn(lsum > 0.f ? acc / lsum : 0.f);
+    if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
+  }
+  if (threadIdx.x == 0) P.ws_cnt[stream] = 0u;  // leave the workspace ready for the next call
+}
+
+// ------------------------------------------------------------------------------------ host side
+namespace {
+
+using KernelFn = void (*)(const DecodeParams);
+
+template <bool SPARSE, int NSTAGE>
+KernelFn pick_rows(bool hirows) {
+  return hirows ? decode_kernel<SPARSE, NSTAGE, true> : decode_kernel<SPARSE, NSTAGE, false>;
+}
+
+KernelFn pick_kernel(bool sparse, int nstage, bool hirows) {
+  if (sparse) {
+    switch (nstage) {
+      case 2: return pick_rows<true, 2>(hirows);
+      case 3: return pick_rows<true, 3>(hirows);
+      default: return pick_rows<true, 4>(hirows);
+    }
+  }
+  switch (nstage) {
+    case 2: return pick_rows<false, 2>(hirows);
+    default: return pick_rows<false, 3>(hirows);
+  }
+}
+
+int kernel_slot(bool sparse, int nstage, bool hirows) { return 1 + (sparse ? 0 : 8) + 2 * nstage + (hirows ? 1 : 0); }
+
+struct DeviceInfo {
+  int sms = 0;
+};
+
+cudaError_t device_info(DeviceInfo *info) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static int cached_sms[64] = {0};
+  if (dev >= 0 && dev < 64 && cached_sms[dev] > 0) {
+    info->sms = cached_sms[dev];
+    return cudaSuccess;
+  }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) cached_sms[dev] = sms;
+  info->sms = sms;
+  return cudaSuccess;
+}
+
+// resident CTAs per SM for a kernel and dynamic smem size, cached per device (the query is
+// made once, outside any stream capture, so planning stays capture-safe afterwards)
+cudaError_t occupancy(KernelFn fn, int slot, int smem, int *per_sm) {
+  static int cache_smem[64][32];
+  static int cache_val[64][32];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < 64 && slot >= 0 && slot < 32;
+  if (cacheable && cache_smem[dev][slot] == smem && cache_val[dev][slot] > 0) {
+    *per_sm = cache_val[dev][slot];
+    return cudaSuccess;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, fn, kDecodeThreads, smem);
+  if (e == cudaSuccess && cacheable) {
+    cache_smem[dev][slot] = smem;
+    cache_val[dev][slot] = *per_sm;
+  }
+  return e;
+}
+
+constexpr int kMaxSplits = 128;
+constexpr int kMinChunksPerCta = 2 * kDecodeWarps;
+constexpr int kMaxCtasPerSm = 4;
+constexpr int kWarpSmemTarget = 18 * 1024;  // ~3 CTAs of 4 warps per SM
+
+}  // namespace
+
+int decode_split_bound(int B, int Hkv, int max_len) {
+  DeviceInfo info;
+  if (device_info(&info) != cudaSuccess) info.sms = 148;
+  const int nch = (max_len + kChunk - 1) / kChunk;
+  const int streams = B * Hkv;
+  int bound = (info.sms * kMaxCtasPerSm) / (streams > 0 ? streams : 1);
+  bound = bound < 1 ? 1 : bound;
+  const int by_len = nch / kMinChunksPerCta;
+  bound = by_len < bound ? by_len : bound;
+  bound = bound < 1 ? 1 : bound;
+  return bound > kMaxSplits ? kMaxSplits : bound;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int splits) {
+  if (splits <= 1) return 256;
+  const size_t cnt = ((static_cast<size_t>(B) * Hkv * 4 + 255) / 256) * 256;
+  const size_t ml = ((static_cast<size_t>(B) * Hq * splits * 2 * 4 + 255) / 256) * 256;
+  const size_t o = static_cast<size_t>(B) * Hq * splits * kHeadDim * 4;
+  return cnt + ml + o;
+}
+
+cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
+                        DecodePlan *plan) {
+  DeviceInfo info;
+  cudaError_t e = device_info(&info);
+  if (e != cudaSuccess) return e;
+  int nstage, stage_bytes, warp_bytes;
+  if (sparse) {
+    stage_bytes = 512 + 32 * (keep_k + keep_v);
+    nstage = (kWarpSmemTarget - 2 * kTileBytes) / stage_bytes;
+    nstage = nstage < 2 ? 2 : (nstage > 4 ? 4 : nstage);
+    warp_bytes = nstage * stage_bytes + 2 * kTileBytes;
+  } else {
+    stage_bytes = 2 * kTileBytes;
+    nstage = 3;
+    warp_bytes = nstage * stage_bytes;
+  }
+  const int merge_bytes = kDecodeWarps * 16 * 2 * 4 + kDecodeWarps * G * kHeadDim * 4;
+  int smem = kDecodeWarps * warp_bytes;
+  smem = smem < merge_bytes ? merge_bytes : smem;
+  const bool hirows = G > 8;
+  KernelFn fn = pick_kernel(sparse, nstage, hirows);
+  e = ensure_smem_limit(reinterpret_cast<const void *>(fn), kernel_slot(sparse, nstage, hirows), smem);
+  if (e != cudaSuccess) return e;
+
+  const int nch = (max_len + kChunk - 1) / kChunk;
+  int splits;
+  if (forced_splits > 0) {
+    splits = forced_splits;
+  } else {
+    int per_sm = 0;
+    e = occupancy(fn, kernel_slot(sparse, nstage, hirows), smem, &per_sm);
+    if (e != cudaSuccess) return e;
+    per_sm = per_sm < 1 ? 1 : (per_sm > kMaxCtasPerSm ? kMaxCtasPerSm : per_sm);
+    const int streams = B * Hkv;
+    splits = (info.sms * per_sm) / streams;  // one full wave of CTAs, no partial second wave
+    const int by_len = nch / kMinChunksPerCta;
+    splits = splits < by_len ? splits : by_len;
+    splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
+  }
+  splits = splits > nch ? nch : splits;
+  splits = splits < 1 ? 1 : splits;
+  const int cps = (nch + splits - 1) / splits;
+  splits = cps > 0 ? (nch + cps - 1) / cps : 1;
+  splits = splits < 1 ? 1 : splits;
+  plan->splits = splits;
+  plan->chunks_per_split = cps > 0 ? cps : 1;
+  plan->nstage = nstage;
+  plan->stage_bytes = stage_bytes;
+  plan->warp_bytes = warp_bytes;
+  plan->smem_bytes = smem;
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode(bool sparse, const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+  KernelFn fn = pick_kernel(sparse, plan.nstage, p.G > 8);
+  dim3 grid(plan.splits, p.Hkv, p.B);
+  fn<<<grid, kDecodeThreads, plan.smem_bytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mustafar

@@ -1,0 +1,62 @@
+// internal.h - declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "mustafar.h"
+
+namespace mustafar {
+
+// Set a kernel's dynamic shared-memory limit once per device.
+cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes);
+
+cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H, int k,
+                            int cap, uint32_t *bitmap, uint16_t *values, uint32_t *tile_offset,
+                            cudaStream_t stream);
+cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H, int k,
+                          int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err, cudaStream_t stream);
+
+struct DecodeParams {
+  const uint16_t *q;  // [B][Hq][128]
+  // compressed caches (sparse kernel)
+  const uint32_t *kbm;
+  const uint16_t *kval;
+  const uint32_t *vbm;
+  const uint16_t *vval;
+  int keep_k, keep_v;
+  // dense caches (baseline kernel), [B][Hkv][cap][128]
+  const uint16_t *kd;
+  const uint16_t *vd;
+  int cap_k, cap_v;
+  const int32_t *seq_len;
+  int B, Hq, Hkv, G;
+  float scale_log2;
+  int num_splits, chunks_per_split;
+  int stage_bytes, warp_bytes;
+  uint16_t *out;
+  float *lse;
+  float *ws_o;        // [B*Hq][splits][128]
+  float *ws_ml;       // [B*Hq][splits][2]
+  uint32_t *ws_cnt;   // [B*Hkv]
+  uint32_t *err;
+};
+
+struct DecodePlan {
+  int splits;
+  int chunks_per_split;
+  int nstage;
+  int stage_bytes;
+  int warp_bytes;
+  int smem_bytes;
+};
+
+// Plan (split count, pipeline depth, shared memory) for one decode call.
+cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
+                        DecodePlan *plan);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int splits);
+int decode_split_bound(int B, int Hkv, int max_len);
+cudaError_t launch_decode(bool sparse, const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
+
+}  // namespace mustafar

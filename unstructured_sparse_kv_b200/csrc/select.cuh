@@ -1,0 +1,90 @@
+// select.cuh - deterministic per-token top-k by magnitude, one thread per 128-channel vector.
+//
+// Per-token magnitude pruning (MUSTAFAR summary, atlas.scime.ai, "Approach"; Mustafar
+// abstract, catalyzex author page): keep the k channels with the largest |x|.  The
+// library fixes the two points the pages leave open: the magnitude key is the fp16
+// bit pattern with the sign cleared (so the order is |x| for finite values and +0 == -0),
+// and on equal keys the lower channel index is kept.
+//
+// Method: a 15-step binary search for the k-th largest key T (the largest T with
+// #{key >= T} >= k).  Each count is SIMD-within-a-register: two 15-bit keys share a
+// 32-bit word, and key + (0x8000 - T) sets bit 15 of its half exactly when key >= T
+// (no carry leaves a half).  Keys are paired as (channel i, channel i+16) of a 32-channel
+// group so that shifting the sum right by 15-i drops both indicator bits onto bits i and
+// 16+i: OR-ing the 16 pairs of a group yields that group's bitmap word directly.
+#pragma once
+
+#include "common.cuh"
+
+namespace mustafar {
+
+// raw[r] holds channels (2r, 2r+1) as two fp16 values (low half = even channel).
+// Produces p[16w + i] = key(32w + i) | key(32w + i + 16) << 16.
+__device__ __forceinline__ void make_keys(const uint32_t (&raw)[64], uint32_t (&p)[64]) {
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t a = raw[16 * w + (i >> 1)];
+      const uint32_t b = raw[16 * w + 8 + (i >> 1)];
+      p[16 * w + i] = __byte_perm(a, b, (i & 1) ? 0x7632u : 0x5410u) & 0x7FFF7FFFu;
+    }
+  }
+}
+
+// Bitmap of {channel : key >= T}, 0 <= T <= 0x8000.
+__device__ __forceinline__ void ge_bitmap(const uint32_t (&p)[64], uint32_t T, uint32_t (&g)[kWords]) {
+  uint32_t c = 0x8000u - T;
+  c |= c << 16;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t t = p[16 * w + i] + c;
+      acc |= (t >> (15 - i)) & ((1u << i) | (1u << (16 + i)));
+    }
+    g[w] = acc;
+  }
+}
+
+__device__ __forceinline__ int popc4(const uint32_t (&g)[kWords]) {
+  return __popc(g[0]) + __popc(g[1]) + __popc(g[2]) + __popc(g[3]);
+}
+
+// Kept-channel bitmap of the k largest keys, ties toward the lower channel index.
+__device__ __forceinline__ void topk_bitmap(const uint32_t (&raw)[64], int k, uint32_t (&bm)[kWords]) {
+  uint32_t p[64];
+  make_keys(raw, p);
+  uint32_t T = 0;
+  uint32_t g[kWords];
+#pragma unroll 1
+  for (int bit = 14; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    ge_bitmap(p, cand, g);
+    if (popc4(g) >= k) T = cand;
+  }
+  ge_bitmap(p, T, g);  // #{key >= T} >= k, and #{key > T} < k
+  if (popc4(g) == k) {
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) bm[w] = g[w];
+    return;
+  }
+  uint32_t gt[kWords];
+  ge_bitmap(p, T + 1, gt);
+  int need = k - popc4(gt);  // how many of the keys equal to T survive, lowest channels first
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    uint32_t e = g[w] & ~gt[w];
+    uint32_t take = 0;
+    while (e != 0u && need > 0) {
+      const uint32_t low = e & (0u - e);
+      take |= low;
+      e ^= low;
+      --need;
+    }
+    bm[w] = gt[w] | take;
+  }
+}
+
+}  // namespace mustafar

@@ -311,9 +311,23 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=64 * 20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-launches", type=int, default=0,
+                    help="ncu case: build the workload, run this many eager steps (append K, append V, "
+                         "attend) over the rotated caches, and exit without timing")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_launches > 0:
+        import torch
+        import unstructured_sparse_kv_b200 as M
+        M.load()
+        wl = Workload(rank_seed(0), torch.device("cuda", 0))
+        for i in range(args.profile_launches):
+            wl.step(i)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": "decode step workload", "steps": args.profile_launches,
+                          "compressed_kv_bytes_per_copy": wl.compressed_bytes, "copies": ROTATE}))
+        return 0
 
     import torch
     import torch.distributed as dist

@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     }
     const int64_t hq = static_cast<int64_t>(b) * P.Hq + static_cast<int64_t>(g) * G + r;
     if (S == 1) {
-      P.out[hq * kHeadDim + c] = __float2half_rn(lsum > 0.f ? acc / lsum : 0.f);
+      P.out[hq * kHeadDim + c] = __half_as_ushort(__float2half_rn(lsum > 0.f ? acc / lsum : 0.f));
       if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
     } else {
       P.ws_o[(hq * S + split) * kHeadDim + c] = acc;
@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
         acc += __ldcg(P.ws_o + (hq * S + sp) * kHeadDim + c) * wt;
       }
     }
-    P.out[hq * kHeadDim + c] = __float2half_rn(lsum > 0.f ? acc / lsum : 0.f);
+    P.out[hq * kHeadDim + c] = __half_as_ushort(__float2half_rn(lsum > 0.f ? acc / lsum : 0.f));
     if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
   }
   if (threadIdx.x == 0) P.ws_cnt[stream] = 0u;  // leave the workspace ready for the next call

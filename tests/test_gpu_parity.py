@@ -114,9 +114,9 @@ def test_append_rows_at_different_positions_and_out_of_range():
     xb = U.bits(x)
     k = c.keep
     for b, p in enumerate([0, 63, 64]):
-        ref = oracle.compress(xb[b][:, None, :], k, 64)
-        assert np.array_equal(bm[b, :, p], ref["bitmap"][:, 0, 0])
-        assert np.array_equal(vals[b, :, p * k:(p + 1) * k], ref["values"][:, 0, :k])
+        ref = oracle.compress(xb[b][None, :, None, :], k, 64)
+        assert np.array_equal(bm[b, :, p], ref["bitmap"][0, :, 0])
+        assert np.array_equal(vals[b, :, p * k:(p + 1) * k], ref["values"][0, :, :k])
     assert (bm[3] == 0).all() and (vals[3] == 0).all()
 
 

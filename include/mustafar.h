@@ -167,6 +167,36 @@ MUSTAFAR_API mustafar_status mustafar_dense_decode_attn(const void *q, int32_t n
                                            size_t workspace_bytes, int32_t num_splits,
                                            uint32_t *d_err, mustafar_stream_t stream);
 
+/* Bytes of device memory the library reserves (on every GPU that loads it, until the
+ * process exits) for mustafar_decode_attn_noalloc's split-K scratch. */
+#define MUSTAFAR_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Sparse decode attention that allocates nothing and takes no workspace.
+ * The paper has no counterpart to this call: it exists for callers that cannot hand the
+ * library a workspace - serving engines that reserve all device memory at start-up and pass
+ * kernels only their inputs and outputs, plugin interfaces whose host framework owns the
+ * allocator, or code that must not trigger a device allocation.  It computes exactly what
+ * mustafar_decode_attn computes (same arguments, minus workspace and workspace_bytes), with
+ * the split-K partial states and ticket counters kept in a fixed array of
+ * MUSTAFAR_NOALLOC_SCRATCH_BYTES inside the library instead.
+ *   - A call whose split plan needs more scratch than that (a very large batch x heads x
+ *     num_splits) is rejected with MUSTAFAR_ERR_WORKSPACE and a message.  On a 148-SM B200
+ *     the automatic plan (num_splits = 0) always fits: it needs at most about 4.9 MB, reached
+ *     with 16 q heads per kv head.
+ *   - The first call on each device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call shares the one array, on every stream: calls that overlap on the GPU race
+ *     and corrupt each other's results.  Each call first clears the ticket counters it uses.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ * Errors: as mustafar_decode_attn, plus WORKSPACE when the scratch is too small. */
+MUSTAFAR_API mustafar_status mustafar_decode_attn_noalloc(const void *q, int32_t num_q_heads,
+                                                          const mustafar_cache_t *k,
+                                                          const mustafar_cache_t *v,
+                                                          const int32_t *d_seq_len, int32_t max_len,
+                                                          float scale, void *out, float *lse,
+                                                          int32_t num_splits, uint32_t *d_err,
+                                                          mustafar_stream_t stream);
+
 /* The split count the automatic plan would use for this call (host query, for
  * benchmarks and tests).  Returns a value >= 1, or -1 on invalid shapes. */
 MUSTAFAR_API int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t head_dim,

@@ -26,6 +26,7 @@ ABI_SYMBOLS = (
     "mustafar_keep_count", "mustafar_cache_sizes", "mustafar_compress", "mustafar_append",
     "mustafar_decode_workspace_bytes", "mustafar_decode_attn", "mustafar_dense_decode_attn",
     "mustafar_decode_plan_splits", "mustafar_status_string", "mustafar_last_error", "mustafar_abi_version",
+    "mustafar_decode_attn_noalloc",
 )
 
 
@@ -68,6 +69,7 @@ def load() -> C.CDLL:
         "mustafar_status_string": (C.c_char_p, [i32]),
         "mustafar_last_error": (C.c_char_p, []),
         "mustafar_abi_version": (i32, []),
+        "mustafar_decode_attn_noalloc": (i32, [vp, i32, P(CacheT), P(CacheT), vp, i32, f32, vp, vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -220,4 +222,20 @@ def mustafar_dense_decode_attn(q: torch.Tensor, k_dense: torch.Tensor, v_dense: 
     _check(load().mustafar_dense_decode_attn(_ptr(q), q.shape[1], _ptr(k_dense), _ptr(v_dense), B, Hkv, d, cap,
                                              _ptr(seq_len), max_len, scale, _ptr(out), _ptr(lse), _ptr(workspace),
                                              workspace.numel(), num_splits, _ptr(err), _stream(stream)))
+    return out, lse
+
+
+def mustafar_decode_attn_noalloc(q: torch.Tensor, k: CompressedCache, v: CompressedCache, seq_len: torch.Tensor,
+                                 max_len: int, scale: float, out=None, lse=None, num_splits: int = 0, err=None,
+                                 stream=None, want_lse: bool = True):
+    """Sparse decode attention for callers that cannot allocate: same result as
+    ``mustafar_decode_attn``, with the split-K scratch kept in the library's own fixed device
+    array (shared by every call, so calls must not overlap on the GPU)."""
+    _cuda_f16(q, "q")
+    if not q.is_contiguous() or q.dim() != 3:
+        raise ValueError("q must be a contiguous [B, Hq, d] tensor")
+    out, lse = _decode_outputs(q, out, lse, want_lse)
+    _check(load().mustafar_decode_attn_noalloc(_ptr(q), q.shape[1], C.byref(k.struct), C.byref(v.struct),
+                                               _ptr(seq_len), max_len, scale, _ptr(out), _ptr(lse), num_splits,
+                                               _ptr(err), _stream(stream)))
     return out, lse

@@ -61,6 +61,8 @@ mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
 
 }  // namespace
 
+void set_last_error(const char *msg) { g_last_error = msg; }
+
 cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes) {
   static int done[64][32];  // bytes already granted per (device, kernel slot)
   int dev = 0;

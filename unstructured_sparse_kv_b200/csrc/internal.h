@@ -9,6 +9,9 @@
 
 namespace mustafar {
 
+// Record the message mustafar_last_error() returns on this thread.
+void set_last_error(const char *msg);
+
 // Set a kernel's dynamic shared-memory limit once per device.
 cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes);
 

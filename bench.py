@@ -311,12 +311,20 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=64 * 20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--suite", default=None, help="write the workload-shape suite (JSONL) to this path and exit")
+    ap.add_argument("--suite-parts", default="c1,c3,c4,sweep")
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="ncu case: build the workload, run this many eager steps (append K, append V, "
                          "attend) over the rotated caches, and exit without timing")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.suite:
+        import unstructured_sparse_kv_b200 as M
+        from unstructured_sparse_kv_b200 import suite
+        M.load()
+        suite.run(args.suite, measured_peak()[0], tuple(args.suite_parts.split(",")))
+        return 0
     if args.profile_launches > 0:
         import torch
         import unstructured_sparse_kv_b200 as M

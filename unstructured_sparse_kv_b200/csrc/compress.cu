@@ -9,7 +9,7 @@
 //   16-byte cp.async (16 threads per 256-byte row), each thread runs the top-k on its
 //   own row, writes its 16-byte bitmap, packs its kept values into a shared staging
 //   run, and the CTA writes the 128*k packed values with coalesced 16-byte stores.
-// append: one thread per (b, kv head) vector of the new token.
+// append: one warp per (b, kv head) vector of the new token.
 #include "internal.h"
 #include "select.cuh"
 
@@ -90,42 +90,72 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
   for (int i = (nvec << 3) + tid; i < n; i += kCompressThreads) vdst[i] = out_stage[i];
 }
 
-__global__ void __launch_bounds__(64)
+// append: one warp per (b, kv head) vector, for latency (a decode step appends only B*Hkv
+// vectors).  Lane l holds channels l, l+32, l+64, l+96, so a ballot over one of its four keys
+// is directly one bitmap word.  The same selection as topk_bitmap: binary search for the k-th
+// largest key T, then the keys equal to T are taken lowest channel first.
+__global__ void __launch_bounds__(128)
 append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int32_t *__restrict__ pos, int B,
               int H, int k, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
               uint32_t *__restrict__ err) {
-  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (v >= B * H) return;
   const int b = v / H, h = v - b * H;
   const int p = pos[b];
   if (p < 0 || p >= cap) {
-    if (err != nullptr) atomicOr(err, MUSTAFAR_DEVERR_POS_RANGE);
+    if (lane == 0 && err != nullptr) atomicOr(err, MUSTAFAR_DEVERR_POS_RANGE);
     return;
   }
   const uint16_t *src = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
-  uint32_t raw[64];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src) + j);
-    raw[4 * j + 0] = q.x;
-    raw[4 * j + 1] = q.y;
-    raw[4 * j + 2] = q.z;
-    raw[4 * j + 3] = q.w;
-  }
-  uint32_t bm[kWords];
-  topk_bitmap(raw, k, bm);
-  const int64_t stream = static_cast<int64_t>(b) * H + h;
-  reinterpret_cast<uint4 *>(bitmap)[stream * cap + p] = make_uint4(bm[0], bm[1], bm[2], bm[3]);
-  uint16_t *dst = values + (stream * cap + p) * static_cast<int64_t>(k);
-  int jj = 0;
+  uint32_t raw[kWords], key[kWords];
 #pragma unroll
   for (int w = 0; w < kWords; ++w) {
-    uint32_t m = bm[w];
-    while (m && jj < k) {
-      const int ch = 32 * w + __ffs(m) - 1;
-      m &= m - 1;
-      dst[jj++] = __ldg(src + ch);
+    raw[w] = src[32 * w + lane];
+    key[w] = raw[w] & 0x7FFFu;
+  }
+  auto count_ge = [&](uint32_t t) {
+    int n = 0;
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) n += __popc(__ballot_sync(0xffffffffu, key[w] >= t));
+    return n;
+  };
+  uint32_t T = 0;
+#pragma unroll 1
+  for (int bit = 14; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    if (count_ge(cand) >= k) T = cand;
+  }
+  uint32_t bm[kWords];
+  int n_gt = 0;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    bm[w] = __ballot_sync(0xffffffffu, key[w] > T);
+    n_gt += __popc(bm[w]);
+  }
+  int need = k - n_gt;  // keys equal to T that survive, lowest channels first
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    uint32_t e = __ballot_sync(0xffffffffu, key[w] == T);
+    while (e != 0u && need > 0) {
+      const uint32_t low = e & (0u - e);
+      bm[w] |= low;
+      e ^= low;
+      --need;
     }
+  }
+  const int64_t stream = static_cast<int64_t>(b) * H + h;
+  if (lane < kWords) {
+    const uint32_t word = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
+    bitmap[(stream * cap + p) * kWords + lane] = word;
+  }
+  uint16_t *dst = values + (stream * cap + p) * static_cast<int64_t>(k);
+  const uint32_t below = (1u << lane) - 1u;
+  int prefix = 0;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    if ((bm[w] >> lane) & 1u) dst[prefix + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[w]);
+    prefix += __popc(bm[w]);
   }
 }
 
@@ -145,10 +175,10 @@ cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t s
 
 cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H, int k,
                           int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err, cudaStream_t stream) {
-  const int n = B * H;
-  const int threads = 64;
-  append_kernel<<<(n + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, k, cap, bitmap,
-                                                                     values, err);
+  const int warps = B * H;
+  const int threads = 128;  // 4 vectors per CTA
+  append_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, k, cap,
+                                                                              bitmap, values, err);
   return cudaGetLastError();
 }
 

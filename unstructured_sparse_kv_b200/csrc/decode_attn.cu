@@ -14,12 +14,16 @@
 //   range: a cp.async ring (NSTAGE deep) stages the chunk's compressed bytes (16 bitmap
 //   rows + 16*k packed values, for K and for V) in the warp's own shared memory, so the
 //   loop needs no CTA barrier.
-// * expansion: lanes 0-15 rebuild the 16 K rows and lanes 16-31 the 16 V rows of the chunk
-//   as dense fp16 rows in shared memory, walking each row's set bits (__ffs) and scattering
-//   its packed values in order.
-// * the group's logits S = Q K~^T (G q heads padded to 16 rows x 16 tokens x 128 channels)
-//   and O += P V~ run as mma.sync m16n8k16 (fp16 in, fp32 accumulate) fed by ldmatrix;
-//   softmax is online (running max / sum per row in the log2 domain).
+// * expansion: lanes 0-15 rebuild the chunk's 16 K rows and lanes 16-31 its 16 V rows as
+//   channel-major fp16 tiles T[channel][token] in shared memory (one lane per token row:
+//   walk the row's set bits from the top of each word with a leading-one search and
+//   scatter the packed values, which are read back to front).  The channel-major layout puts
+//   a lane's scatter in the bank chosen by its token, so concurrent scatters rarely collide;
+//   a 16-byte gap after every 4 channel rows keeps the 8-row ldmatrix reads conflict-free.
+// * S = Q K~^T: the G q heads (padded to 16 rows) x 16 tokens x 128 channels, mma.sync
+//   m16n8k16 (fp16 in, fp32 accumulate); online softmax per head in the log2 domain;
+//   O^T += V~^T P^T with the 128 channels as the M dimension (8 m-tiles) and the heads as N,
+//   so the fp32 accumulator is 128 x 8 (32 registers per lane) for G <= 8.
 // * warps merge in shared memory; with splits > 1 each CTA writes its (m, l, o) partial to
 //   the workspace and the last CTA of the stream (atomic ticket, no spin-wait) merges all
 //   splits in a fixed order and writes out / lse.
@@ -33,6 +37,11 @@ namespace mustafar {
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr float kNegInf = -INFINITY;
+// channel-major tile of one side: 128 channel rows x 16 tokens (32 B), 16-byte gap per 4 rows
+constexpr int kTTileBytes = kHeadDim * 32 + (kHeadDim / 4) * 16;  // 4608
+constexpr int kTStep = 16 * 32 + 4 * 16;                           // bytes per 16 channels (576)
+
+__device__ __forceinline__ uint32_t ttile_off(int ch, int tok) { return ch * 32 + (ch >> 2) * 16 + tok * 2; }
 
 template <bool SPARSE>
 __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t stream, int c, uint8_t *stage,
@@ -68,30 +77,46 @@ __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t strea
   }
 }
 
-// Rebuild the chunk's 16 K rows (lanes 0-15) and 16 V rows (lanes 16-31) as dense fp16.
+// Scatter the set bits of one bitmap word (channels 32w + p) of token column `tok`, highest
+// channel first; `vp` points at the word's last packed value and walks backwards.
+__device__ __forceinline__ void walk_word(uint32_t m, uint8_t *wbase, const uint16_t *vp) {
+  while (m) {
+    const int p = 31 - __clz(m);
+    m &= ~(1u << p);
+    *reinterpret_cast<uint16_t *>(wbase + p * 32 + (p >> 2) * 16) = *vp--;
+  }
+}
+
+// Rebuild the chunk's 16 K rows (lanes 0-15) and 16 V rows (lanes 16-31) as channel-major tiles.
 __device__ __forceinline__ void expand_chunk(const DecodeParams &P, const uint8_t *stage, uint8_t *dense, int lane,
                                              int t0, int L) {
-  const int side = lane >> 4, r = lane & 15;
-  uint8_t *row = dense + side * kTileBytes + r * kRowBytes;
+  const int side = lane >> 4, t = lane & 15;
+  uint8_t *tile = dense + side * kTTileBytes;
+  // zero the 128 x 32 B data rows of this side: 16 lanes x 8 rows x 2 halves
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-  for (int j = 0; j < 16; ++j) reinterpret_cast<uint4 *>(row)[j] = z;
-  if (t0 + r < L) {
-    const uint4 bm = *reinterpret_cast<const uint4 *>(stage + side * 256 + r * 16);
+  for (int i = 0; i < 8; ++i) {
+    const int ch = t * 8 + i;
+    uint8_t *row = tile + ch * 32 + (ch >> 2) * 16;
+    reinterpret_cast<uint4 *>(row)[0] = z;
+    reinterpret_cast<uint4 *>(row)[1] = z;
+  }
+  __syncwarp();
+  if (t0 + t < L) {
+    const uint4 bm = *reinterpret_cast<const uint4 *>(stage + side * 256 + t * 16);
     const int kk = side ? P.keep_v : P.keep_k;
-    const uint16_t *vals = reinterpret_cast<const uint16_t *>(stage + 512 + side * 32 * P.keep_k) + r * kk;
-    uint16_t *drow = reinterpret_cast<uint16_t *>(row);
-    const uint32_t words[4] = {bm.x, bm.y, bm.z, bm.w};
-    int j = 0;
-#pragma unroll
-    for (int w = 0; w < kWords; ++w) {
-      uint32_t m = words[w];
-      while (m && j < kk) {  // a bitmap never holds more than k bits; the bound only guards the buffer
-        const int ch = 32 * w + __ffs(m) - 1;
-        m &= m - 1;
-        drow[ch] = vals[j++];
-      }
-    }
+    const uint16_t *vals = reinterpret_cast<const uint16_t *>(stage + 512 + side * 32 * P.keep_k) + t * kk;
+    uint8_t *col = tile + t * 2;
+    // words from the top: channels 96..127, 64..95, 32..63, 0..31; values read back to front
+    const uint16_t *vp = vals + kk - 1;
+    const uint32_t w3 = bm.w, w2 = bm.z, w1 = bm.y, w0 = bm.x;
+    walk_word(w3, col + 96 * 32 + 24 * 16, vp);
+    vp -= __popc(w3);
+    walk_word(w2, col + 64 * 32 + 16 * 16, vp);
+    vp -= __popc(w2);
+    walk_word(w1, col + 32 * 32 + 8 * 16, vp);
+    vp -= __popc(w1);
+    walk_word(w0, col, vp);
   }
 }
 
@@ -132,9 +157,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     }
   }
 
-  float o[16][4];
+  // O^T accumulators: m-tile mt covers channels 16mt..16mt+15; [0]/[1] = heads 2q/2q+1 at channel
+  // 16mt+g, [2]/[3] the same heads at channel 16mt+g+8.  oh: heads 8+2q, 8+2q+1 (G > 8).
+  float ot[8][4];
+  float oh[HIROWS ? 8 : 1][4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  for (int i = 0; i < 8; ++i) ot[i][0] = ot[i][1] = ot[i][2] = ot[i][3] = 0.f;
+#pragma unroll
+  for (int i = 0; i < (HIROWS ? 8 : 1); ++i) oh[i][0] = oh[i][1] = oh[i][2] = oh[i][3] = 0.f;
   float m_run[2] = {kNegInf, kNegInf};
   float l_run[2] = {0.f, 0.f};
 
@@ -144,10 +174,18 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     cp_async_commit();
   }
 
-  // per-lane ldmatrix address offsets
-  const int mat = lane >> 3;
-  const uint32_t k_off = (((mat >> 1) << 3) + (lane & 7)) * kRowBytes + ((mat & 1) << 4);
-  const uint32_t v_off = (((mat & 1) << 3) + (lane & 7)) * kRowBytes + ((mat >> 1) << 4);
+  // per-lane ldmatrix row addresses (matrix = lane / 8, row = lane % 8)
+  const int mat = lane >> 3, r8 = lane & 7;
+  uint32_t k_off, v_off;
+  constexpr uint32_t kStepK = SPARSE ? kTStep : 32;  // bytes between 16-channel steps
+  if constexpr (SPARSE) {
+    // channel rows (mat & 1)*8 + r8 of each 16-channel step, token half mat >> 1
+    const int ch = (mat & 1) * 8 + r8;
+    k_off = v_off = ttile_off(ch, 0) + (mat >> 1) * 16;
+  } else {
+    // token rows (mat >> 1)*8 + r8, channel half (mat & 1) of each 16-channel step
+    k_off = v_off = (((mat >> 1) << 3) + r8) * kRowBytes + ((mat & 1) << 4);
+  }
 
 #pragma unroll 1
   for (int i = 0; i < my_n; ++i) {
@@ -168,7 +206,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
       expand_chunk(P, stage, dense, lane, t0, L);
       __syncwarp();
       ktile = dense;
-      vtile = dense + kTileBytes;
+      vtile = dense + kTTileBytes;
     } else {
       ktile = stage;
       vtile = stage + kTileBytes;
@@ -182,12 +220,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * 32);
+      if constexpr (SPARSE)
+        ldmatrix_x4_trans(b0, b1, b2, b3, kaddr + ks * kStepK);
+      else
+        ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * kStepK);
       mma_f16_16816(s[0], qa[ks], b0, b1);
       mma_f16_16816(s[1], qa[ks], b2, b3);
     }
 
-    // scale into the log2 domain, mask tokens >= L, online softmax per row
+    // scale into the log2 domain, mask tokens >= L, online softmax per row (= q head)
     float mx[2] = {kNegInf, kNegInf};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -222,29 +263,47 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     }
     l_run[0] = l_run[0] * alpha[0] + psum[0];
     l_run[1] = l_run[1] * alpha[1] + psum[1];
-    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || (HIROWS && alpha[1] != 1.f))) {
+      // the O^T columns this lane holds are heads 2q and 2q+1, whose factors live in lanes 8q and 8q+4
+      const float a_lo = __shfl_sync(0xffffffffu, alpha[0], 8 * qq);
+      const float a_hi = __shfl_sync(0xffffffffu, alpha[0], 8 * qq + 4);
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        o[nt][0] *= alpha[0];
-        o[nt][1] *= alpha[0];
-        o[nt][2] *= alpha[1];
-        o[nt][3] *= alpha[1];
+      for (int mt = 0; mt < 8; ++mt) {
+        ot[mt][0] *= a_lo;
+        ot[mt][1] *= a_hi;
+        ot[mt][2] *= a_lo;
+        ot[mt][3] *= a_hi;
+      }
+      if constexpr (HIROWS) {
+        const float b_lo = __shfl_sync(0xffffffffu, alpha[1], 8 * qq);
+        const float b_hi = __shfl_sync(0xffffffffu, alpha[1], 8 * qq + 4);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          oh[mt][0] *= b_lo;
+          oh[mt][1] *= b_hi;
+          oh[mt][2] *= b_lo;
+          oh[mt][3] *= b_hi;
+        }
       }
     }
-    uint32_t pa[4];
-    pa[0] = pack_half2(s[0][0], s[0][1]);
-    pa[1] = pack_half2(s[0][2], s[0][3]);
-    pa[2] = pack_half2(s[1][0], s[1][1]);
-    pa[3] = pack_half2(s[1][2], s[1][3]);
+    // P^T as the B operand: the S accumulator layout (row = head, columns = tokens) is exactly the
+    // m16n8k16 B layout for K = tokens, N = heads
+    const uint32_t pb0 = pack_half2(s[0][0], s[0][1]);
+    const uint32_t pb1 = pack_half2(s[1][0], s[1][1]);
+    const uint32_t pc0 = HIROWS ? pack_half2(s[0][2], s[0][3]) : 0u;
+    const uint32_t pc1 = HIROWS ? pack_half2(s[1][2], s[1][3]) : 0u;
 
-    // O += P V~ : 16 n-tiles of 8 channels
+    // O^T += V~^T P^T : 8 m-tiles of 16 channels
     const uint32_t vaddr = smem_addr(vtile) + v_off;
 #pragma unroll
-    for (int ntp = 0; ntp < 8; ++ntp) {
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4_trans(b0, b1, b2, b3, vaddr + ntp * 32);
-      mma_f16_16816(o[2 * ntp], pa, b0, b1);
-      mma_f16_16816(o[2 * ntp + 1], pa, b2, b3);
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t a[4];
+      if constexpr (SPARSE)
+        ldmatrix_x4(a[0], a[1], a[2], a[3], vaddr + mt * kStepK);
+      else
+        ldmatrix_x4_trans(a[0], a[1], a[2], a[3], vaddr + mt * kStepK);
+      mma_f16_16816(ot[mt], a, pb0, pb1);
+      if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
     }
     __syncwarp();
   }
@@ -271,13 +330,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
       sm_l[warp * 16 + gq + 8] = l_run[1];
     }
   }
+  {
+    const int h0 = 2 * qq, h1 = 2 * qq + 1;
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt) {
-    const int ch = nt * 8 + 2 * qq;
-    if (gq < G)
-      *reinterpret_cast<float2 *>(sm_o + (warp * G + gq) * kHeadDim + ch) = make_float2(o[nt][0], o[nt][1]);
-    if (HIROWS && gq + 8 < G)
-      *reinterpret_cast<float2 *>(sm_o + (warp * G + gq + 8) * kHeadDim + ch) = make_float2(o[nt][2], o[nt][3]);
+    for (int mt = 0; mt < 8; ++mt) {
+      const int ch = mt * 16 + gq;
+      if (h0 < G) {
+        sm_o[(warp * G + h0) * kHeadDim + ch] = ot[mt][0];
+        sm_o[(warp * G + h0) * kHeadDim + ch + 8] = ot[mt][2];
+      }
+      if (h1 < G) {
+        sm_o[(warp * G + h1) * kHeadDim + ch] = ot[mt][1];
+        sm_o[(warp * G + h1) * kHeadDim + ch + 8] = ot[mt][3];
+      }
+      if constexpr (HIROWS) {
+        if (h0 + 8 < G) {
+          sm_o[(warp * G + h0 + 8) * kHeadDim + ch] = oh[mt][0];
+          sm_o[(warp * G + h0 + 8) * kHeadDim + ch + 8] = oh[mt][2];
+        }
+        if (h1 + 8 < G) {
+          sm_o[(warp * G + h1 + 8) * kHeadDim + ch] = oh[mt][1];
+          sm_o[(warp * G + h1 + 8) * kHeadDim + ch + 8] = oh[mt][3];
+        }
+      }
+    }
   }
   __syncthreads();
 
@@ -441,9 +517,9 @@ cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int kee
   int nstage, stage_bytes, warp_bytes;
   if (sparse) {
     stage_bytes = 512 + 32 * (keep_k + keep_v);
-    nstage = (kWarpSmemTarget - 2 * kTileBytes) / stage_bytes;
+    nstage = (kWarpSmemTarget - 2 * kTTileBytes) / stage_bytes;
     nstage = nstage < 2 ? 2 : (nstage > 4 ? 4 : nstage);
-    warp_bytes = nstage * stage_bytes + 2 * kTileBytes;
+    warp_bytes = nstage * stage_bytes + 2 * kTTileBytes;
   } else {
     stage_bytes = 2 * kTileBytes;
     nstage = 3;

@@ -15,11 +15,11 @@
 //   rows + 16*k packed values, for K and for V) in the warp's own shared memory, so the
 //   loop needs no CTA barrier.
 // * expansion: lanes 0-15 rebuild the chunk's 16 K rows and lanes 16-31 its 16 V rows as
-//   channel-major fp16 tiles T[channel][token] in shared memory (one lane per token row:
-//   walk the row's set bits from the top of each word with a leading-one search and
-//   scatter the packed values, which are read back to front).  The channel-major layout puts
-//   a lane's scatter in the bank chosen by its token, so concurrent scatters rarely collide;
-//   a 16-byte gap after every 4 channel rows keeps the 8-row ldmatrix reads conflict-free.
+//   channel-major fp16 tiles T[channel][token] in shared memory (one lane per token row,
+//   walking the row's four bitmap words together: isolate the lowest set bit, find its
+//   position with a leading-one count, scatter the next packed value).  The channel-major
+//   layout puts a lane's scatter near the bank chosen by its token, so concurrent scatters
+//   rarely collide; a 48-byte channel-row stride keeps the 8-row ldmatrix reads conflict-free.
 // * S = Q K~^T: the G q heads (padded to 16 rows) x 16 tokens x 128 channels, mma.sync
 //   m16n8k16 (fp16 in, fp32 accumulate); online softmax per head in the log2 domain;
 //   O^T += V~^T P^T with the 128 channels as the M dimension (8 m-tiles) and the heads as N,
@@ -37,11 +37,14 @@ namespace mustafar {
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr float kNegInf = -INFINITY;
-// channel-major tile of one side: 128 channel rows x 16 tokens (32 B), 16-byte gap per 4 rows
-constexpr int kTTileBytes = kHeadDim * 32 + (kHeadDim / 4) * 16;  // 4608
-constexpr int kTStep = 16 * 32 + 4 * 16;                           // bytes per 16 channels (576)
+// channel-major tile of one side: 128 channel rows x 16 tokens (32 B) at a 48-byte row stride.
+// Rows r..r+7 then start in 8 different 16-byte bank groups (3r mod 8), so ldmatrix reads of
+// 8 rows are conflict-free, and a scatter address is one multiply-add.
+constexpr int kTRowBytes = 48;
+constexpr int kTTileBytes = kHeadDim * kTRowBytes;  // 6144
+constexpr int kTStep = 16 * kTRowBytes;             // bytes per 16 channels (768)
 
-__device__ __forceinline__ uint32_t ttile_off(int ch, int tok) { return ch * 32 + (ch >> 2) * 16 + tok * 2; }
+__device__ __forceinline__ uint32_t ttile_off(int ch, int tok) { return ch * kTRowBytes + tok * 2; }
 
 template <bool SPARSE>
 __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t stream, int c, uint8_t *stage,
@@ -77,46 +80,69 @@ __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t strea
   }
 }
 
-// Scatter the set bits of one bitmap word (channels 32w + p) of token column `tok`, highest
-// channel first; `vp` points at the word's last packed value and walks backwards.
-__device__ __forceinline__ void walk_word(uint32_t m, uint8_t *wbase, const uint16_t *vp) {
-  while (m) {
-    const int p = 31 - __clz(m);
-    m &= ~(1u << p);
-    *reinterpret_cast<uint16_t *>(wbase + p * 32 + (p >> 2) * 16) = *vp--;
-  }
+// Predicated 16-bit shared-memory load and store (no branch: the walk of four words stays
+// straight-line, so the four loads of an iteration are in flight together).
+__device__ __forceinline__ uint32_t lds16_if(uint32_t pred, uint32_t addr) {
+  uint32_t v = 0;
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b16 h;\n setp.ne.u32 p, %1, 0;\n mov.b16 h, 0;\n @p ld.shared.b16 h, [%2];\n"
+      " cvt.u32.u16 %0, h;\n}\n"
+      : "=r"(v)
+      : "r"(pred), "r"(addr)
+      : "memory");
+  return v;
+}
+__device__ __forceinline__ void sts16_if(uint32_t pred, uint32_t addr, uint32_t v) {
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b16 h;\n setp.ne.u32 p, %0, 0;\n cvt.u16.u32 h, %2;\n @p st.shared.b16 [%1], h;\n}\n" ::"r"(
+          pred),
+      "r"(addr), "r"(v)
+      : "memory");
 }
 
 // Rebuild the chunk's 16 K rows (lanes 0-15) and 16 V rows (lanes 16-31) as channel-major tiles.
+// Each lane walks the four bitmap words of its row together (four independent chains): per step,
+// isolate the lowest remaining set bit of each word, locate its channel row with a leading-zero
+// count, load the next packed value of that word and store it at (channel, token).
 __device__ __forceinline__ void expand_chunk(const DecodeParams &P, const uint8_t *stage, uint8_t *dense, int lane,
                                              int t0, int L) {
   const int side = lane >> 4, t = lane & 15;
   uint8_t *tile = dense + side * kTTileBytes;
-  // zero the 128 x 32 B data rows of this side: 16 lanes x 8 rows x 2 halves
+  // zero the 32 data bytes of the 128 channel rows: lane t clears rows t, t+16, ..., t+112
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int ch = t * 8 + i;
-    uint8_t *row = tile + ch * 32 + (ch >> 2) * 16;
-    reinterpret_cast<uint4 *>(row)[0] = z;
-    reinterpret_cast<uint4 *>(row)[1] = z;
+    uint4 *row = reinterpret_cast<uint4 *>(tile + (t + 16 * i) * kTRowBytes);
+    row[0] = z;
+    row[1] = z;
   }
   __syncwarp();
   if (t0 + t < L) {
     const uint4 bm = *reinterpret_cast<const uint4 *>(stage + side * 256 + t * 16);
     const int kk = side ? P.keep_v : P.keep_k;
-    const uint16_t *vals = reinterpret_cast<const uint16_t *>(stage + 512 + side * 32 * P.keep_k) + t * kk;
-    uint8_t *col = tile + t * 2;
-    // words from the top: channels 96..127, 64..95, 32..63, 0..31; values read back to front
-    const uint16_t *vp = vals + kk - 1;
-    const uint32_t w3 = bm.w, w2 = bm.z, w1 = bm.y, w0 = bm.x;
-    walk_word(w3, col + 96 * 32 + 24 * 16, vp);
-    vp -= __popc(w3);
-    walk_word(w2, col + 64 * 32 + 16 * 16, vp);
-    vp -= __popc(w2);
-    walk_word(w1, col + 32 * 32 + 8 * 16, vp);
-    vp -= __popc(w1);
-    walk_word(w0, col, vp);
+    const uint32_t vals = smem_addr(stage + 512 + side * 32 * P.keep_k) + 2 * t * kk;
+    uint32_t m0 = bm.x, m1 = bm.y, m2 = bm.z, m3 = bm.w;
+    const uint32_t n0 = __popc(m0), n1 = __popc(m1), n2 = __popc(m2);
+    uint32_t v0 = vals, v1 = vals + 2 * n0, v2 = v1 + 2 * n1, v3 = v2 + 2 * n2;
+    // destination of channel row 31 of each word in this lane's token column
+    const uint32_t col = smem_addr(tile) + t * 2 + 31 * kTRowBytes;
+    const uint32_t d0 = col, d1 = col + 32 * kTRowBytes, d2 = col + 64 * kTRowBytes, d3 = col + 96 * kTRowBytes;
+    while (m0 | m1 | m2 | m3) {
+      const uint32_t l0 = m0 & (0u - m0), l1 = m1 & (0u - m1), l2 = m2 & (0u - m2), l3 = m3 & (0u - m3);
+      m0 ^= l0;
+      m1 ^= l1;
+      m2 ^= l2;
+      m3 ^= l3;
+      const uint32_t x0 = lds16_if(l0, v0), x1 = lds16_if(l1, v1), x2 = lds16_if(l2, v2), x3 = lds16_if(l3, v3);
+      sts16_if(l0, d0 - __clz(l0) * kTRowBytes, x0);
+      sts16_if(l1, d1 - __clz(l1) * kTRowBytes, x1);
+      sts16_if(l2, d2 - __clz(l2) * kTRowBytes, x2);
+      sts16_if(l3, d3 - __clz(l3) * kTRowBytes, x3);
+      v0 += l0 ? 2u : 0u;
+      v1 += l1 ? 2u : 0u;
+      v2 += l2 ? 2u : 0u;
+      v3 += l3 ? 2u : 0u;
+    }
   }
 }
 

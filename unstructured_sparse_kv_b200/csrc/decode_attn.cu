@@ -14,16 +14,17 @@
 //   range: a cp.async ring (NSTAGE deep) stages the chunk's compressed bytes (16 bitmap
 //   rows + 16*k packed values, for K and for V) in the warp's own shared memory, so the
 //   loop needs no CTA barrier.
-// * expansion: lanes 0-15 rebuild the chunk's 16 K rows and lanes 16-31 its 16 V rows as
-//   channel-major fp16 tiles T[channel][token] in shared memory (one lane per token row,
-//   walking the row's four bitmap words together: isolate the lowest set bit, find its
-//   position with a leading-one count, scatter the next packed value).  The channel-major
-//   layout puts a lane's scatter near the bank chosen by its token, so concurrent scatters
-//   rarely collide; a 48-byte channel-row stride keeps the 8-row ldmatrix reads conflict-free.
-// * S = Q K~^T: the G q heads (padded to 16 rows) x 16 tokens x 128 channels, mma.sync
-//   m16n8k16 (fp16 in, fp32 accumulate); online softmax per head in the log2 domain;
-//   O^T += V~^T P^T with the 128 channels as the M dimension (8 m-tiles) and the heads as N,
-//   so the fp32 accumulator is 128 x 8 (32 registers per lane) for G <= 8.
+// * S = Q K~^T and O^T += V~^T P^T run as mma.sync m16n8k16 (fp16 in, fp32 accumulate):
+//   S has the G q heads (padded to 16) as M and the 16 tokens as N; O^T has the 128
+//   channels as M (8 m-tiles), the heads as N and the tokens as K, so the fp32 accumulator
+//   is 128 x 8 (32 registers per lane) for G <= 8.  Online softmax per head, log2 domain.
+// * no dense tile is ever built: each lane expands, straight into its mma fragment
+//   registers, exactly the (token, channel) elements the fragment layouts give it, with one
+//   predicated 16-bit shared load per channel (the bit of the bitmap is the predicate; the
+//   value pointer advances past each kept value).  The contraction index is permuted so
+//   that a lane's channels are one contiguous bitmap word (K: 32 channels of each of its
+//   2 tokens) or half-word (V: 16 channels of each of its 4 tokens); Q's fragments use the
+//   same permutation and the output columns are put back in order when the warps merge.
 // * warps merge in shared memory; with splits > 1 each CTA writes its (m, l, o) partial to
 //   the workspace and the last CTA of the stream (atomic ticket, no spin-wait) merges all
 //   splits in a fixed order and writes out / lse.
@@ -37,14 +38,6 @@ namespace mustafar {
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr float kNegInf = -INFINITY;
-// channel-major tile of one side: 128 channel rows x 16 tokens (32 B) at a 48-byte row stride.
-// Rows r..r+7 then start in 8 different 16-byte bank groups (3r mod 8), so ldmatrix reads of
-// 8 rows are conflict-free, and a scatter address is one multiply-add.
-constexpr int kTRowBytes = 48;
-constexpr int kTTileBytes = kHeadDim * kTRowBytes;  // 6144
-constexpr int kTStep = 16 * kTRowBytes;             // bytes per 16 channels (768)
-
-__device__ __forceinline__ uint32_t ttile_off(int ch, int tok) { return ch * kTRowBytes + tok * 2; }
 
 template <bool SPARSE>
 __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t stream, int c, uint8_t *stage,
@@ -80,70 +73,46 @@ __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t strea
   }
 }
 
-// Predicated 16-bit shared-memory load and store (no branch: the walk of four words stays
-// straight-line, so the four loads of an iteration are in flight together).
-__device__ __forceinline__ uint32_t lds16_if(uint32_t pred, uint32_t addr) {
-  uint32_t v = 0;
+// x = (bits & MASK) ? the fp16 at shared address ra : 0; ra advances past a loaded value.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t take(uint32_t bits, uint32_t &ra) {
+  uint32_t x = 0;
   asm volatile(
-      "{\n .reg .pred p;\n .reg .b16 h;\n setp.ne.u32 p, %1, 0;\n mov.b16 h, 0;\n @p ld.shared.b16 h, [%2];\n"
-      " cvt.u32.u16 %0, h;\n}\n"
-      : "=r"(v)
-      : "r"(pred), "r"(addr)
+      "{\n .reg .pred p;\n .reg .b32 t;\n and.b32 t, %2, %3;\n setp.ne.u32 p, t, 0;\n"
+      " @p ld.shared.u16 %0, [%1];\n @p add.u32 %1, %1, 2;\n}\n"
+      : "+r"(x), "+r"(ra)
+      : "r"(bits), "n"(MASK)
       : "memory");
-  return v;
-}
-__device__ __forceinline__ void sts16_if(uint32_t pred, uint32_t addr, uint32_t v) {
-  asm volatile(
-      "{\n .reg .pred p;\n .reg .b16 h;\n setp.ne.u32 p, %0, 0;\n cvt.u16.u32 h, %2;\n @p st.shared.b16 [%1], h;\n}\n" ::"r"(
-          pred),
-      "r"(addr), "r"(v)
-      : "memory");
+  return x;
 }
 
-// Rebuild the chunk's 16 K rows (lanes 0-15) and 16 V rows (lanes 16-31) as channel-major tiles.
-// Each lane walks the four bitmap words of its row together (four independent chains): per step,
-// isolate the lowest remaining set bit of each word, locate its channel row with a leading-zero
-// count, load the next packed value of that word and store it at (channel, token).
-__device__ __forceinline__ void expand_chunk(const DecodeParams &P, const uint8_t *stage, uint8_t *dense, int lane,
-                                             int t0, int L) {
-  const int side = lane >> 4, t = lane & 15;
-  uint8_t *tile = dense + side * kTTileBytes;
-  // zero the 32 data bytes of the 128 channel rows: lane t clears rows t, t+16, ..., t+112
-  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint4 *row = reinterpret_cast<uint4 *>(tile + (t + 16 * i) * kTRowBytes);
-    row[0] = z;
-    row[1] = z;
+// Expand the 32 channels of one bitmap word into 16 packed fp16 pairs (channels 2i, 2i+1).
+template <int I = 0>
+__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t (&out)[16]) {
+  if constexpr (I < 16) {
+    const uint32_t lo = take<(1u << (2 * I))>(bits, ra);
+    const uint32_t hi = take<(1u << (2 * I + 1))>(bits, ra);
+    out[I] = __byte_perm(lo, hi, 0x5410);
+    expand_word<I + 1>(bits, ra, out);
   }
-  __syncwarp();
-  if (t0 + t < L) {
-    const uint4 bm = *reinterpret_cast<const uint4 *>(stage + side * 256 + t * 16);
-    const int kk = side ? P.keep_v : P.keep_k;
-    const uint32_t vals = smem_addr(stage + 512 + side * 32 * P.keep_k) + 2 * t * kk;
-    uint32_t m0 = bm.x, m1 = bm.y, m2 = bm.z, m3 = bm.w;
-    const uint32_t n0 = __popc(m0), n1 = __popc(m1), n2 = __popc(m2);
-    uint32_t v0 = vals, v1 = vals + 2 * n0, v2 = v1 + 2 * n1, v3 = v2 + 2 * n2;
-    // destination of channel row 31 of each word in this lane's token column
-    const uint32_t col = smem_addr(tile) + t * 2 + 31 * kTRowBytes;
-    const uint32_t d0 = col, d1 = col + 32 * kTRowBytes, d2 = col + 64 * kTRowBytes, d3 = col + 96 * kTRowBytes;
-    while (m0 | m1 | m2 | m3) {
-      const uint32_t l0 = m0 & (0u - m0), l1 = m1 & (0u - m1), l2 = m2 & (0u - m2), l3 = m3 & (0u - m3);
-      m0 ^= l0;
-      m1 ^= l1;
-      m2 ^= l2;
-      m3 ^= l3;
-      const uint32_t x0 = lds16_if(l0, v0), x1 = lds16_if(l1, v1), x2 = lds16_if(l2, v2), x3 = lds16_if(l3, v3);
-      sts16_if(l0, d0 - __clz(l0) * kTRowBytes, x0);
-      sts16_if(l1, d1 - __clz(l1) * kTRowBytes, x1);
-      sts16_if(l2, d2 - __clz(l2) * kTRowBytes, x2);
-      sts16_if(l3, d3 - __clz(l3) * kTRowBytes, x3);
-      v0 += l0 ? 2u : 0u;
-      v1 += l1 ? 2u : 0u;
-      v2 += l2 ? 2u : 0u;
-      v3 += l3 ? 2u : 0u;
-    }
+}
+
+// Expand the 16 channels of a half word (bits 0..15 of `bits`) into 16 separate fp16 values.
+template <int I = 0>
+__device__ __forceinline__ void expand_half(uint32_t bits, uint32_t ra, uint32_t (&out)[16]) {
+  if constexpr (I < 16) {
+    out[I] = take<(1u << I)>(bits, ra);
+    expand_half<I + 1>(bits, ra, out);
   }
+}
+
+__device__ __forceinline__ uint32_t pick(const uint4 &w, int i) {
+  return i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
+}
+
+// popcount of the bitmap words below word i
+__device__ __forceinline__ uint32_t prefix_words(const uint4 &w, int i) {
+  return (i > 0 ? __popc(w.x) : 0) + (i > 1 ? __popc(w.y) : 0) + (i > 2 ? __popc(w.z) : 0);
 }
 
 template <bool SPARSE, int NSTAGE, bool HIROWS>
@@ -165,9 +134,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
   const int64_t stream = static_cast<int64_t>(b) * P.Hkv + g;
 
   uint8_t *wbase = smem + warp * P.warp_bytes;
-  uint8_t *dense = wbase + NSTAGE * P.stage_bytes;  // sparse only
 
-  // Q A-fragments (rows = q heads of the group, zero beyond G), 8 k-steps of 16 channels
+  // Q A-fragments (rows = q heads of the group, zero beyond G), 8 k-steps.  Sparse path: k-step
+  // ks, fragment column 2q+e is channel 32q+4ks+e and column 2q+8+e is 32q+4ks+2+e (the
+  // permutation that gives lane q the 32 channels of bitmap word q); dense path: natural order.
   const int gq = lane >> 2, qq = lane & 3;
   uint32_t qa[8][4];
   {
@@ -175,16 +145,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     const bool r0 = gq < G, r1 = HIROWS && (gq + 8 < G);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const int col = ks * 16 + 2 * qq;
-      qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + col) : 0u;
-      qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + col) : 0u;
-      qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + col + 8) : 0u;
-      qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + col + 8) : 0u;
+      const int c0 = SPARSE ? 32 * qq + 4 * ks : ks * 16 + 2 * qq;
+      const int c1 = SPARSE ? c0 + 2 : c0 + 8;
+      qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + c0) : 0u;
+      qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + c0) : 0u;
+      qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + c1) : 0u;
+      qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + c1) : 0u;
     }
   }
 
-  // O^T accumulators: m-tile mt covers channels 16mt..16mt+15; [0]/[1] = heads 2q/2q+1 at channel
-  // 16mt+g, [2]/[3] the same heads at channel 16mt+g+8.  oh: heads 8+2q, 8+2q+1 (G > 8).
+  // O^T accumulators, m-tile mt.  Sparse: rows g / g+8 are channels 16g+2mt / 16g+2mt+1;
+  // dense: channels 16mt+g / 16mt+g+8.  Columns 2q, 2q+1 are heads; oh holds heads 8+2q, 8+2q+1.
   float ot[8][4];
   float oh[HIROWS ? 8 : 1][4];
 #pragma unroll
@@ -200,18 +171,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     cp_async_commit();
   }
 
-  // per-lane ldmatrix row addresses (matrix = lane / 8, row = lane % 8)
+  // dense path: per-lane ldmatrix row addresses (token rows (mat>>1)*8 + r, channel half mat&1)
   const int mat = lane >> 3, r8 = lane & 7;
-  uint32_t k_off, v_off;
-  constexpr uint32_t kStepK = SPARSE ? kTStep : 32;  // bytes between 16-channel steps
-  if constexpr (SPARSE) {
-    // channel rows (mat & 1)*8 + r8 of each 16-channel step, token half mat >> 1
-    const int ch = (mat & 1) * 8 + r8;
-    k_off = v_off = ttile_off(ch, 0) + (mat >> 1) * 16;
-  } else {
-    // token rows (mat >> 1)*8 + r8, channel half (mat & 1) of each 16-channel step
-    k_off = v_off = (((mat >> 1) << 3) + r8) * kRowBytes + ((mat & 1) << 4);
-  }
+  const uint32_t t_off = (((mat >> 1) << 3) + r8) * kRowBytes + ((mat & 1) << 4);
 
 #pragma unroll 1
   for (int i = 0; i < my_n; ++i) {
@@ -226,42 +188,43 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     __syncwarp();
     const uint8_t *stage = wbase + (i % NSTAGE) * P.stage_bytes;
     const int t0 = (c_begin + warp + kDecodeWarps * i) * kChunk;
-    const uint8_t *ktile;
-    const uint8_t *vtile;
-    if constexpr (SPARSE) {
-      expand_chunk(P, stage, dense, lane, t0, L);
-      __syncwarp();
-      ktile = dense;
-      vtile = dense + kTTileBytes;
-    } else {
-      ktile = stage;
-      vtile = stage + kTileBytes;
-    }
 
-    // S = Q K~^T for the chunk's 16 tokens (two n-tiles of 8)
+    // ---- S = Q K~^T for the chunk's 16 tokens (two n-tiles of 8)
     float s[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-    const uint32_t kaddr = smem_addr(ktile) + k_off;
+    if constexpr (SPARSE) {
+      const uint32_t kvals = smem_addr(stage + 512);
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t b0, b1, b2, b3;
-      if constexpr (SPARSE)
-        ldmatrix_x4_trans(b0, b1, b2, b3, kaddr + ks * kStepK);
-      else
-        ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * kStepK);
-      mma_f16_16816(s[0], qa[ks], b0, b1);
-      mma_f16_16816(s[1], qa[ks], b2, b3);
+      for (int nt = 0; nt < 2; ++nt) {
+        const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (t0 + T < L) w = *reinterpret_cast<const uint4 *>(stage + T * 16);
+        uint32_t kb[16];
+        expand_word(pick(w, qq), kvals + 2 * (T * P.keep_k + prefix_words(w, qq)), kb);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
+      }
+    } else {
+      const uint32_t kaddr = smem_addr(stage) + t_off;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * 32);
+        mma_f16_16816(s[0], qa[ks], b0, b1);
+        mma_f16_16816(s[1], qa[ks], b2, b3);
+      }
     }
 
-    // scale into the log2 domain, mask tokens >= L, online softmax per row (= q head)
+    // ---- scale into the log2 domain, mask tokens >= L, online softmax per row (= q head)
     float mx[2] = {kNegInf, kNegInf};
+    const bool full = t0 + kChunk <= L;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = t0 + nt * 8 + 2 * qq + (e & 1);
-        const float x = tok < L ? s[nt][e] * P.scale_log2 : kNegInf;
+        const float x = (full || tok < L) ? s[nt][e] * P.scale_log2 : kNegInf;
         s[nt][e] = x;
         mx[e >> 1] = fmaxf(mx[e >> 1], x);
       }
@@ -319,17 +282,47 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     const uint32_t pc0 = HIROWS ? pack_half2(s[0][2], s[0][3]) : 0u;
     const uint32_t pc1 = HIROWS ? pack_half2(s[1][2], s[1][3]) : 0u;
 
-    // O^T += V~^T P^T : 8 m-tiles of 16 channels
-    const uint32_t vaddr = smem_addr(vtile) + v_off;
+    // ---- O^T += V~^T P^T : 8 m-tiles of 16 channels
+    if constexpr (SPARSE) {
+      // this lane's A fragments cover channels 16g..16g+15 (half hv of bitmap word wv) of
+      // tokens 2q, 2q+1 (k = 2q, 2q+1) and 2q+8, 2q+9 (k = 2q+8, 2q+9)
+      const int wv = gq >> 1, hv = gq & 1;
+      const uint32_t vvals = smem_addr(stage + 512 + 32 * P.keep_k);
+      uint32_t va[8][4];
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      uint32_t a[4];
-      if constexpr (SPARSE)
-        ldmatrix_x4(a[0], a[1], a[2], a[3], vaddr + mt * kStepK);
-      else
-        ldmatrix_x4_trans(a[0], a[1], a[2], a[3], vaddr + mt * kStepK);
-      mma_f16_16816(ot[mt], a, pb0, pb1);
-      if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
+      for (int pair = 0; pair < 2; ++pair) {
+        uint32_t x0[16], x1[16];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int T = 2 * qq + 8 * pair + e;
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (t0 + T < L) w = *reinterpret_cast<const uint4 *>(stage + 256 + T * 16);
+          const uint32_t word = pick(w, wv);
+          const uint32_t bits = hv ? (word >> 16) : (word & 0xFFFFu);
+          const uint32_t pre = prefix_words(w, wv) + (hv ? __popc(word & 0xFFFFu) : 0u);
+          expand_half(bits, vvals + 2 * (T * P.keep_v + pre), e ? x1 : x0);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          va[mt][2 * pair] = __byte_perm(x0[2 * mt], x1[2 * mt], 0x5410);
+          va[mt][2 * pair + 1] = __byte_perm(x0[2 * mt + 1], x1[2 * mt + 1], 0x5410);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        const uint32_t a[4] = {va[mt][0], va[mt][1], va[mt][2], va[mt][3]};
+        mma_f16_16816(ot[mt], a, pb0, pb1);
+        if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
+      }
+    } else {
+      const uint32_t vaddr = smem_addr(stage + kTileBytes) + t_off;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(a[0], a[1], a[2], a[3], vaddr + mt * 32);
+        mma_f16_16816(ot[mt], a, pb0, pb1);
+        if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
+      }
     }
     __syncwarp();
   }
@@ -360,23 +353,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
     const int h0 = 2 * qq, h1 = 2 * qq + 1;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      const int ch = mt * 16 + gq;
+      const int ch0 = SPARSE ? 16 * gq + 2 * mt : 16 * mt + gq;  // channel of accumulator rows g
+      const int ch1 = SPARSE ? ch0 + 1 : ch0 + 8;                // and g+8
       if (h0 < G) {
-        sm_o[(warp * G + h0) * kHeadDim + ch] = ot[mt][0];
-        sm_o[(warp * G + h0) * kHeadDim + ch + 8] = ot[mt][2];
+        sm_o[(warp * G + h0) * kHeadDim + ch0] = ot[mt][0];
+        sm_o[(warp * G + h0) * kHeadDim + ch1] = ot[mt][2];
       }
       if (h1 < G) {
-        sm_o[(warp * G + h1) * kHeadDim + ch] = ot[mt][1];
-        sm_o[(warp * G + h1) * kHeadDim + ch + 8] = ot[mt][3];
+        sm_o[(warp * G + h1) * kHeadDim + ch0] = ot[mt][1];
+        sm_o[(warp * G + h1) * kHeadDim + ch1] = ot[mt][3];
       }
       if constexpr (HIROWS) {
         if (h0 + 8 < G) {
-          sm_o[(warp * G + h0 + 8) * kHeadDim + ch] = oh[mt][0];
-          sm_o[(warp * G + h0 + 8) * kHeadDim + ch + 8] = oh[mt][2];
+          sm_o[(warp * G + h0 + 8) * kHeadDim + ch0] = oh[mt][0];
+          sm_o[(warp * G + h0 + 8) * kHeadDim + ch1] = oh[mt][2];
         }
         if (h1 + 8 < G) {
-          sm_o[(warp * G + h1 + 8) * kHeadDim + ch] = oh[mt][1];
-          sm_o[(warp * G + h1 + 8) * kHeadDim + ch + 8] = oh[mt][3];
+          sm_o[(warp * G + h1 + 8) * kHeadDim + ch0] = oh[mt][1];
+          sm_o[(warp * G + h1 + 8) * kHeadDim + ch1] = oh[mt][3];
         }
       }
     }
@@ -543,9 +537,9 @@ cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int kee
   int nstage, stage_bytes, warp_bytes;
   if (sparse) {
     stage_bytes = 512 + 32 * (keep_k + keep_v);
-    nstage = (kWarpSmemTarget - 2 * kTTileBytes) / stage_bytes;
+    nstage = kWarpSmemTarget / stage_bytes;
     nstage = nstage < 2 ? 2 : (nstage > 4 ? 4 : nstage);
-    warp_bytes = nstage * stage_bytes + 2 * kTTileBytes;
+    warp_bytes = nstage * stage_bytes;
   } else {
     stage_bytes = 2 * kTileBytes;
     nstage = 3;

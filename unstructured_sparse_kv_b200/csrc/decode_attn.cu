@@ -73,36 +73,38 @@ __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t strea
   }
 }
 
-// x = (bits & MASK) ? the fp16 at shared address ra : 0; ra advances past a loaded value.
+// x = (bits & MASK) ? the fp16 at shared address ra : 0 (read from the CTA's zero slot `za`);
+// ra advances past a taken value.  No branch and no register zeroing: pruned channels load the
+// zero slot, which every pruned lane of a warp reads at the same address (a broadcast).
 template <uint32_t MASK>
-__device__ __forceinline__ uint32_t take(uint32_t bits, uint32_t &ra) {
-  uint32_t x = 0;
+__device__ __forceinline__ uint32_t take(uint32_t bits, uint32_t &ra, uint32_t za) {
+  uint32_t x;
   asm volatile(
-      "{\n .reg .pred p;\n .reg .b32 t;\n and.b32 t, %2, %3;\n setp.ne.u32 p, t, 0;\n"
-      " @p ld.shared.u16 %0, [%1];\n @p add.u32 %1, %1, 2;\n}\n"
-      : "+r"(x), "+r"(ra)
-      : "r"(bits), "n"(MASK)
+      "{\n .reg .pred p;\n .reg .b32 t, a;\n and.b32 t, %2, %3;\n setp.ne.u32 p, t, 0;\n"
+      " selp.u32 a, %1, %4, p;\n ld.shared.u16 %0, [a];\n @p add.u32 %1, %1, 2;\n}\n"
+      : "=r"(x), "+r"(ra)
+      : "r"(bits), "n"(MASK), "r"(za)
       : "memory");
   return x;
 }
 
 // Expand the 32 channels of one bitmap word into 16 packed fp16 pairs (channels 2i, 2i+1).
 template <int I = 0>
-__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t (&out)[16]) {
+__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t za, uint32_t (&out)[16]) {
   if constexpr (I < 16) {
-    const uint32_t lo = take<(1u << (2 * I))>(bits, ra);
-    const uint32_t hi = take<(1u << (2 * I + 1))>(bits, ra);
+    const uint32_t lo = take<(1u << (2 * I))>(bits, ra, za);
+    const uint32_t hi = take<(1u << (2 * I + 1))>(bits, ra, za);
     out[I] = __byte_perm(lo, hi, 0x5410);
-    expand_word<I + 1>(bits, ra, out);
+    expand_word<I + 1>(bits, ra, za, out);
   }
 }
 
 // Expand the 16 channels of a half word (bits 0..15 of `bits`) into 16 separate fp16 values.
 template <int I = 0>
-__device__ __forceinline__ void expand_half(uint32_t bits, uint32_t ra, uint32_t (&out)[16]) {
+__device__ __forceinline__ void expand_half(uint32_t bits, uint32_t ra, uint32_t za, uint32_t (&out)[16]) {
   if constexpr (I < 16) {
-    out[I] = take<(1u << I)>(bits, ra);
-    expand_half<I + 1>(bits, ra, out);
+    out[I] = take<(1u << I)>(bits, ra, za);
+    expand_half<I + 1>(bits, ra, za, out);
   }
 }
 
@@ -116,7 +118,7 @@ __device__ __forceinline__ uint32_t prefix_words(const uint4 &w, int i) {
 }
 
 template <bool SPARSE, int NSTAGE, bool HIROWS>
-__global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeParams P) {
+__global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -134,6 +136,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
   const int64_t stream = static_cast<int64_t>(b) * P.Hkv + g;
 
   uint8_t *wbase = smem + warp * P.warp_bytes;
+  __shared__ __align__(16) uint32_t zero_slot[4];
+  if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
+  __syncthreads();
+  const uint32_t za = smem_addr(zero_slot);
 
   // Q A-fragments (rows = q heads of the group, zero beyond G), 8 k-steps.  Sparse path: k-step
   // ks, fragment column 2q+e is channel 32q+4ks+e and column 2q+8+e is 32q+4ks+2+e (the
@@ -201,7 +207,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
         uint4 w = make_uint4(0u, 0u, 0u, 0u);
         if (t0 + T < L) w = *reinterpret_cast<const uint4 *>(stage + T * 16);
         uint32_t kb[16];
-        expand_word(pick(w, qq), kvals + 2 * (T * P.keep_k + prefix_words(w, qq)), kb);
+        expand_word(pick(w, qq), kvals + 2 * (T * P.keep_k + prefix_words(w, qq)), za, kb);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
       }
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel(const DecodeP
           const uint32_t word = pick(w, wv);
           const uint32_t bits = hv ? (word >> 16) : (word & 0xFFFFu);
           const uint32_t pre = prefix_words(w, wv) + (hv ? __popc(word & 0xFFFFu) : 0u);
-          expand_half(bits, vvals + 2 * (T * P.keep_v + pre), e ? x1 : x0);
+          expand_half(bits, vvals + 2 * (T * P.keep_v + pre), za, e ? x1 : x0);
         }
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
@@ -503,7 +509,7 @@ cudaError_t occupancy(KernelFn fn, int slot, int smem, int *per_sm) {
 
 constexpr int kMaxSplits = 128;
 constexpr int kMinChunksPerCta = 2 * kDecodeWarps;
-constexpr int kMaxCtasPerSm = 4;
+constexpr int kMaxCtasPerSm = 4;  // the split bound assumes at most this many resident CTAs
 constexpr int kWarpSmemTarget = 18 * 1024;  // ~3 CTAs of 4 warps per SM
 
 }  // namespace

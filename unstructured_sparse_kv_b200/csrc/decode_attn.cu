@@ -108,15 +108,6 @@ __device__ __forceinline__ void expand_half(uint32_t bits, uint32_t ra, uint32_t
   }
 }
 
-__device__ __forceinline__ uint32_t pick(const uint4 &w, int i) {
-  return i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
-}
-
-// popcount of the bitmap words below word i
-__device__ __forceinline__ uint32_t prefix_words(const uint4 &w, int i) {
-  return (i > 0 ? __popc(w.x) : 0) + (i > 1 ? __popc(w.y) : 0) + (i > 2 ? __popc(w.z) : 0);
-}
-
 template <bool SPARSE, int NSTAGE, bool HIROWS>
 __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -136,6 +127,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
   const int64_t stream = static_cast<int64_t>(b) * P.Hkv + g;
 
   uint8_t *wbase = smem + warp * P.warp_bytes;
+  uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // sparse: [32 rows][8 half words] u16 prefixes
   __shared__ __align__(16) uint32_t zero_slot[4];
   if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
   __syncthreads();
@@ -192,22 +184,41 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     }
     cp_async_wait<NSTAGE - 1>();
     __syncwarp();
-    const uint8_t *stage = wbase + (i % NSTAGE) * P.stage_bytes;
+    uint8_t *stage = wbase + (i % NSTAGE) * P.stage_bytes;
     const int t0 = (c_begin + warp + kDecodeWarps * i) * kChunk;
+    const bool full = t0 + kChunk <= L;
 
     // ---- S = Q K~^T for the chunk's 16 tokens (two n-tiles of 8)
     float s[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
     if constexpr (SPARSE) {
+      // per-row table: lane r (K rows 0-15, V rows 16-31) zeroes the bitmap of a token >= L in
+      // place and stores the popcount prefix of each of its row's 8 half words (u16 each)
+      {
+        uint4 *row = reinterpret_cast<uint4 *>(stage + lane * 16);
+        uint4 w = *row;
+        if (!full && t0 + (lane & 15) >= L) {
+          w = make_uint4(0u, 0u, 0u, 0u);
+          *row = w;
+        }
+        const uint32_t h0 = __popc(w.x & 0xFFFFu), c0 = __popc(w.x);
+        const uint32_t h1 = c0 + __popc(w.y & 0xFFFFu), c1 = c0 + __popc(w.y);
+        const uint32_t h2 = c1 + __popc(w.z & 0xFFFFu), c2 = c1 + __popc(w.z);
+        const uint32_t h3 = c2 + __popc(w.w & 0xFFFFu);
+        // half words 0..7 start at 0, h0, c0, h1, c1, h2, c2, h3 kept values
+        *reinterpret_cast<uint4 *>(htab + lane * 16) =
+            make_uint4(h0 << 16, c0 | (h1 << 16), c1 | (h2 << 16), c2 | (h3 << 16));
+      }
+      __syncwarp();
       const uint32_t kvals = smem_addr(stage + 512);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (t0 + T < L) w = *reinterpret_cast<const uint4 *>(stage + T * 16);
+        const uint32_t word = *reinterpret_cast<const uint32_t *>(stage + T * 16 + qq * 4);
+        const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + T * 16 + qq * 4);
         uint32_t kb[16];
-        expand_word(pick(w, qq), kvals + 2 * (T * P.keep_k + prefix_words(w, qq)), za, kb);
+        expand_word(word, kvals + 2 * (T * P.keep_k + pre), za, kb);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
       }
@@ -224,20 +235,19 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
 
     // ---- scale into the log2 domain, mask tokens >= L, online softmax per row (= q head)
     float mx[2] = {kNegInf, kNegInf};
-    const bool full = t0 + kChunk <= L;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
+      for (int e = 0; e < (HIROWS ? 4 : 2); ++e) {
         const int tok = t0 + nt * 8 + 2 * qq + (e & 1);
         const float x = (full || tok < L) ? s[nt][e] * P.scale_log2 : kNegInf;
         s[nt][e] = x;
         mx[e >> 1] = fmaxf(mx[e >> 1], x);
       }
     }
-    float alpha[2];
+    float alpha[2] = {1.f, 1.f};
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < (HIROWS ? 2 : 1); ++h) {
       mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
       mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
       const float m_new = fmaxf(m_run[h], mx[h]);
@@ -250,14 +260,14 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
+      for (int e = 0; e < (HIROWS ? 4 : 2); ++e) {
         const float p = fast_exp2(s[nt][e] - mx[e >> 1]);
         s[nt][e] = p;
         psum[e >> 1] += p;
       }
     }
     l_run[0] = l_run[0] * alpha[0] + psum[0];
-    l_run[1] = l_run[1] * alpha[1] + psum[1];
+    if constexpr (HIROWS) l_run[1] = l_run[1] * alpha[1] + psum[1];
     if (__any_sync(0xffffffffu, alpha[0] != 1.f || (HIROWS && alpha[1] != 1.f))) {
       // the O^T columns this lane holds are heads 2q and 2q+1, whose factors live in lanes 8q and 8q+4
       const float a_lo = __shfl_sync(0xffffffffu, alpha[0], 8 * qq);
@@ -290,9 +300,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
 
     // ---- O^T += V~^T P^T : 8 m-tiles of 16 channels
     if constexpr (SPARSE) {
-      // this lane's A fragments cover channels 16g..16g+15 (half hv of bitmap word wv) of
+      // this lane's A fragments cover channels 16g..16g+15 (half word g of the bitmap) of
       // tokens 2q, 2q+1 (k = 2q, 2q+1) and 2q+8, 2q+9 (k = 2q+8, 2q+9)
-      const int wv = gq >> 1, hv = gq & 1;
       const uint32_t vvals = smem_addr(stage + 512 + 32 * P.keep_k);
       uint32_t va[8][4];
 #pragma unroll
@@ -301,11 +310,9 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int T = 2 * qq + 8 * pair + e;
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (t0 + T < L) w = *reinterpret_cast<const uint4 *>(stage + 256 + T * 16);
-          const uint32_t word = pick(w, wv);
-          const uint32_t bits = hv ? (word >> 16) : (word & 0xFFFFu);
-          const uint32_t pre = prefix_words(w, wv) + (hv ? __popc(word & 0xFFFFu) : 0u);
+          // half word gq of V row T: its 16 bits and the number of kept values before it
+          const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
+          const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
           expand_half(bits, vvals + 2 * (T * P.keep_v + pre), za, e ? x1 : x0);
         }
 #pragma unroll
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
   cp_async_wait<0>();
 
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < (HIROWS ? 2 : 1); ++h) {
     l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
     l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
   }
@@ -543,9 +550,9 @@ cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int kee
   int nstage, stage_bytes, warp_bytes;
   if (sparse) {
     stage_bytes = 512 + 32 * (keep_k + keep_v);
-    nstage = kWarpSmemTarget / stage_bytes;
+    nstage = (kWarpSmemTarget - 512) / stage_bytes;
     nstage = nstage < 2 ? 2 : (nstage > 4 ? 4 : nstage);
-    warp_bytes = nstage * stage_bytes;
+    warp_bytes = nstage * stage_bytes + 512;  // + the per-row half-word prefix table
   } else {
     stage_bytes = 2 * kTileBytes;
     nstage = 3;

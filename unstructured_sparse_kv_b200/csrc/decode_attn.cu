@@ -89,13 +89,18 @@ __device__ __forceinline__ uint32_t take(uint32_t bits, uint32_t &ra, uint32_t z
 }
 
 // Expand the 32 channels of one bitmap word into 16 packed fp16 pairs (channels 2i, 2i+1).
+// The low and high half words advance two independent value pointers (ra, rb), interleaved.
 template <int I = 0>
-__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t za, uint32_t (&out)[16]) {
-  if constexpr (I < 16) {
-    const uint32_t lo = take<(1u << (2 * I))>(bits, ra, za);
-    const uint32_t hi = take<(1u << (2 * I + 1))>(bits, ra, za);
-    out[I] = __byte_perm(lo, hi, 0x5410);
-    expand_word<I + 1>(bits, ra, za, out);
+__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t rb, uint32_t za,
+                                            uint32_t (&out)[16]) {
+  if constexpr (I < 8) {
+    const uint32_t a0 = take<(1u << (2 * I))>(bits, ra, za);
+    const uint32_t b0 = take<(1u << (2 * I + 16))>(bits, rb, za);
+    const uint32_t a1 = take<(1u << (2 * I + 1))>(bits, ra, za);
+    const uint32_t b1 = take<(1u << (2 * I + 17))>(bits, rb, za);
+    out[I] = __byte_perm(a0, a1, 0x5410);
+    out[I + 8] = __byte_perm(b0, b1, 0x5410);
+    expand_word<I + 1>(bits, ra, rb, za, out);
   }
 }
 
@@ -216,9 +221,10 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
       for (int nt = 0; nt < 2; ++nt) {
         const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
         const uint32_t word = *reinterpret_cast<const uint32_t *>(stage + T * 16 + qq * 4);
-        const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + T * 16 + qq * 4);
+        const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
+        const uint32_t rbase = kvals + 2 * T * P.keep_k;
         uint32_t kb[16];
-        expand_word(word, kvals + 2 * (T * P.keep_k + pre), za, kb);
+        expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
       }
@@ -429,15 +435,33 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
   __threadfence();
   for (int r = 0; r < G; ++r) {
     const int64_t hq = static_cast<int64_t>(b) * P.Hq + static_cast<int64_t>(g) * G + r;
-    const float *ml = P.ws_ml + hq * S * 2;
+    const float2 *ml = reinterpret_cast<const float2 *>(P.ws_ml) + hq * S;
+    const float *po = P.ws_o + hq * S * kHeadDim + c;
     float M = kNegInf;
-    for (int sp = 0; sp < S; ++sp) M = fmaxf(M, __ldcg(ml + 2 * sp));
+    for (int s0 = 0; s0 < S; s0 += 8) {  // 8 loads in flight per step
+      float mv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mv[j] = s0 + j < S ? __ldcg(ml + s0 + j).x : kNegInf;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) M = fmaxf(M, mv[j]);
+    }
     float lsum = 0.f, acc = 0.f;
     if (M != kNegInf) {
-      for (int sp = 0; sp < S; ++sp) {
-        const float wt = fast_exp2(__ldcg(ml + 2 * sp) - M);
-        lsum += __ldcg(ml + 2 * sp + 1) * wt;
-        acc += __ldcg(P.ws_o + (hq * S + sp) * kHeadDim + c) * wt;
+      for (int s0 = 0; s0 < S; s0 += 8) {
+        float2 mlv[8];
+        float ov[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool in = s0 + j < S;
+          mlv[j] = in ? __ldcg(ml + s0 + j) : make_float2(kNegInf, 0.f);
+          ov[j] = in ? __ldcg(po + (s0 + j) * kHeadDim) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float wt = fast_exp2(mlv[j].x - M);
+          lsum += mlv[j].y * wt;
+          acc += ov[j] * wt;
+        }
       }
     }
     P.out[hq * kHeadDim + c] = __half_as_ushort(__float2half_rn(lsum > 0.f ? acc / lsum : 0.f));
@@ -517,7 +541,7 @@ cudaError_t occupancy(KernelFn fn, int slot, int smem, int *per_sm) {
 constexpr int kMaxSplits = 128;
 constexpr int kMinChunksPerCta = 2 * kDecodeWarps;
 constexpr int kMaxCtasPerSm = 4;  // the split bound assumes at most this many resident CTAs
-constexpr int kWarpSmemTarget = 18 * 1024;  // ~3 CTAs of 4 warps per SM
+constexpr int kWarpSmemTarget = 12 * 1024;  // lets 4 CTAs of 4 warps share an SM at the common keep counts
 
 }  // namespace
 

@@ -1,8 +1,10 @@
 """Benchmark of the Mustafar hot path on B200.
 
 A step is one decode step of the Llama-3-8B-like GQA workload at batch 8: prune +
-compress the new token's K and V into the compressed caches (two append launches),
-then sparse decode attention over the 4097..4160-token compressed context (one launch).
+compress the new token's K and V into the compressed caches, then sparse decode
+attention over the 4097..4160-token compressed context, all in one launch of the
+fused decode step (``mustafar_decode_step``).  The same step as three launches (append
+K, append V, attend) is timed beside it.
 The workload is 4096 prefill tokens plus 64 decode steps at K and V sparsity 0.7; timed
 steps cycle through the 64 decode positions.  Inputs are synthetic (seeded; see
 ``unstructured_sparse_kv_b200/synth.py``).
@@ -88,7 +90,7 @@ def decode_algorithmic_bytes(B, Hq, Hkv, d, lens, kK, kV):
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("common.cuh", "decode_attn.cu"):
+    for f in ("common.cuh", "select.cuh", "decode_attn.cu"):
         with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -194,23 +196,29 @@ class Workload:
         self.splits = M.mustafar_decode_plan_splits(B, Hkv, cap, self.kc[0].keep, self.vc[0].keep)
         self.compressed_bytes = self.kc[0].nbytes() + self.vc[0].nbytes()
 
-    def step(self, i: int, attend_only: bool = False):
+    def step(self, i: int, mode: str = "fused"):
+        """One decode step: "fused" (one launch), "separate" (append K, append V, attend) or
+        "attend" (the attention launch alone)."""
         M, r, j = self.M, i % ROTATE, i % self.steps
-        if not attend_only:
+        if mode == "fused":
+            M.mustafar_decode_step(self.q[j], self.kn[j], self.vn[j], self.pos[j], self.kc[r], self.vc[r], self.cap,
+                                   1.0, out=self.out, lse=self.lse, workspace=self.ws)
+            return
+        if mode == "separate":
             M.mustafar_append(self.kn[j], self.pos[j], self.kc[r])
             M.mustafar_append(self.vn[j], self.pos[j], self.vc[r])
         M.mustafar_decode_attn(self.q[j], self.kc[r], self.vc[r], self.seq[j], self.cap, 1.0, out=self.out,
                                lse=self.lse, workspace=self.ws)
 
-    def graph(self, attend_only=False, dense=None):
+    def graph(self, mode="fused", dense=None):
         torch = self.torch
         g = torch.cuda.CUDAGraph()
         for i in range(GRAPH_STEPS):  # warm once eagerly (plans, attributes) before capture
-            (dense.step(i) if dense else self.step(i, attend_only))
+            (dense.step(i) if dense else self.step(i, mode))
         torch.cuda.synchronize()
         with torch.cuda.graph(g):
             for i in range(GRAPH_STEPS):
-                (dense.step(i) if dense else self.step(i, attend_only))
+                (dense.step(i) if dense else self.step(i, mode))
         return g
 
 
@@ -297,7 +305,8 @@ def run_reference(args):
 def config_dict():
     w = WORKLOAD
     return {"workload": "Llama-3-8B-like GQA decode (q32/kv8/d128), batch 8, context 4096 + 64 decode steps, "
-                        "K/V sparsity 0.7; step = append K + append V + sparse decode attention",
+                        "K/V sparsity 0.7; step = one fused launch: compress the new K and V token + sparse decode "
+                        "attention",
             "batch": w["batch"], "context": w["context"], "decode_steps": w["decode_steps"],
             "sparsity_k": w["sparsity_k"], "sparsity_v": w["sparsity_v"],
             "l2": f"{ROTATE} rotating compressed-cache copies (> 2x the 126 MB L2)", "timing": "CUDA graphs of 64 steps"}
@@ -314,8 +323,8 @@ def main(argv=None):
     ap.add_argument("--suite", default=None, help="write the workload-shape suite (JSONL) to this path and exit")
     ap.add_argument("--suite-parts", default="c1,c3,c4,sweep")
     ap.add_argument("--profile-launches", type=int, default=0,
-                    help="ncu case: build the workload, run this many eager steps (append K, append V, "
-                         "attend) over the rotated caches, and exit without timing")
+                    help="ncu case: build the workload, run this many eager fused steps over the rotated "
+                         "caches, and exit without timing")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
@@ -374,19 +383,25 @@ def main(argv=None):
     us_per_step = aggregate_us_per_step(elapsed_ms, args.steps, world)
     clk = clocks.summary()
 
-    # ---- dominant kernel alone (decode attention), same inputs and rotation
-    g_att = wl.graph(attend_only=True)
-    for _ in range(3):
-        g_att.replay()
-    torch.cuda.synchronize()
-    att_reps = max(20, min(400, reps))
-    att_ms = time_graph(g_att, att_reps, stream)
-    att_us = att_ms * 1000.0 / (att_reps * GRAPH_STEPS)
+    # ---- the dominant (and only) kernel of the step is the fused decode kernel: one launch per
+    # step, so its average launch duration is the timed region's time per step
     lens = [wl.L0 + 1 + i for i in range(wl.steps)]
     avg_bytes = sum(decode_algorithmic_bytes(wl.B, wl.Hq, wl.Hkv, wl.d, [L] * wl.B, wl.kc[0].keep, wl.vc[0].keep)
                     for L in lens) / len(lens)
     peak, peak_kind = measured_peak()
-    achieved = avg_bytes / (att_us * 1e-6) / 1e9
+    achieved = avg_bytes / (us_per_step * world * 1e-6) / 1e9  # per launch on one GPU
+
+    # ---- the same step as three launches, and the attention launch alone (same inputs and rotation)
+    extra_us = {}
+    for mode in ("separate", "attend"):
+        g = wl.graph(mode)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        n = max(20, min(400, reps))
+        extra_us[mode] = time_graph(g, n, stream) * 1000.0 / (n * GRAPH_STEPS)
+        del g
+    att_us = extra_us["attend"]
 
     # ---- dense fp16 baseline on the same context
     dense = DenseBaseline(wl)
@@ -406,7 +421,6 @@ def main(argv=None):
         outh = torch.empty((wl.steps,) + tuple(wl.out.shape), dtype=torch.float16).pin_memory()
         qd, knd, vnd = torch.empty_like(wl.q[0]), torch.empty_like(wl.kn[0]), torch.empty_like(wl.vn[0])
         posd = torch.empty_like(wl.pos[0])
-        seqd = torch.empty_like(wl.pos[0])
         n_e2e = 64 * 10
 
         def e2e_step(i):
@@ -415,10 +429,7 @@ def main(argv=None):
             knd.copy_(knh[j], non_blocking=True)
             vnd.copy_(vnh[j], non_blocking=True)
             posd.copy_(posh[j], non_blocking=True)
-            M.mustafar_append(knd, posd, wl.kc[r])
-            M.mustafar_append(vnd, posd, wl.vc[r])
-            torch.add(posd, 1, out=seqd)
-            M.mustafar_decode_attn(qd, wl.kc[r], wl.vc[r], seqd, wl.cap, 1.0, out=wl.out, lse=wl.lse,
+            M.mustafar_decode_step(qd, knd, vnd, posd, wl.kc[r], wl.vc[r], wl.cap, 1.0, out=wl.out, lse=wl.lse,
                                    workspace=wl.ws)
             outh[j].copy_(wl.out, non_blocking=True)
 
@@ -437,18 +448,22 @@ def main(argv=None):
         bi = (wl.q[0].numel() + wl.kn[0].numel() + wl.vn[0].numel()) * 2 + wl.pos[0].numel() * 4
         e2e = {"value": aggregate_us_per_step(e2e_ms, n_e2e, world), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": wl.out.numel() * 2, "steps": n_e2e,
-               "how": "eager public-API calls per step: pinned H2D of q/k_new/v_new/pos, 3 library launches "
-                      "(+1 torch add for seq_len), D2H of out"}
+               "how": "eager public-API calls per step: pinned H2D of q/k_new/v_new/pos, one fused "
+                      "decode-step launch, D2H of out"}
 
     line = {"metric": METRIC, "value": us_per_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": reps_w * GRAPH_STEPS, "ms_per_step": us_per_step / 1000.0, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config_dict(),
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "peak_kind": peak_kind, "traffic": recorded_traffic(), "kernel": "decode_kernel (sparse)",
-                         "algorithmic_bytes_per_launch": avg_bytes, "us_per_launch": att_us,
-                         "splits": wl.splits},
+                         "peak_kind": peak_kind, "traffic": recorded_traffic(),
+                         "kernel": "decode_kernel (sparse, fused append)", "algorithmic_bytes_per_launch": avg_bytes,
+                         "us_per_launch": us_per_step * world, "splits": wl.splits},
+            "separate_launches": {"us_per_step": extra_us["separate"], "attend_us_per_launch": att_us,
+                                  "attend_frac": avg_bytes / (att_us * 1e-6) / 1e9 / peak,
+                                  "how": "append K + append V + decode_attn, 3 launches per step"},
             "dense_baseline": {"us_per_launch": dense_us, "sparse_speedup": dense_us / att_us,
+                               "fused_step_speedup": dense_us / (us_per_step * world),
                                "bytes_per_launch": sum(4 * wl.B * wl.Hkv * L * wl.d for L in lens) / len(lens)
                                + 4 * wl.B * wl.Hq * wl.d},
             "compressed_kv_bytes": wl.compressed_bytes,
@@ -457,7 +472,7 @@ def main(argv=None):
         line["cpu_baseline"] = oracle_decode_sample()
     if rank == 0:
         print(json.dumps(line))
-    del g_step, g_att, g_dense
+    del g_step, g_dense
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -154,6 +154,27 @@ MUSTAFAR_API mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_h
                                      void *workspace, size_t workspace_bytes, int32_t num_splits,
                                      uint32_t *d_err, mustafar_stream_t stream);
 
+/* One decode step in a single launch: append + attend.  For every (b, kv head) the new
+ * token's K and V vectors are pruned and compressed into slot pos[b] of both caches (exactly
+ * what mustafar_append writes), then the attention of mustafar_decode_attn runs over the
+ * pos[b] + 1 tokens [0, pos[b]] - the new token included (the pages prune and compress at
+ * run time: Mustafar abstract).  The CTA that will read the new token's 16-token chunk
+ * compresses it first, so no separate append launch is needed.
+ *   k_new, v_new : fp16 [batch][num_kv_heads][head_dim], element (b, h, c) at
+ *                  k_new[b*k_stride_b + h*k_stride_h + c]; 16-byte aligned, strides multiples of 8.
+ *   d_pos        : int32 [batch]; a slot outside [0, capacity) skips the append, sets
+ *                  MUSTAFAR_DEVERR_POS_RANGE and clamps the row.
+ *   max_len      : host upper bound on pos[b] + 1 (sizes the split plan and the workspace).
+ * Other arguments as in mustafar_decode_attn (same workspace query).
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
+MUSTAFAR_API mustafar_status mustafar_decode_step(const void *q, int32_t num_q_heads, const void *k_new,
+                                                  int64_t k_stride_b, int64_t k_stride_h, const void *v_new,
+                                                  int64_t v_stride_b, int64_t v_stride_h, const int32_t *d_pos,
+                                                  const mustafar_cache_t *k, const mustafar_cache_t *v,
+                                                  int32_t max_len, float scale, void *out, float *lse,
+                                                  void *workspace, size_t workspace_bytes, int32_t num_splits,
+                                                  uint32_t *d_err, mustafar_stream_t stream);
+
 /* Dense fp16 decode attention over uncompressed caches, the baseline the pages
  * compare against ("FlashAttention", "cuBLAS dense": MUSTAFAR summary,
  * "Experimental setup").  Same math and kernel skeleton as mustafar_decode_attn.

@@ -115,6 +115,22 @@ def test_append_and_decode_argument_checks(lib):
     assert st == 1 and "16" in err
 
 
+def test_decode_step_argument_checks(lib):
+    kc, vc = _cache(), _cache()
+    base = dict(q=0x7000, hq=8, kn=0x5000, ksb=256, ksh=128, vn=0x5800, vsb=256, vsh=128, pos=0x6000, L=64)
+
+    def call(**over):
+        a = dict(base, **over)
+        return _status(lib, "mustafar_decode_step", a["q"], a["hq"], a["kn"], a["ksb"], a["ksh"], a["vn"], a["vsb"],
+                       a["vsh"], a["pos"], C.byref(kc), C.byref(vc), a["L"], 1.0, 0x8000, None, None, 0, 0, None,
+                       None)
+    for over, want, msg in [(dict(kn=None), 1, "k_new"), (dict(pos=None), 1, "pos must be non-NULL"), (dict(pos=0x6002), 3, "pos needs"),
+                            (dict(vn=0x5808), 3, "multiples of 8"), (dict(ksh=100), 3, "multiples of 8"),
+                            (dict(vsb=-256), 1, "negative"), (dict(hq=5), 1, "multiple"), (dict(L=0), 1, "max_len")]:
+        st, err = call(**over)
+        assert st == want and msg in err, (over, st, err)
+
+
 def test_workspace_query(lib):
     n1 = M.mustafar_decode_workspace_bytes(8, 32, 8, 4160, num_splits=1)
     n4 = M.mustafar_decode_workspace_bytes(8, 32, 8, 4160, num_splits=4)

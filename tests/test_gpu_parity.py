@@ -178,6 +178,93 @@ def test_dense_baseline_matches_oracle_and_sdpa():
     assert float((sd - out[:1].float()).abs().max()) < 2e-3
 
 
+# ------------------------------------------------------------------------------------ fused decode step
+def _row_cache_matches(cache, x_bits_bhld, lens):
+    """Per-row bit-exact check: row b's first lens[b] tokens against the oracle's compression."""
+    bm, vals, _ = U.cache_np(cache)
+    k, cap = cache.keep, cache.capacity
+    for b, Lb in enumerate(lens):
+        ref = oracle.compress(x_bits_bhld[b:b + 1, :, :Lb], k, cap, Lb)
+        assert np.array_equal(bm[b, :, :Lb], ref["bitmap"][0, :, :Lb]), ("bitmap", b)
+        assert np.array_equal(vals[b, :, :Lb * k], ref["values"][0, :, :Lb * k]), ("values", b)
+
+
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_decode_step_ragged_positions_match_oracle(splits):
+    # rows at different positions; appends cross 16-token chunks, a 64-token tile and split
+    # boundaries, and overwrite slots that the prefill compression had filled with other tokens
+    B, Hq, Hkv, cap, steps = 3, 8, 2, 256, 20
+    L0 = [100, 15, 60]
+    K0 = synth.keys(B, Hkv, max(L0), D, 31, DEV, capacity=cap)
+    V0 = synth.values(B, Hkv, max(L0), D, 31, DEV, capacity=cap)
+    kc, vc = M.CompressedCache(B, Hkv, cap, 0.7), M.CompressedCache(B, Hkv, cap, 0.5)
+    M.mustafar_compress(K0, max(L0), 0.7, kc)
+    M.mustafar_compress(V0, max(L0), 0.5, vc)
+    Kt, Vt = K0.clone(), V0.clone()  # the dense truth each row's cache must hold
+    vbuf = torch.zeros(B, Hkv, 2 * D, dtype=torch.float16, device=DEV)  # strided v_new
+    rows = torch.arange(B, device=DEV)
+    for st in range(steps):
+        pos = torch.tensor([l + st for l in L0], dtype=torch.int32, device=DEV)
+        kn, vn = synth.step_tokens(B, Hkv, D, 31, st, DEV)
+        vbuf[:, :, D:] = vn
+        Kt[rows, :, pos.long()] = kn
+        Vt[rows, :, pos.long()] = vn
+        qs = synth.queries(B, Hq, D, 31, DEV, step=st)
+        out, lse = M.mustafar_decode_step(qs, kn, vbuf[:, :, D:], pos, kc, vc, max(L0) + steps, 1.0,
+                                          num_splits=splits)
+        if st in (0, 1, 4, 5, 19):
+            lens = (pos + 1).cpu().numpy()
+            o_ref, l_ref = U.oracle_attention(qs, U.bits(Kt), U.bits(Vt), kc.keep, vc.keep, lens, 1.0)
+            U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"step {st} splits {splits}")
+    final = [l + steps for l in L0]
+    _row_cache_matches(kc, U.bits(Kt), final)
+    _row_cache_matches(vc, U.bits(Vt), final)
+
+
+def test_decode_step_same_bits_as_append_then_attend():
+    B, Hq, Hkv, L0, cap = 8, 32, 8, 500, 640
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L0, cap, 0.7, 0.7, 77)
+    kc2, vc2 = M.CompressedCache(B, Hkv, cap, 0.7), M.CompressedCache(B, Hkv, cap, 0.7)
+    for a, b in ((kc, kc2), (vc, vc2)):
+        b.bitmap.copy_(a.bitmap)
+        b.values.copy_(a.values)
+        b.tile_offset.copy_(a.tile_offset)
+    for st in range(3):
+        kn, vn = synth.step_tokens(B, Hkv, D, 77, st, DEV)
+        pos = torch.full((B,), L0 + st, dtype=torch.int32, device=DEV)
+        qs = synth.queries(B, Hq, D, 77, DEV, step=st)
+        o1, l1 = M.mustafar_decode_step(qs, kn, vn, pos, kc, vc, cap, 1.0)
+        M.mustafar_append(kn, pos, kc2)
+        M.mustafar_append(vn, pos, vc2)
+        o2, l2 = M.mustafar_decode_attn(qs, kc2, vc2, pos + 1, cap, 1.0)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {st}"
+    for a, b in ((kc, kc2), (vc, vc2)):
+        assert torch.equal(a.bitmap, b.bitmap) and torch.equal(a.values, b.values)
+
+
+def test_decode_step_out_of_range_positions():
+    B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 23)
+    bm0, vals0 = kc.bitmap.clone(), kc.values.clone()
+    kn, vn = synth.step_tokens(B, Hkv, D, 23, 0, DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pos = torch.tensor([-1, cap, 20], dtype=torch.int32, device=DEV)
+    out, lse = M.mustafar_decode_step(q, kn, vn, pos, kc, vc, cap, 1.0, err=err)
+    assert int(err.item()) & M.DEVERR_POS_RANGE
+    assert float(out[0].abs().max()) == 0.0 and torch.isinf(lse[0]).all() and (lse[0] < 0).all()
+    assert torch.equal(kc.bitmap[:2], bm0[:2]) and torch.equal(kc.values[:2], vals0[:2])  # rows 0, 1: no append
+    Kt, Vt = K.clone(), V.clone()
+    Kt[2, :, 20] = kn[2]
+    Vt[2, :, 20] = vn[2]
+    o_ref, l_ref = U.oracle_attention(q[1:], U.bits(Kt)[1:], U.bits(Vt)[1:], kc.keep, vc.keep, [cap, 21], 1.0)
+    U.assert_attn_close(out[1:], o_ref, lse[1:], l_ref, tag="clamped step")
+    _row_cache_matches(kc, U.bits(Kt), [cap, cap, cap])
+    err.zero_()
+    pos = torch.tensor([5, 6, 60], dtype=torch.int32, device=DEV)
+    M.mustafar_decode_step(q, kn, vn, pos, kc, vc, 16, 1.0, err=err)  # max_len does not cover row 2
+    assert int(err.item()) & M.DEVERR_LEN_RANGE
+
+
 # ------------------------------------------------------------------------------------ the workload shapes
 def test_llama3_gqa_b1_ctx1024_s05():
     B, Hq, Hkv, L = 1, 32, 8, 1024
@@ -189,7 +276,8 @@ def test_llama3_gqa_b1_ctx1024_s05():
     U.assert_attn_close(out, o_ref, lse, l_ref, tag="b1 ctx1024")
 
 
-def test_llama3_gqa_b8_ctx4096_s07_64_decode_steps():
+@pytest.mark.parametrize("fused", [False, True])
+def test_llama3_gqa_b8_ctx4096_s07_64_decode_steps(fused):
     B, Hq, Hkv, L0, steps = 8, 32, 8, 4096, 64
     cap = L0 + steps
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L0, cap, 0.7, 0.7, 1002)
@@ -199,10 +287,13 @@ def test_llama3_gqa_b8_ctx4096_s07_64_decode_steps():
         K[:, :, L0 + st] = kn
         V[:, :, L0 + st] = vn
         pos = torch.full((B,), L0 + st, dtype=torch.int32, device=DEV)
-        M.mustafar_append(kn, pos, kc)
-        M.mustafar_append(vn, pos, vc)
         qs = synth.queries(B, Hq, D, 1002, DEV, step=st)
-        out, lse = M.mustafar_decode_attn(qs, kc, vc, pos + 1, cap, 1.0)
+        if fused:
+            out, lse = M.mustafar_decode_step(qs, kn, vn, pos, kc, vc, cap, 1.0)
+        else:
+            M.mustafar_append(kn, pos, kc)
+            M.mustafar_append(vn, pos, vc)
+            out, lse = M.mustafar_decode_attn(qs, kc, vc, pos + 1, cap, 1.0)
         if st in (0, 1, 31, 63):
             saved[st] = (qs.clone(), out.clone(), lse.clone())
     Kb, Vb = U.bits(K), U.bits(V)

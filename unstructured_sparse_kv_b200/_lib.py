@@ -26,7 +26,7 @@ ABI_SYMBOLS = (
     "mustafar_keep_count", "mustafar_cache_sizes", "mustafar_compress", "mustafar_append",
     "mustafar_decode_workspace_bytes", "mustafar_decode_attn", "mustafar_dense_decode_attn",
     "mustafar_decode_plan_splits", "mustafar_status_string", "mustafar_last_error", "mustafar_abi_version",
-    "mustafar_decode_attn_noalloc",
+    "mustafar_decode_attn_noalloc", "mustafar_decode_step",
 )
 
 
@@ -70,6 +70,8 @@ def load() -> C.CDLL:
         "mustafar_last_error": (C.c_char_p, []),
         "mustafar_abi_version": (i32, []),
         "mustafar_decode_attn_noalloc": (i32, [vp, i32, P(CacheT), P(CacheT), vp, i32, f32, vp, vp, i32, vp, vp]),
+        "mustafar_decode_step": (i32, [vp, i32, vp, i64, i64, vp, i64, i64, vp, P(CacheT), P(CacheT), i32, f32, vp,
+                                       vp, vp, sz, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -238,4 +240,30 @@ def mustafar_decode_attn_noalloc(q: torch.Tensor, k: CompressedCache, v: Compres
     _check(load().mustafar_decode_attn_noalloc(_ptr(q), q.shape[1], C.byref(k.struct), C.byref(v.struct),
                                                _ptr(seq_len), max_len, scale, _ptr(out), _ptr(lse), num_splits,
                                                _ptr(err), _stream(stream)))
+    return out, lse
+
+
+def mustafar_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
+                         k: CompressedCache, v: CompressedCache, max_len: int, scale: float, out=None, lse=None,
+                         workspace=None, num_splits: int = 0, err=None, stream=None, want_lse: bool = True):
+    """One decode step in one launch: compress ``k_new``/``v_new`` ([B, Hkv, d] fp16) into slot
+    ``pos[b]`` of the caches, then attend over the ``pos[b] + 1`` tokens ``[0, pos[b]]``.
+    Returns (out [B,Hq,d] fp16, lse [B,Hq] fp32); ``max_len`` bounds ``pos[b] + 1``."""
+    _cuda_f16(q, "q")
+    if not q.is_contiguous() or q.dim() != 3:
+        raise ValueError("q must be a contiguous [B, Hq, d] tensor")
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _cuda_f16(t, n)
+        if t.dim() != 3 or t.stride(2) != 1 or tuple(t.shape) != (k.batch, k.num_kv_heads, k.head_dim):
+            raise ValueError(f"{n} must be [B, Hkv, d] with contiguous channels, matching the cache")
+    if not (pos.is_cuda and pos.dtype == torch.int32 and pos.numel() == k.batch):
+        raise ValueError("pos must be a CUDA int32 tensor of length batch")
+    out, lse = _decode_outputs(q, out, lse, want_lse)
+    if workspace is None:
+        workspace = torch.zeros(mustafar_decode_workspace_bytes(q.shape[0], q.shape[1], k.num_kv_heads, max_len,
+                                                                num_splits), dtype=torch.uint8, device=q.device)
+    _check(load().mustafar_decode_step(_ptr(q), q.shape[1], _ptr(k_new), k_new.stride(0), k_new.stride(1),
+                                       _ptr(v_new), v_new.stride(0), v_new.stride(1), _ptr(pos), C.byref(k.struct),
+                                       C.byref(v.struct), max_len, scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                                       workspace.numel(), num_splits, _ptr(err), _stream(stream)))
     return out, lse

@@ -207,16 +207,16 @@ mustafar_status run_decode(bool sparse, DecodeParams &p, int max_len, int num_sp
 
 mustafar_status check_decode_common(const void *q, int32_t Hq, int32_t B, int32_t Hkv, const int32_t *d_seq_len,
                                     int32_t max_len, float scale, const void *out, const float *lse,
-                                    const char *name) {
+                                    const char *name, const char *len_name = "seq_len") {
   if (q == nullptr || out == nullptr || d_seq_len == nullptr)
-    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: q, out and seq_len must be non-NULL", name);
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: q, out and %s must be non-NULL", name, len_name);
   if (Hq <= 0 || Hq % Hkv != 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: num_q_heads must be a multiple of num_kv_heads", name);
   if (Hq / Hkv > 16) return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: at most 16 q heads per kv head", name);
   if (max_len <= 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: max_len must be positive", name);
   if (!std::isfinite(scale)) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: scale must be finite", name);
   if (!aligned(q, 16) || !aligned(out, 16)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: q and out need 16-byte alignment", name);
   if (lse != nullptr && !aligned(lse, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: lse needs 4-byte alignment", name);
-  if (!aligned(d_seq_len, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: seq_len needs 4-byte alignment", name);
+  if (!aligned(d_seq_len, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: %s needs 4-byte alignment", name, len_name);
   (void)B;
   return MUSTAFAR_OK;
 }
@@ -257,6 +257,58 @@ mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_heads, const m
   p.lse = lse;
   p.err = d_err;
   return run_decode(true, p, max_len, num_splits, workspace, workspace_bytes, "decode_attn",
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+mustafar_status mustafar_decode_step(const void *q, int32_t num_q_heads, const void *k_new, int64_t k_stride_b,
+                                     int64_t k_stride_h, const void *v_new, int64_t v_stride_b, int64_t v_stride_h,
+                                     const int32_t *d_pos, const mustafar_cache_t *k, const mustafar_cache_t *v,
+                                     int32_t max_len, float scale, void *out, float *lse, void *workspace,
+                                     size_t workspace_bytes, int32_t num_splits, uint32_t *d_err,
+                                     mustafar_stream_t stream) {
+  mustafar_status s = check_cache(k, "decode_step(k)");
+  if (s != MUSTAFAR_OK) return s;
+  s = check_cache(v, "decode_step(v)");
+  if (s != MUSTAFAR_OK) return s;
+  if (k->batch != v->batch || k->num_kv_heads != v->num_kv_heads || k->head_dim != v->head_dim)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "decode_step: K and V caches disagree on batch/heads/head_dim");
+  s = check_decode_common(q, num_q_heads, k->batch, k->num_kv_heads, d_pos, max_len, scale, out, lse,
+                          "decode_step", "pos");
+  if (s != MUSTAFAR_OK) return s;
+  if (num_splits < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "decode_step: num_splits must be >= 0");
+  if (k_new == nullptr || v_new == nullptr)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "decode_step: k_new and v_new must be non-NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || k_stride_b % 8 != 0 || k_stride_h % 8 != 0 ||
+      v_stride_b % 8 != 0 || v_stride_h % 8 != 0)
+    return fail(MUSTAFAR_ERR_MISALIGNED, "decode_step: k_new, v_new and their strides must be multiples of 8 elements");
+  if (k_stride_b < 0 || k_stride_h < 0 || v_stride_b < 0 || v_stride_h < 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "decode_step: negative strides are not supported");
+  DecodeParams p{};
+  p.q = static_cast<const uint16_t *>(q);
+  p.kbm = k->bitmap;
+  p.kval = k->values;
+  p.vbm = v->bitmap;
+  p.vval = v->values;
+  p.keep_k = k->keep;
+  p.keep_v = v->keep;
+  p.cap_k = k->capacity;
+  p.cap_v = v->capacity;
+  p.B = k->batch;
+  p.Hq = num_q_heads;
+  p.Hkv = k->num_kv_heads;
+  p.G = num_q_heads / k->num_kv_heads;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.out = static_cast<uint16_t *>(out);
+  p.lse = lse;
+  p.err = d_err;
+  p.pos = d_pos;
+  p.kn = static_cast<const uint16_t *>(k_new);
+  p.vn = static_cast<const uint16_t *>(v_new);
+  p.kn_sb = k_stride_b;
+  p.kn_sh = k_stride_h;
+  p.vn_sb = v_stride_b;
+  p.vn_sh = v_stride_h;
+  return run_decode(true, p, max_len, num_splits, workspace, workspace_bytes, "decode_step",
                     reinterpret_cast<cudaStream_t>(stream));
 }
 

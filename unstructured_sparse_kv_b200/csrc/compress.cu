@@ -108,55 +108,9 @@ append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int3
     return;
   }
   const uint16_t *src = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
-  uint32_t raw[kWords], key[kWords];
-#pragma unroll
-  for (int w = 0; w < kWords; ++w) {
-    raw[w] = src[32 * w + lane];
-    key[w] = raw[w] & 0x7FFFu;
-  }
-  auto count_ge = [&](uint32_t t) {
-    int n = 0;
-#pragma unroll
-    for (int w = 0; w < kWords; ++w) n += __popc(__ballot_sync(0xffffffffu, key[w] >= t));
-    return n;
-  };
-  uint32_t T = 0;
-#pragma unroll 1
-  for (int bit = 14; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    if (count_ge(cand) >= k) T = cand;
-  }
-  uint32_t bm[kWords];
-  int n_gt = 0;
-#pragma unroll
-  for (int w = 0; w < kWords; ++w) {
-    bm[w] = __ballot_sync(0xffffffffu, key[w] > T);
-    n_gt += __popc(bm[w]);
-  }
-  int need = k - n_gt;  // keys equal to T that survive, lowest channels first
-#pragma unroll
-  for (int w = 0; w < kWords; ++w) {
-    uint32_t e = __ballot_sync(0xffffffffu, key[w] == T);
-    while (e != 0u && need > 0) {
-      const uint32_t low = e & (0u - e);
-      bm[w] |= low;
-      e ^= low;
-      --need;
-    }
-  }
   const int64_t stream = static_cast<int64_t>(b) * H + h;
-  if (lane < kWords) {
-    const uint32_t word = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
-    bitmap[(stream * cap + p) * kWords + lane] = word;
-  }
-  uint16_t *dst = values + (stream * cap + p) * static_cast<int64_t>(k);
-  const uint32_t below = (1u << lane) - 1u;
-  int prefix = 0;
-#pragma unroll
-  for (int w = 0; w < kWords; ++w) {
-    if ((bm[w] >> lane) & 1u) dst[prefix + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[w]);
-    prefix += __popc(bm[w]);
-  }
+  warp_compress_vector(src, k, bitmap + (stream * cap + p) * kWords, values + (stream * cap + p) * static_cast<int64_t>(k),
+                       lane);
 }
 
 cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H, int k,

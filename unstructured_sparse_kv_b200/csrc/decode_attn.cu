@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace mustafar {
 
@@ -120,12 +121,27 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int G = P.G;
   const int cap = SPARSE ? min(P.cap_k, P.cap_v) : P.cap_k;
-  int L = P.seq_len[b];
-  if (L < 0 || L > cap) {
-    if (threadIdx.x == 0 && split == 0 && g == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_LEN_RANGE);
-    L = L < 0 ? 0 : cap;
+  int L;
+  int append_at = -1;  // slot this CTA compresses the new token into (fused decode step), or -1
+  if (SPARSE && P.pos != nullptr) {
+    const int p = P.pos[b];
+    if (p < 0 || p >= cap) {
+      if (threadIdx.x == 0 && split == 0 && g == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_POS_RANGE);
+      L = p < 0 ? 0 : cap;
+    } else {
+      L = p + 1;
+      if ((p / kChunk) / P.chunks_per_split == split) append_at = p;  // the CTA that will read that chunk
+    }
+  } else {
+    L = P.seq_len[b];
+    if (L < 0 || L > cap) {
+      if (threadIdx.x == 0 && split == 0 && g == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_LEN_RANGE);
+      L = L < 0 ? 0 : cap;
+    }
   }
   const int nch = (L + kChunk - 1) / kChunk;
+  if (nch > P.num_splits * P.chunks_per_split && threadIdx.x == 0 && split == 0 && P.err != nullptr)
+    atomicOr(P.err, MUSTAFAR_DEVERR_LEN_RANGE);  // the row is longer than max_len: its tail is not covered
   const int c_begin = split * P.chunks_per_split;
   const int c_end = min(nch, c_begin + P.chunks_per_split);
   const int my_n = (c_end - c_begin > warp) ? (c_end - c_begin - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
@@ -135,6 +151,18 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
   uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // sparse: [32 rows][8 half words] u16 prefixes
   __shared__ __align__(16) uint32_t zero_slot[4];
   if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
+  if (SPARSE && append_at >= 0 && warp < 2) {
+    // fused decode step: warp 0 compresses the new K token, warp 1 the new V token, into slot
+    // append_at of this stream; the fence makes them visible to the chunk loads below
+    const bool kside = warp == 0;
+    const uint16_t *src = kside ? P.kn + b * P.kn_sb + g * P.kn_sh : P.vn + b * P.vn_sb + g * P.vn_sh;
+    const int keep = kside ? P.keep_k : P.keep_v;
+    const int64_t slot = stream * (kside ? P.cap_k : P.cap_v) + append_at;
+    uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + slot * kWords;
+    uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + slot * keep;
+    warp_compress_vector(src, keep, bm, vals, lane);
+    __threadfence();
+  }
   __syncthreads();
   const uint32_t za = smem_addr(zero_slot);
 

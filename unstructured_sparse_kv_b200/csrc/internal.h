@@ -44,6 +44,12 @@ struct DecodeParams {
   float *ws_ml;       // [B*Hq][splits][2]
   uint32_t *ws_cnt;   // [B*Hkv]
   uint32_t *err;
+  // fused decode step (sparse kernel, pos != nullptr): append the new token of every (b, kv head)
+  // at slot pos[b] of both caches, then attend over pos[b] + 1 tokens
+  const int32_t *pos;
+  const uint16_t *kn;  // [B][Hkv][128] strided
+  const uint16_t *vn;
+  int64_t kn_sb, kn_sh, vn_sb, vn_sh;
 };
 
 struct DecodePlan {

@@ -87,4 +87,54 @@ __device__ __forceinline__ void topk_bitmap(const uint32_t (&raw)[64], int k, ui
   }
 }
 
+// One warp prunes and compresses one 128-channel vector (fp16 at src, device memory):
+// writes its 4 bitmap words to bm_dst and its k kept values, ascending channel, to val_dst.
+// Lane l holds channels l, l+32, l+64, l+96, so a ballot over one of its four keys is one bitmap
+// word.  Same selection as topk_bitmap: binary search for the k-th largest key T, then the keys
+// equal to T are taken lowest channel first.  All 32 lanes must call it.
+__device__ __forceinline__ void warp_compress_vector(const uint16_t *src, int k, uint32_t *bm_dst, uint16_t *val_dst,
+                                                     int lane) {
+  uint32_t raw[kWords], key[kWords];
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    raw[w] = src[32 * w + lane];
+    key[w] = raw[w] & 0x7FFFu;
+  }
+  uint32_t T = 0;
+#pragma unroll 1
+  for (int bit = 14; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int n = 0;
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) n += __popc(__ballot_sync(0xffffffffu, key[w] >= cand));
+    if (n >= k) T = cand;
+  }
+  uint32_t bm[kWords];
+  int n_gt = 0;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    bm[w] = __ballot_sync(0xffffffffu, key[w] > T);
+    n_gt += __popc(bm[w]);
+  }
+  int need = k - n_gt;  // keys equal to T that survive, lowest channels first
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    uint32_t e = __ballot_sync(0xffffffffu, key[w] == T);
+    while (e != 0u && need > 0) {
+      const uint32_t low = e & (0u - e);
+      bm[w] |= low;
+      e ^= low;
+      --need;
+    }
+  }
+  if (lane < kWords) bm_dst[lane] = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
+  const uint32_t below = (1u << lane) - 1u;
+  int prefix = 0;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    if ((bm[w] >> lane) & 1u) val_dst[prefix + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[w]);
+    prefix += __popc(bm[w]);
+  }
+}
+
 }  // namespace mustafar

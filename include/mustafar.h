@@ -6,8 +6,8 @@
  * caches is pruned by magnitude to an unstructured sparsity, compressed into a
  * bitmap-based sparse format, and decode attention is computed directly over
  * the compressed caches.  New decode tokens are pruned and compressed at run
- * time.  K and V take separate sparsities ("k_sparsity / v_sparsity",
- * Mustafar README, Part II).
+ * time.  K and V take separate sparsities (Mustafar README, Part II: one
+ * sparsity setting for the keys, another for the values).
  *
  * Conventions for every call
  * --------------------------
@@ -70,6 +70,7 @@ typedef enum {
 /* device-side error bits ORed into *d_err (never a trap) */
 #define MUSTAFAR_DEVERR_POS_RANGE 0x1u /* append: pos[b] < 0 or >= capacity; row skipped     */
 #define MUSTAFAR_DEVERR_LEN_RANGE 0x2u /* decode: seq_len[b] < 0 or > capacity; row clamped  */
+#define MUSTAFAR_DEVERR_TIMEOUT 0x4u   /* decode: a staged copy did not land in time; result invalid */
 
 /* One compressed cache (K or V).  The three arrays are caller-owned device
  * memory sized by mustafar_cache_sizes(); bitmap and values 16-byte aligned,
@@ -86,7 +87,7 @@ typedef struct {
 } mustafar_cache_t;
 
 /* Keep count for a pruning sparsity s (fraction of channels removed, README
- * Part II: "50% sparsity is 0.5").  Returns head_dim - floor(s*head_dim), or -1
+ * Part II: a setting of 0.5 prunes half of them).  Returns head_dim - floor(s*head_dim), or -1
  * when head_dim <= 0, head_dim % 32 != 0 or s is outside [0, 1). */
 MUSTAFAR_API int32_t mustafar_keep_count(int32_t head_dim, float sparsity);
 
@@ -122,19 +123,21 @@ MUSTAFAR_API mustafar_status mustafar_append(const void *x, int64_t stride_b, in
                                 const int32_t *d_pos, const mustafar_cache_t *c, uint32_t *d_err,
                                 mustafar_stream_t stream);
 
-/* Workspace bytes for mustafar_decode_attn / mustafar_dense_decode_attn with
- * these shapes.  num_splits = 0 asks for the automatic split plan; a positive
- * value forces that many context splits (clamped to the number of 16-token chunks).
- * The workspace holds per-split partial softmax states and one ticket counter per
- * (b, kv head).  It must be zero-filled once when allocated; every completed call
+/* Workspace bytes for mustafar_decode_attn / mustafar_decode_step /
+ * mustafar_dense_decode_attn with these shapes (enough for any of them).
+ * num_splits = 0 asks for the automatic plan; a positive value asks the sparse
+ * kernel for about that many CTAs per (b, kv head) stream, and the dense baseline
+ * for that many context splits (clamped to the number of 16-token chunks).
+ * The workspace holds one ticket counter per (b, kv head) and partial softmax
+ * states.  It must be zero-filled once when allocated; every completed call
  * leaves the counters at zero again.  Calls that share a workspace must not overlap. */
 MUSTAFAR_API mustafar_status mustafar_decode_workspace_bytes(int32_t batch, int32_t num_q_heads,
                                                 int32_t num_kv_heads, int32_t head_dim,
                                                 int32_t max_len, int32_t num_splits,
                                                 size_t *bytes);
 
-/* Sparse decode attention over the compressed caches (Mustafar abstract: a
- * custom attention kernel "directly computing over compressed caches").
+/* Sparse decode attention computed straight from the compressed caches (Mustafar
+ * abstract: the method's attention kernel reads the compressed caches directly).
  * For q head hq (kv head g = hq / (Hq/Hkv)) of batch row b:
  *   z_t = scale * q[b,hq] . K~[b,g,t]   for t < seq_len[b]
  *   out[b,hq] = sum_t softmax(z)_t V~[b,g,t]          (fp16, fp32 accumulation)
@@ -144,7 +147,8 @@ MUSTAFAR_API mustafar_status mustafar_decode_workspace_bytes(int32_t batch, int3
  *               keep counts (sparsities) may differ.
  *   d_seq_len : int32 [batch]; each in [1, capacity] (longer rows are clamped
  *               and flagged in d_err; 0 gives out = 0 and lse = -inf).
- *   max_len   : host upper bound on seq_len, sizes the split plan.
+ *   max_len   : the longest row the caller expects; it sizes the work split and the
+ *               workspace.  A row longer than it is still attended in full.
  *   workspace : see mustafar_decode_workspace_bytes (same max_len and num_splits).
  *   d_err     : optional device error word.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
@@ -164,7 +168,8 @@ MUSTAFAR_API mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_h
  *                  k_new[b*k_stride_b + h*k_stride_h + c]; 16-byte aligned, strides multiples of 8.
  *   d_pos        : int32 [batch]; a slot outside [0, capacity) skips the append, sets
  *                  MUSTAFAR_DEVERR_POS_RANGE and clamps the row.
- *   max_len      : host upper bound on pos[b] + 1 (sizes the split plan and the workspace).
+ *   max_len      : the longest pos[b] + 1 the caller expects (sizes the work split and the
+ *                  workspace, as in mustafar_decode_attn).
  * Other arguments as in mustafar_decode_attn (same workspace query).
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA. */
 MUSTAFAR_API mustafar_status mustafar_decode_step(const void *q, int32_t num_q_heads, const void *k_new,
@@ -176,8 +181,8 @@ MUSTAFAR_API mustafar_status mustafar_decode_step(const void *q, int32_t num_q_h
                                                   uint32_t *d_err, mustafar_stream_t stream);
 
 /* Dense fp16 decode attention over uncompressed caches, the baseline the pages
- * compare against ("FlashAttention", "cuBLAS dense": MUSTAFAR summary,
- * "Experimental setup").  Same math and kernel skeleton as mustafar_decode_attn.
+ * compare against (dense FlashAttention-style and cuBLAS attention: MUSTAFAR
+ * summary, "Experimental setup").  Same math and kernel skeleton as mustafar_decode_attn.
  *   k_dense, v_dense : fp16 [batch][num_kv_heads][capacity][head_dim], 16-byte aligned.
  * Other arguments as in mustafar_decode_attn. */
 MUSTAFAR_API mustafar_status mustafar_dense_decode_attn(const void *q, int32_t num_q_heads, const void *k_dense,

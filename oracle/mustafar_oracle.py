@@ -45,7 +45,7 @@ WORD_BITS = 32
 def keep_count(d: int, sparsity: float) -> int:
     """Number of channels a token keeps: ``d - floor(s*d)``.
 
-    Sparsity "s" is the fraction pruned (README, Part II: "50% sparsity is 0.5").
+    Sparsity s is the fraction pruned (README, Part II: a setting of 0.5 prunes half the channels).
     ``s`` arrives as a 32-bit float (as it does through the library's C call) and
     the product is formed in double, so the target sparsity is never exceeded.
     """

@@ -259,10 +259,17 @@ def test_decode_step_out_of_range_positions():
     o_ref, l_ref = U.oracle_attention(q[1:], U.bits(Kt)[1:], U.bits(Vt)[1:], kc.keep, vc.keep, [cap, 21], 1.0)
     U.assert_attn_close(out[1:], o_ref, lse[1:], l_ref, tag="clamped step")
     _row_cache_matches(kc, U.bits(Kt), [cap, cap, cap])
+    # max_len only sizes the plan: a row longer than it is still attended in full, without a flag
     err.zero_()
+    kn2, vn2 = synth.step_tokens(B, Hkv, D, 23, 1, DEV)
     pos = torch.tensor([5, 6, 60], dtype=torch.int32, device=DEV)
-    M.mustafar_decode_step(q, kn, vn, pos, kc, vc, 16, 1.0, err=err)  # max_len does not cover row 2
-    assert int(err.item()) & M.DEVERR_LEN_RANGE
+    out, lse = M.mustafar_decode_step(q, kn2, vn2, pos, kc, vc, 16, 1.0, err=err)
+    assert int(err.item()) == 0
+    for b, p in enumerate([5, 6, 60]):
+        Kt[b, :, p] = kn2[b]
+        Vt[b, :, p] = vn2[b]
+    o_ref, l_ref = U.oracle_attention(q, U.bits(Kt), U.bits(Vt), kc.keep, vc.keep, [6, 7, 61], 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag="row longer than max_len")
 
 
 # ------------------------------------------------------------------------------------ the workload shapes

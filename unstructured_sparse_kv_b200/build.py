@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmustafar.so")
-SOURCES = ["abi.cu", "compress.cu", "decode_attn.cu", "decode_noalloc.cu"]
+SOURCES = ["abi.cu", "compress.cu", "decode_attn.cu", "decode_sparse.cu", "decode_noalloc.cu"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

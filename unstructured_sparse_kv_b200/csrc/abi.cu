@@ -164,7 +164,11 @@ mustafar_status mustafar_decode_workspace_bytes(int32_t batch, int32_t num_q_hea
   if (head_dim != kHeadDim) return fail(MUSTAFAR_ERR_UNSUPPORTED, "workspace_bytes: head_dim must be 128");
   const int nch = (max_len + kChunk - 1) / kChunk;
   int splits = num_splits > 0 ? (num_splits < nch ? num_splits : nch) : decode_split_bound(batch, num_kv_heads, max_len);
-  *bytes = decode_workspace_bytes(batch, num_q_heads, num_kv_heads, splits);
+  // enough for the dense baseline's split-K and for the sparse kernel's partial slots
+  const size_t dense = decode_workspace_bytes(batch, num_q_heads, num_kv_heads, splits);
+  const size_t sparse =
+      sparse_workspace_bound(batch, num_kv_heads, num_q_heads / num_kv_heads, max_len, num_splits);
+  *bytes = dense > sparse ? dense : sparse;
   return MUSTAFAR_OK;
 }
 
@@ -173,14 +177,41 @@ int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t
   if (batch <= 0 || num_kv_heads <= 0 || head_dim != kHeadDim || max_len <= 0) return -1;
   if (!dense && (keep_k < 1 || keep_k > kHeadDim || keep_v < 1 || keep_v > kHeadDim)) return -1;
   DecodePlan plan;
-  if (plan_decode(!dense, batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, &plan) != cudaSuccess) return -1;
-  return plan.splits;
+  if (dense) {
+    if (plan_decode(false, batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, &plan) != cudaSuccess) return -1;
+    return plan.splits;
+  }
+  // the sparse kernel cuts the end-to-end chunk sequence into CTA ranges; report the CTAs per stream
+  if (plan_sparse(batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, &plan) != cudaSuccess) return -1;
+  const int streams = batch * num_kv_heads;
+  return (plan.splits + streams - 1) / streams;
 }
 
 namespace {
 
+mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *workspace, size_t workspace_bytes,
+                           const char *name, cudaStream_t stream) {
+  DecodePlan plan;
+  cudaError_t e = plan_sparse(p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, &plan);
+  if (e != cudaSuccess) return cuda_fail(e, name);
+  p.stage_bytes = plan.stage_bytes;
+  p.warp_bytes = plan.warp_bytes;
+  const size_t need = sparse_workspace_bytes(p.B, p.Hkv, p.G, plan.splits);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(MUSTAFAR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed (%d CTAs), got %zu", name, need,
+                plan.splits, workspace == nullptr ? size_t(0) : workspace_bytes);
+  if (!aligned(workspace, 256)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned", name);
+  uint8_t *w = static_cast<uint8_t *>(workspace);
+  const size_t cnt = ((static_cast<size_t>(p.B) * p.Hkv * 4 + 255) / 256) * 256;
+  p.ws_cnt = reinterpret_cast<uint32_t *>(w);
+  p.ws_part = reinterpret_cast<float *>(w + cnt);
+  e = launch_sparse(p, plan, stream);
+  return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, name);
+}
+
 mustafar_status run_decode(bool sparse, DecodeParams &p, int max_len, int num_splits, void *workspace,
                            size_t workspace_bytes, const char *name, cudaStream_t stream) {
+  if (sparse) return run_sparse(p, max_len, num_splits, workspace, workspace_bytes, name, stream);
   DecodePlan plan;
   cudaError_t e = plan_decode(sparse, p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, &plan);
   if (e != cudaSuccess) return cuda_fail(e, name);

@@ -1,0 +1,745 @@
+// decode_sparse.cu - decode attention computed directly over the bitmap-compressed caches.
+//
+// For each batch row b and q head hq (kv head g = hq / G):
+//   out = softmax(scale * q K~^T) V~  over the pruned caches K~, V~,
+// read in their compressed form (Mustafar abstract, catalyzex author page: a custom attention
+// kernel that works on the compressed caches; MUSTAFAR summary, atlas.scime.ai, "Approach": an
+// SpMV-style attention kernel over the bitmap format).  The fused decode step (pos != nullptr)
+// first prunes and compresses each stream's new token into slot pos[b] (the runtime pruning of
+// the Mustafar abstract), then attends over pos[b] + 1 tokens.
+//
+// Work decomposition (B200-first, not the pages' design):
+// * a stream is one (b, kv head); its context is cut into 16-token chunks.  The chunks of all
+//   streams are laid end to end (stream-major) and the sequence is cut into one contiguous,
+//   equal range per CTA, for one wave of CTAs.  Warp w of a CTA takes chunks w, w+4, ... of the
+//   range, so every warp of the grid gets the same number of chunks to within one, whatever the
+//   mix of row lengths.
+// * a range may cross streams.  Its pieces are taken in order; at the end of each piece the four
+//   warps merge (m, l, o) in shared memory.  A stream whose chunks all lie in one range is
+//   finished by that CTA; a stream cut by range edges leaves one partial per CTA in the
+//   workspace and the last of those CTAs to finish (atomic ticket, no waiting) merges them.
+// * each warp stages its chunks through its own ring of NSTAGE buffers.  One lane issues, per
+//   chunk, four bulk copies of contiguous bytes (K bitmap rows, V bitmap rows, K packed values,
+//   V packed values) that complete on the buffer's mbarrier; every wait is bounded in time.
+// * per chunk, S = Q K~^T and O^T += V~^T P^T run as mma.sync m16n8k16 (fp16 in, fp32
+//   accumulate) on fragments that each lane expands straight from the compressed bytes: one
+//   predicated 16-bit shared load per channel, the bitmap bit as the predicate, pruned channels
+//   reading a shared zero.  The contraction index is permuted so that a lane's channels are one
+//   bitmap word (K) or half word (V); q's fragments use the same permutation and the output
+//   channels are put back in order at the merge.  Online softmax per head in the log2 domain.
+#include <cfloat>
+
+#include "common.cuh"
+#include "internal.h"
+#include "select.cuh"
+
+namespace mustafar {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr float kNegInf = -INFINITY;
+constexpr long long kWaitCycles = 4000000000LL;   // a bulk copy not landed after ~2 s is an error
+constexpr long long kWaitCyclesAfter = 2000000LL;  // later waits of a warp that already timed out
+
+__device__ __forceinline__ int n_chunks(int L) { return (L + kChunk - 1) / kChunk; }
+
+// Tokens of batch row b that the attention covers (clamped to [0, cap]); `bits` collects the
+// device error flags of the row.
+__device__ __forceinline__ int row_len(const DecodeParams &P, int b, int cap, uint32_t &bits) {
+  if (P.pos != nullptr) {
+    const int p = P.pos[b];
+    if (p < 0 || p >= cap) {
+      bits |= MUSTAFAR_DEVERR_POS_RANGE;
+      return p < 0 ? 0 : cap;
+    }
+    return p + 1;
+  }
+  const int L = P.seq_len[b];
+  if (L < 0 || L > cap) {
+    bits |= MUSTAFAR_DEVERR_LEN_RANGE;
+    return L < 0 ? 0 : cap;
+  }
+  return L;
+}
+
+__device__ __forceinline__ int row_len(const DecodeParams &P, int b, int cap) {
+  uint32_t ignored = 0;
+  return row_len(P, b, cap, ignored);
+}
+
+// The chunk units of one stream in the end-to-end sequence: [start, start + n).
+struct Stream {
+  int b, g;   // batch row, kv head
+  int n;      // its chunks
+  int start;  // its first unit
+  __device__ __forceinline__ int end() const { return start + n; }
+};
+
+// Step to the next stream in (b, g) order; false past the last one.
+__device__ __forceinline__ bool next_stream(const DecodeParams &P, int cap, Stream &s) {
+  s.start += s.n;
+  if (++s.g == P.Hkv) {
+    s.g = 0;
+    if (++s.b >= P.B) return false;
+    s.n = n_chunks(row_len(P, s.b, cap));
+  }
+  return true;
+}
+
+// The CTA whose range holds unit u: ranges are [floor(c U / n), floor((c+1) U / n)).
+__device__ __forceinline__ int cta_of(long long u, long long U, long long n) {
+  return static_cast<int>(((u + 1) * n - 1) / U);
+}
+__device__ __forceinline__ int range_start(long long c, long long U, long long n) {
+  return static_cast<int>(c * U / n);
+}
+
+// x = (bits & MASK) ? the fp16 at shared address ra : 0 (read from the CTA's zero slot `za`);
+// ra advances past a taken value.  No branch and no register zeroing: pruned channels load the
+// zero slot, which every pruned lane of a warp reads at the same address (a broadcast).
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t take(uint32_t bits, uint32_t &ra, uint32_t za) {
+  uint32_t x;
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b32 t, a;\n and.b32 t, %2, %3;\n setp.ne.u32 p, t, 0;\n"
+      " selp.u32 a, %1, %4, p;\n ld.shared.u16 %0, [a];\n @p add.u32 %1, %1, 2;\n}\n"
+      : "=r"(x), "+r"(ra)
+      : "r"(bits), "n"(MASK), "r"(za)
+      : "memory");
+  return x;
+}
+
+// The 32 channels of one bitmap word as 16 packed fp16 pairs (channels 2i, 2i+1); the low and
+// high half words walk two independent value pointers (ra, rb), interleaved.
+template <int I = 0>
+__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t rb, uint32_t za,
+                                            uint32_t (&out)[16]) {
+  if constexpr (I < 8) {
+    const uint32_t a0 = take<(1u << (2 * I))>(bits, ra, za);
+    const uint32_t b0 = take<(1u << (2 * I + 16))>(bits, rb, za);
+    const uint32_t a1 = take<(1u << (2 * I + 1))>(bits, ra, za);
+    const uint32_t b1 = take<(1u << (2 * I + 17))>(bits, rb, za);
+    out[I] = __byte_perm(a0, a1, 0x5410);
+    out[I + 8] = __byte_perm(b0, b1, 0x5410);
+    expand_word<I + 1>(bits, ra, rb, za, out);
+  }
+}
+
+// The 16 channels of a half word (bits 0..15 of `bits`) as 16 separate fp16 values.
+template <int I = 0>
+__device__ __forceinline__ void expand_half(uint32_t bits, uint32_t ra, uint32_t za, uint32_t (&out)[16]) {
+  if constexpr (I < 16) {
+    out[I] = take<(1u << I)>(bits, ra, za);
+    expand_half<I + 1>(bits, ra, za, out);
+  }
+}
+
+// Running state of one warp over one stream piece: online softmax (m, l) per q-head row and the
+// O^T accumulators.  Sparse layout: accumulator rows g / g+8 of m-tile mt are channels
+// 16g+2mt / 16g+2mt+1; columns 2q, 2q+1 are heads (oh: heads 8+2q, 8+2q+1).
+template <bool HIROWS>
+struct Acc {
+  float ot[8][4];
+  float oh[HIROWS ? 8 : 1][4];
+  float m_run[2], l_run[2];
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ot[i][0] = ot[i][1] = ot[i][2] = ot[i][3] = 0.f;
+#pragma unroll
+    for (int i = 0; i < (HIROWS ? 8 : 1); ++i) oh[i][0] = oh[i][1] = oh[i][2] = oh[i][3] = 0.f;
+    m_run[0] = m_run[1] = kNegInf;
+    l_run[0] = l_run[1] = 0.f;
+  }
+};
+
+// q's A fragments for stream (b, g): rows = the G q heads (zero beyond G), 8 k-steps; k-step ks,
+// fragment column 2q+e is channel 32q+4ks+e and column 2q+8+e is 32q+4ks+2+e (the permutation
+// that gives lane q the 32 channels of bitmap word q).
+template <bool HIROWS>
+__device__ __forceinline__ void load_q(const DecodeParams &P, int b, int g, int lane, uint32_t (&qa)[8][4]) {
+  const int G = P.G, gq = lane >> 2, qq = lane & 3;
+  const uint16_t *qb = P.q + (static_cast<int64_t>(b) * P.Hq + static_cast<int64_t>(g) * G) * kHeadDim;
+  const bool r0 = gq < G, r1 = HIROWS && (gq + 8 < G);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int c0 = 32 * qq + 4 * ks, c1 = c0 + 2;
+    qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + c0) : 0u;
+    qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + c0) : 0u;
+    qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + c1) : 0u;
+    qa[ks][3] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + c1) : 0u;
+  }
+}
+
+// One 16-token chunk staged at `stage` ([K bitmap rows 16x16 B][V bitmap rows][K values 16*kK]
+// [V values 16*kV]); tokens t0 .. t0+15 of a row of length L.  `htab` is the warp's 512-byte
+// per-row half-word prefix table.
+template <bool HIROWS>
+__device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *stage, uint8_t *htab, uint32_t za,
+                                              int t0, int L, int lane, const uint32_t (&qa)[8][4],
+                                              Acc<HIROWS> &acc) {
+  const int gq = lane >> 2, qq = lane & 3;
+  const bool full = t0 + kChunk <= L;
+  // lane r (K rows 0-15, V rows 16-31) zeroes the bitmap of a token >= L in place and stores the
+  // kept-value count before each of its row's 8 half words (u16 each)
+  {
+    uint4 *row = reinterpret_cast<uint4 *>(stage + lane * 16);
+    uint4 w = *row;
+    if (!full && t0 + (lane & 15) >= L) {
+      w = make_uint4(0u, 0u, 0u, 0u);
+      *row = w;
+    }
+    const uint32_t h0 = __popc(w.x & 0xFFFFu), c0 = __popc(w.x);
+    const uint32_t h1 = c0 + __popc(w.y & 0xFFFFu), c1 = c0 + __popc(w.y);
+    const uint32_t h2 = c1 + __popc(w.z & 0xFFFFu), c2 = c1 + __popc(w.z);
+    const uint32_t h3 = c2 + __popc(w.w & 0xFFFFu);
+    *reinterpret_cast<uint4 *>(htab + lane * 16) =
+        make_uint4(h0 << 16, c0 | (h1 << 16), c1 | (h2 << 16), c2 | (h3 << 16));
+  }
+  __syncwarp();
+
+  // ---- S = Q K~^T for the 16 tokens (two n-tiles of 8)
+  float s[2][4];
+  const uint32_t kvals = smem_addr(stage + 512);
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
+    const uint32_t word = *reinterpret_cast<const uint32_t *>(stage + T * 16 + qq * 4);
+    const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
+    const uint32_t rbase = kvals + 2 * T * P.keep_k;
+    uint32_t kb[16];
+    expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
+  }
+
+  // ---- scale into the log2 domain, mask tokens >= L, online softmax per row (= q head)
+  float mx[2] = {kNegInf, kNegInf};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int e = 0; e < (HIROWS ? 4 : 2); ++e) {
+      const int tok = t0 + nt * 8 + 2 * qq + (e & 1);
+      const float x = (full || tok < L) ? s[nt][e] * P.scale_log2 : kNegInf;
+      s[nt][e] = x;
+      mx[e >> 1] = fmaxf(mx[e >> 1], x);
+    }
+  }
+  float alpha[2] = {1.f, 1.f};
+#pragma unroll
+  for (int h = 0; h < (HIROWS ? 2 : 1); ++h) {
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
+    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
+    const float m_new = fmaxf(acc.m_run[h], mx[h]);
+    const float base = m_new == kNegInf ? 0.f : m_new;
+    alpha[h] = fast_exp2(acc.m_run[h] - base);
+    acc.m_run[h] = m_new;
+    mx[h] = base;
+  }
+  float psum[2] = {0.f, 0.f};
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int e = 0; e < (HIROWS ? 4 : 2); ++e) {
+      const float p = fast_exp2(s[nt][e] - mx[e >> 1]);
+      s[nt][e] = p;
+      psum[e >> 1] += p;
+    }
+  }
+  acc.l_run[0] = acc.l_run[0] * alpha[0] + psum[0];
+  if constexpr (HIROWS) acc.l_run[1] = acc.l_run[1] * alpha[1] + psum[1];
+  if (__any_sync(0xffffffffu, alpha[0] != 1.f || (HIROWS && alpha[1] != 1.f))) {
+    // the O^T columns this lane holds are heads 2q and 2q+1, whose factors live in lanes 8q and 8q+4
+    const float a_lo = __shfl_sync(0xffffffffu, alpha[0], 8 * qq);
+    const float a_hi = __shfl_sync(0xffffffffu, alpha[0], 8 * qq + 4);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      acc.ot[mt][0] *= a_lo;
+      acc.ot[mt][1] *= a_hi;
+      acc.ot[mt][2] *= a_lo;
+      acc.ot[mt][3] *= a_hi;
+    }
+    if constexpr (HIROWS) {
+      const float b_lo = __shfl_sync(0xffffffffu, alpha[1], 8 * qq);
+      const float b_hi = __shfl_sync(0xffffffffu, alpha[1], 8 * qq + 4);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        acc.oh[mt][0] *= b_lo;
+        acc.oh[mt][1] *= b_hi;
+        acc.oh[mt][2] *= b_lo;
+        acc.oh[mt][3] *= b_hi;
+      }
+    }
+  }
+  // P^T as the B operand: the S accumulator layout (row = head, columns = tokens) is exactly the
+  // m16n8k16 B layout for K = tokens, N = heads
+  const uint32_t pb0 = pack_half2(s[0][0], s[0][1]);
+  const uint32_t pb1 = pack_half2(s[1][0], s[1][1]);
+  const uint32_t pc0 = HIROWS ? pack_half2(s[0][2], s[0][3]) : 0u;
+  const uint32_t pc1 = HIROWS ? pack_half2(s[1][2], s[1][3]) : 0u;
+
+  // ---- O^T += V~^T P^T : 8 m-tiles of 16 channels.  This lane's A fragments cover channels
+  // 16g..16g+15 (half word g of the bitmap) of tokens 2q, 2q+1 and 2q+8, 2q+9.
+  const uint32_t vvals = smem_addr(stage + 512 + 32 * P.keep_k);
+  uint32_t va[8][4];
+#pragma unroll
+  for (int pair = 0; pair < 2; ++pair) {
+    uint32_t x0[16], x1[16];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int T = 2 * qq + 8 * pair + e;
+      const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
+      const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
+      expand_half(bits, vvals + 2 * (T * P.keep_v + pre), za, e ? x1 : x0);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      va[mt][2 * pair] = __byte_perm(x0[2 * mt], x1[2 * mt], 0x5410);
+      va[mt][2 * pair + 1] = __byte_perm(x0[2 * mt + 1], x1[2 * mt + 1], 0x5410);
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const uint32_t a[4] = {va[mt][0], va[mt][1], va[mt][2], va[mt][3]};
+    mma_f16_16816(acc.ot[mt], a, pb0, pb1);
+    if constexpr (HIROWS) mma_f16_16816(acc.oh[mt], a, pc0, pc1);
+  }
+}
+
+// Write the merged row r (out, lse) of q head hq from its (m, l, o[c]) sums.
+__device__ __forceinline__ void write_row(const DecodeParams &P, int64_t hq, int c, float M, float lsum, float acc) {
+  P.out[hq * kHeadDim + c] = __half_as_ushort(__float2half_rn(lsum > 0.f ? acc / lsum : 0.f));
+  if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
+}
+
+// End of one piece [seg_a, seg_e) of stream st: the four warps merge their (m, l, o) in shared
+// memory (`mer`: m[4][16], l[4][16], o[4][G][128] fp32); a stream held by this CTA alone is
+// written out, otherwise the CTA's partial goes to its workspace slot and the last CTA of the
+// stream merges all partials.  Called by every thread of the CTA.
+template <bool HIROWS>
+__device__ void flush_piece(const DecodeParams &P, Acc<HIROWS> &acc, float *mer, int warp, int lane,
+                            const Stream &st, int seg_a, int u0, int U, int cta, int nctas, int *sh_flag) {
+  const int G = P.G, gq = lane >> 2, qq = lane & 3;
+  float *sm_m = mer, *sm_l = mer + kWarps * 16, *sm_o = mer + 2 * kWarps * 16;
+#pragma unroll
+  for (int h = 0; h < (HIROWS ? 2 : 1); ++h) {
+    acc.l_run[h] += __shfl_xor_sync(0xffffffffu, acc.l_run[h], 1);
+    acc.l_run[h] += __shfl_xor_sync(0xffffffffu, acc.l_run[h], 2);
+  }
+  if (qq == 0) {
+    if (gq < G) {
+      sm_m[warp * 16 + gq] = acc.m_run[0];
+      sm_l[warp * 16 + gq] = acc.l_run[0];
+    }
+    if (HIROWS && gq + 8 < G) {
+      sm_m[warp * 16 + gq + 8] = acc.m_run[1];
+      sm_l[warp * 16 + gq + 8] = acc.l_run[1];
+    }
+  }
+  {
+    const int h0 = 2 * qq, h1 = 2 * qq + 1;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int ch0 = 16 * gq + 2 * mt, ch1 = ch0 + 1;  // channels of accumulator rows g and g+8
+      if (h0 < G) {
+        sm_o[(warp * G + h0) * kHeadDim + ch0] = acc.ot[mt][0];
+        sm_o[(warp * G + h0) * kHeadDim + ch1] = acc.ot[mt][2];
+      }
+      if (h1 < G) {
+        sm_o[(warp * G + h1) * kHeadDim + ch0] = acc.ot[mt][1];
+        sm_o[(warp * G + h1) * kHeadDim + ch1] = acc.ot[mt][3];
+      }
+      if constexpr (HIROWS) {
+        if (h0 + 8 < G) {
+          sm_o[(warp * G + h0 + 8) * kHeadDim + ch0] = acc.oh[mt][0];
+          sm_o[(warp * G + h0 + 8) * kHeadDim + ch1] = acc.oh[mt][2];
+        }
+        if (h1 + 8 < G) {
+          sm_o[(warp * G + h1 + 8) * kHeadDim + ch0] = acc.oh[mt][1];
+          sm_o[(warp * G + h1 + 8) * kHeadDim + ch1] = acc.oh[mt][3];
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // the CTAs holding part of this stream: ca .. cb (an empty range that starts exactly where
+  // the stream starts belongs to no stream)
+  const int ca = cta_of(st.start, U, nctas), cb = cta_of(st.end() - 1, U, nctas);
+  const bool mine = cta >= ca && cta <= cb;
+  const int slot_floats = 32 + G * kHeadDim;
+  const int c = threadIdx.x;  // output channel
+  const int64_t hq0 = static_cast<int64_t>(st.b) * P.Hq + static_cast<int64_t>(st.g) * G;
+  if (mine) {
+    float *part = P.ws_part + static_cast<int64_t>(2 * cta + (seg_a == u0 ? 0 : 1)) * slot_floats;
+    for (int r = 0; r < G; ++r) {
+      float M = kNegInf;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
+      float lsum = 0.f, o = 0.f;
+      if (M != kNegInf) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const float wt = fast_exp2(sm_m[w * 16 + r] - M);
+          lsum += sm_l[w * 16 + r] * wt;
+          o += sm_o[(w * G + r) * kHeadDim + c] * wt;
+        }
+      }
+      if (ca == cb) {
+        write_row(P, hq0 + r, c, M, lsum, o);
+      } else {
+        part[32 + r * kHeadDim + c] = o;
+        if (c == 0) {
+          part[r] = M;
+          part[16 + r] = lsum;
+        }
+      }
+    }
+  }
+  if (mine && ca != cb) {
+    // ---- last CTA of this stream merges every partial (no waiting: an atomic ticket)
+    __threadfence();
+    __syncthreads();
+    const int sid = st.b * P.Hkv + st.g;
+    if (threadIdx.x == 0) {
+      const uint32_t ticket = atomicAdd(P.ws_cnt + sid, 1u);
+      *sh_flag = ticket == static_cast<uint32_t>(cb - ca);
+    }
+    __syncthreads();
+    if (*sh_flag) {
+      __threadfence();
+      const int n = cb - ca + 1;
+      const int first_slot = 2 * ca + (range_start(ca, U, nctas) < st.start ? 1 : 0);
+      for (int r = 0; r < G; ++r) {
+        float M = kNegInf;
+        for (int j0 = 0; j0 < n; j0 += 8) {  // 8 loads in flight per step
+          float mv[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int sl = j0 + j == 0 ? first_slot : 2 * (ca + j0 + j);
+            mv[j] = j0 + j < n ? __ldcg(P.ws_part + static_cast<int64_t>(sl) * slot_floats + r) : kNegInf;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) M = fmaxf(M, mv[j]);
+        }
+        float lsum = 0.f, o = 0.f;
+        if (M != kNegInf) {
+          for (int j0 = 0; j0 < n; j0 += 8) {
+            float mv[8], lv[8], ov[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int sl = j0 + j == 0 ? first_slot : 2 * (ca + j0 + j);
+              const float *pp = P.ws_part + static_cast<int64_t>(sl) * slot_floats;
+              const bool in = j0 + j < n;
+              mv[j] = in ? __ldcg(pp + r) : kNegInf;
+              lv[j] = in ? __ldcg(pp + 16 + r) : 0.f;
+              ov[j] = in ? __ldcg(pp + 32 + r * kHeadDim + c) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float wt = fast_exp2(mv[j] - M);
+              lsum += lv[j] * wt;
+              o += ov[j] * wt;
+            }
+          }
+        }
+        write_row(P, hq0 + r, c, M, lsum, o);
+      }
+      if (threadIdx.x == 0) P.ws_cnt[sid] = 0u;  // leave the workspace ready for the next call
+    }
+  }
+  __syncthreads();  // the merge area is reused by the next piece
+}
+
+template <int NSTAGE, bool HIROWS>
+__global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(16) uint32_t zero_slot[4];
+  __shared__ int sh_info[3];  // U, batch row of this CTA's first unit (-1: none), that row's first unit
+  __shared__ int sh_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x, nctas = gridDim.x;
+  const int cap = min(P.cap_k, P.cap_v);
+
+  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts
+  if (warp == 0) {
+    int tot = 0;
+    for (int b0 = 0; b0 < P.B; b0 += 32) {
+      const int b = b0 + lane;
+      tot += b < P.B ? n_chunks(row_len(P, b, cap)) : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    tot *= P.Hkv;
+    const int u0 = range_start(cta, tot, nctas);
+    int row = -1, row_start = 0, before = 0;
+    for (int b0 = 0; b0 < P.B && u0 < tot; b0 += 32) {
+      const int b = b0 + lane;
+      const int n = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, before + incl > u0);
+      if (hit != 0u) {
+        const int f = __ffs(hit) - 1;
+        row = b0 + f;
+        row_start = before + __shfl_sync(0xffffffffu, incl - n, f);
+        break;
+      }
+      before += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      sh_info[0] = tot;
+      sh_info[1] = row;
+      sh_info[2] = row_start;
+    }
+  }
+  if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
+  uint8_t *wbase = smem + warp * P.warp_bytes;
+  uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // [32 rows][8 half words] u16 prefixes
+  const uint32_t bars = smem_addr(htab + 512);     // NSTAGE mbarriers of this warp
+  float *mer = reinterpret_cast<float *>(smem + kWarps * P.warp_bytes);
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < NSTAGE; ++i) mbar_init(bars + 8 * i, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  const int U = sh_info[0];
+  const int u0 = range_start(cta, U, nctas), u1 = range_start(cta + 1, U, nctas);
+
+  // ---- rows this CTA reports on: device error flags, and the output of rows with no tokens
+  for (int b = cta; b < P.B; b += nctas) {
+    uint32_t bits = 0;
+    const int L = row_len(P, b, cap, bits);
+    if (threadIdx.x == 0 && bits != 0u && P.err != nullptr) atomicOr(P.err, bits);
+    if (L == 0) {
+      uint16_t *o = P.out + static_cast<int64_t>(b) * P.Hq * kHeadDim;
+      for (int i = threadIdx.x; i < P.Hq * kHeadDim; i += kThreads) o[i] = 0;
+      if (P.lse != nullptr)
+        for (int i = threadIdx.x; i < P.Hq; i += kThreads) P.lse[static_cast<int64_t>(b) * P.Hq + i] = kNegInf;
+    }
+  }
+  if (sh_info[1] < 0) return;  // an empty range at the end of the sequence
+
+  Stream first;
+  first.b = sh_info[1];
+  first.n = n_chunks(row_len(P, first.b, cap));
+  first.g = (u0 - sh_info[2]) / first.n;
+  first.start = sh_info[2] + first.g * first.n;
+
+  // ---- fused decode step: compress the new token of every stream whose new-token chunk lies in
+  // this range (warp 0: K, warp 1: V) before any chunk is copied in
+  if (P.pos != nullptr) {
+    Stream st = first;
+    bool any = false;
+    while (st.start < u1) {
+      const int p = P.pos[st.b];
+      if (st.n > 0 && p >= 0 && p < cap) {
+        const int unit = st.start + p / kChunk;
+        if (unit >= u0 && unit < u1) {
+          any = true;
+          if (warp < 2) {
+            const bool kside = warp == 0;
+            const uint16_t *src =
+                kside ? P.kn + st.b * P.kn_sb + st.g * P.kn_sh : P.vn + st.b * P.vn_sb + st.g * P.vn_sh;
+            const int keep = kside ? P.keep_k : P.keep_v;
+            const int64_t slot = (static_cast<int64_t>(st.b) * P.Hkv + st.g) * (kside ? P.cap_k : P.cap_v) + p;
+            uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + slot * kWords;
+            uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + slot * keep;
+            warp_compress_vector(src, keep, bm, vals, lane);
+          }
+        }
+      }
+      if (!next_stream(P, cap, st)) break;
+    }
+    if (any) {
+      fence_proxy_async_global();  // these stores before the bulk copies that read them
+      __syncthreads();
+    }
+  }
+
+  // ---- the warp's chunks: units u0 + warp + 4j of the range, through a ring of NSTAGE buffers
+  const uint32_t za = smem_addr(zero_slot);
+  const uint32_t stage_bytes_tx = 512 + 32 * (P.keep_k + P.keep_v);
+  Stream ps = first;        // producer: stream of the next unit to copy in
+  int punit = u0 + warp;    // producer: next unit
+  int pitem = 0;            // producer: items issued
+  auto produce = [&]() {
+    if (punit >= u1) return;
+    while (punit >= ps.end()) next_stream(P, cap, ps);
+    if (lane == 0) {
+      const int slot = pitem % NSTAGE;
+      const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
+      const uint32_t bar = bars + 8 * slot;
+      const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
+      const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
+      const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
+      fence_proxy_async_smem();  // earlier generic writes to this buffer come before the copy
+      mbar_expect_tx(bar, stage_bytes_tx);
+      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
+      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
+    }
+    ++pitem;
+    punit += kWarps;
+  };
+#pragma unroll
+  for (int i = 0; i < NSTAGE; ++i) produce();
+
+  Stream cs = first;
+  int cunit = u0 + warp, citem = 0;
+  bool timed_out = false;
+  Acc<HIROWS> acc;
+  uint32_t qa[8][4];
+  for (;;) {
+    const int seg_a = max(cs.start, u0), seg_e = min(cs.end(), u1);
+    const int L = row_len(P, cs.b, cap);
+    load_q<HIROWS>(P, cs.b, cs.g, lane, qa);
+    acc.reset();
+#pragma unroll 1
+    for (; cunit < seg_e; cunit += kWarps, ++citem) {
+      const int slot = citem % NSTAGE;
+      uint8_t *stage = wbase + slot * P.stage_bytes;
+      if (!mbar_wait(bars + 8 * slot, (citem / NSTAGE) & 1, timed_out ? kWaitCyclesAfter : kWaitCycles))
+        timed_out = true;
+      consume_chunk<HIROWS>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, lane, qa, acc);
+      __syncwarp();
+      produce();  // the unit NSTAGE items ahead goes into the buffer just read
+    }
+    flush_piece<HIROWS>(P, acc, mer, warp, lane, cs, seg_a, u0, U, cta, nctas, &sh_flag);
+    if (seg_e >= u1) break;
+    bool more;
+    do {
+      more = next_stream(P, cap, cs);
+    } while (more && cs.n == 0);
+    if (!more) break;
+  }
+  if (timed_out && lane == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------------------------ host side
+using SparseFn = void (*)(const DecodeParams);
+
+template <int NSTAGE>
+SparseFn pick_rows(bool hirows) {
+  return hirows ? sparse_decode_kernel<NSTAGE, true> : sparse_decode_kernel<NSTAGE, false>;
+}
+
+SparseFn pick_sparse(int nstage, bool hirows) {
+  switch (nstage) {
+    case 2: return pick_rows<2>(hirows);
+    case 3: return pick_rows<3>(hirows);
+    default: return pick_rows<4>(hirows);
+  }
+}
+
+int sparse_slot(int nstage, bool hirows) { return 20 + 2 * nstage + (hirows ? 1 : 0); }
+
+constexpr int kMinUnitsPerCta = 2 * kWarps;  // at least two chunks per warp
+constexpr int kMaxCtasPerSm = 4;
+constexpr int kCtaSmemBudget = 56000;        // four CTAs per SM fit in 228 KB with this much each
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+int sms_of_current_device() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+  if (dev >= 0 && dev < 64) cached[dev] = sms;
+  return sms;
+}
+
+// resident CTAs per SM, cached per (device, kernel, smem) so that planning stays capture-safe
+cudaError_t resident_ctas(SparseFn fn, int slot, int smem, int *per_sm) {
+  static int cache_smem[64][32];
+  static int cache_val[64][32];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < 64 && slot >= 0 && slot < 32;
+  if (cacheable && cache_smem[dev][slot] == smem && cache_val[dev][slot] > 0) {
+    *per_sm = cache_val[dev][slot];
+    return cudaSuccess;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, fn, kThreads, smem);
+  if (e == cudaSuccess && cacheable) {
+    cache_smem[dev][slot] = smem;
+    cache_val[dev][slot] = *per_sm;
+  }
+  return e;
+}
+
+}  // namespace
+
+int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_sm) {
+  const long long streams = static_cast<long long>(B) * Hkv;
+  const long long units = streams * ((max_len + kChunk - 1) / kChunk);
+  long long ctas;
+  if (forced_splits > 0) {
+    ctas = forced_splits * streams;
+  } else {
+    ctas = static_cast<long long>(sms_of_current_device()) * per_sm;
+    const long long by_len = units / kMinUnitsPerCta;
+    ctas = by_len < ctas ? by_len : ctas;
+  }
+  ctas = ctas > units ? units : ctas;
+  ctas = ctas > (1 << 20) ? (1 << 20) : ctas;
+  return ctas < 1 ? 1 : static_cast<int>(ctas);
+}
+
+size_t sparse_workspace_bytes(int B, int Hkv, int G, int ctas) {
+  const size_t cnt = ((static_cast<size_t>(B) * Hkv * 4 + 255) / 256) * 256;
+  return cnt + static_cast<size_t>(2) * ctas * (32 + static_cast<size_t>(G) * kHeadDim) * 4;
+}
+
+size_t sparse_workspace_bound(int B, int Hkv, int G, int max_len, int forced_splits) {
+  return sparse_workspace_bytes(B, Hkv, G, sparse_decode_ctas(B, Hkv, max_len, forced_splits, kMaxCtasPerSm));
+}
+
+cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
+                        DecodePlan *plan) {
+  const bool hirows = G > 8;
+  const int stage_bytes = round_up(512 + 32 * (keep_k + keep_v), 128);
+  const int merge_bytes = (2 * kWarps * 16 + kWarps * G * kHeadDim) * 4;
+  auto warp_bytes_of = [&](int ns) { return round_up(ns * stage_bytes + 512 + 8 * ns, 128); };
+  int nstage = 2;
+  for (int ns = 4; ns > 2; --ns)
+    if (kWarps * warp_bytes_of(ns) + merge_bytes <= kCtaSmemBudget) {
+      nstage = ns;
+      break;
+    }
+  const int warp_bytes = warp_bytes_of(nstage);
+  const int smem = kWarps * warp_bytes + merge_bytes;
+  SparseFn fn = pick_sparse(nstage, hirows);
+  const int slot = sparse_slot(nstage, hirows);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), slot, smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = resident_ctas(fn, slot, smem, &per_sm);
+  if (e != cudaSuccess) return e;
+  per_sm = per_sm < 1 ? 1 : (per_sm > kMaxCtasPerSm ? kMaxCtasPerSm : per_sm);
+  plan->splits = sparse_decode_ctas(B, Hkv, max_len, forced_splits, per_sm);
+  plan->chunks_per_split = 0;
+  plan->nstage = nstage;
+  plan->stage_bytes = stage_bytes;
+  plan->warp_bytes = warp_bytes;
+  plan->smem_bytes = smem;
+  return cudaSuccess;
+}
+
+cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+  SparseFn fn = pick_sparse(plan.nstage, p.G > 8);
+  fn<<<plan.splits, kThreads, plan.smem_bytes, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace mustafar

@@ -40,6 +40,7 @@ struct DecodeParams {
   int stage_bytes, warp_bytes;
   uint16_t *out;
   float *lse;
+  float *ws_part;     // sparse kernel: [2 * ctas][32 + G*128] partial (m, l, o) slots
   float *ws_o;        // [B*Hq][splits][128]
   float *ws_ml;       // [B*Hq][splits][2]
   uint32_t *ws_cnt;   // [B*Hkv]
@@ -67,5 +68,15 @@ cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int kee
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int splits);
 int decode_split_bound(int B, int Hkv, int max_len);
 cudaError_t launch_decode(bool sparse, const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
+
+// Sparse decode over the compressed caches (one wave of CTAs over the end-to-end chunk sequence):
+// plan->splits holds the CTA count.
+cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
+                        DecodePlan *plan);
+cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
+int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_sm);
+size_t sparse_workspace_bytes(int B, int Hkv, int G, int ctas);
+// workspace that suffices for any plan of these shapes (assumes the most resident CTAs per SM)
+size_t sparse_workspace_bound(int B, int Hkv, int G, int max_len, int forced_splits);
 
 }  // namespace mustafar

@@ -313,13 +313,22 @@ __device__ __forceinline__ void write_row(const DecodeParams &P, int64_t hq, int
   if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
 }
 
-// End of one piece [seg_a, seg_e) of stream st: the four warps merge their (m, l, o) in shared
-// memory (`mer`: m[4][16], l[4][16], o[4][G][128] fp32); a stream held by this CTA alone is
-// written out, otherwise the CTA's partial goes to its workspace slot and the last CTA of the
-// stream merges all partials.  Called by every thread of the CTA.
+// A piece of a stream that other CTAs share: this CTA's partial is in the workspace, and the
+// ticket is taken when the CTA has finished its whole range.
+struct Pending {
+  int b, g;        // the stream
+  int ca, cb;      // the CTAs holding part of it
+  int first_slot;  // workspace slot of CTA ca's partial (CTA ca + j > ca uses slot 2 (ca + j))
+};
+
+// End of one piece [seg_a, ...) of stream st: the four warps merge their (m, l, o) in shared
+// memory (`mer`: m[4][16], l[4][16], o[4][G][128] fp32).  A stream held by this CTA alone is
+// written out; otherwise the CTA's partial goes to its workspace slot and the piece is queued in
+// `pend`.  Called by every thread of the CTA.
 template <bool HIROWS>
 __device__ void flush_piece(const DecodeParams &P, Acc<HIROWS> &acc, float *mer, int warp, int lane,
-                            const Stream &st, int seg_a, int u0, int U, int cta, int nctas, int *sh_flag) {
+                            const Stream &st, int seg_a, int u0, int U, int cta, int nctas, Pending *pend,
+                            int *npend) {
   const int G = P.G, gq = lane >> 2, qq = lane & 3;
   float *sm_m = mer, *sm_l = mer + kWarps * 16, *sm_o = mer + 2 * kWarps * 16;
 #pragma unroll
@@ -367,11 +376,10 @@ __device__ void flush_piece(const DecodeParams &P, Acc<HIROWS> &acc, float *mer,
   // the CTAs holding part of this stream: ca .. cb (an empty range that starts exactly where
   // the stream starts belongs to no stream)
   const int ca = cta_of(st.start, U, nctas), cb = cta_of(st.end() - 1, U, nctas);
-  const bool mine = cta >= ca && cta <= cb;
-  const int slot_floats = 32 + G * kHeadDim;
-  const int c = threadIdx.x;  // output channel
-  const int64_t hq0 = static_cast<int64_t>(st.b) * P.Hq + static_cast<int64_t>(st.g) * G;
-  if (mine) {
+  if (cta >= ca && cta <= cb) {
+    const int slot_floats = 32 + G * kHeadDim;
+    const int c = threadIdx.x;  // output channel
+    const int64_t hq0 = static_cast<int64_t>(st.b) * P.Hq + static_cast<int64_t>(st.g) * G;
     float *part = P.ws_part + static_cast<int64_t>(2 * cta + (seg_a == u0 ? 0 : 1)) * slot_floats;
     for (int r = 0; r < G; ++r) {
       float M = kNegInf;
@@ -396,60 +404,82 @@ __device__ void flush_piece(const DecodeParams &P, Acc<HIROWS> &acc, float *mer,
         }
       }
     }
-  }
-  if (mine && ca != cb) {
-    // ---- last CTA of this stream merges every partial (no waiting: an atomic ticket)
-    __threadfence();
-    __syncthreads();
-    const int sid = st.b * P.Hkv + st.g;
-    if (threadIdx.x == 0) {
-      const uint32_t ticket = atomicAdd(P.ws_cnt + sid, 1u);
-      *sh_flag = ticket == static_cast<uint32_t>(cb - ca);
-    }
-    __syncthreads();
-    if (*sh_flag) {
-      __threadfence();
-      const int n = cb - ca + 1;
-      const int first_slot = 2 * ca + (range_start(ca, U, nctas) < st.start ? 1 : 0);
-      for (int r = 0; r < G; ++r) {
-        float M = kNegInf;
-        for (int j0 = 0; j0 < n; j0 += 8) {  // 8 loads in flight per step
-          float mv[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int sl = j0 + j == 0 ? first_slot : 2 * (ca + j0 + j);
-            mv[j] = j0 + j < n ? __ldcg(P.ws_part + static_cast<int64_t>(sl) * slot_floats + r) : kNegInf;
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) M = fmaxf(M, mv[j]);
-        }
-        float lsum = 0.f, o = 0.f;
-        if (M != kNegInf) {
-          for (int j0 = 0; j0 < n; j0 += 8) {
-            float mv[8], lv[8], ov[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int sl = j0 + j == 0 ? first_slot : 2 * (ca + j0 + j);
-              const float *pp = P.ws_part + static_cast<int64_t>(sl) * slot_floats;
-              const bool in = j0 + j < n;
-              mv[j] = in ? __ldcg(pp + r) : kNegInf;
-              lv[j] = in ? __ldcg(pp + 16 + r) : 0.f;
-              ov[j] = in ? __ldcg(pp + 32 + r * kHeadDim + c) : 0.f;
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float wt = fast_exp2(mv[j] - M);
-              lsum += lv[j] * wt;
-              o += ov[j] * wt;
-            }
-          }
-        }
-        write_row(P, hq0 + r, c, M, lsum, o);
-      }
-      if (threadIdx.x == 0) P.ws_cnt[sid] = 0u;  // leave the workspace ready for the next call
+    if (ca != cb && threadIdx.x == 0) {
+      Pending &pd = pend[(*npend)++];
+      pd.b = st.b;
+      pd.g = st.g;
+      pd.ca = ca;
+      pd.cb = cb;
+      pd.first_slot = 2 * ca + (range_start(ca, U, nctas) < st.start ? 1 : 0);
     }
   }
   __syncthreads();  // the merge area is reused by the next piece
+}
+
+// The last CTA of a shared stream: merge its n = cb - ca + 1 partials and write out / lse.
+// Latency-bound, so every load of a block of 16 partials (their m, l and this thread's float4 of
+// o) is issued before any is used; blocks are combined with an online rescale.  Thread t handles
+// the (row, 4-channel quad) pairs t, t+128, ... (G <= 16 -> at most 4).
+__device__ void merge_stream(const DecodeParams &P, const Pending &pd) {
+  const int G = P.G, n = pd.cb - pd.ca + 1;
+  const int slot_floats = 32 + G * kHeadDim;
+  const int64_t hq0 = static_cast<int64_t>(pd.b) * P.Hq + static_cast<int64_t>(pd.g) * G;
+  for (int it = threadIdx.x; it < G * (kHeadDim / 4); it += kThreads) {
+    const int r = it >> 5, q4 = it & 31;
+    float M = kNegInf, Lsum = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < n; j0 += 16) {
+      float mv[16], lv[16];
+      float4 ov[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int j = j0 + u;
+        if (j < n) {
+          const int slot = j == 0 ? pd.first_slot : 2 * (pd.ca + j);
+          const float *pp = P.ws_part + static_cast<int64_t>(slot) * slot_floats;
+          mv[u] = __ldcg(pp + r);
+          lv[u] = __ldcg(pp + 16 + r);
+          ov[u] = __ldcg(reinterpret_cast<const float4 *>(pp + 32 + r * kHeadDim) + q4);
+        } else {
+          mv[u] = kNegInf;
+          lv[u] = 0.f;
+          ov[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mb = M;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) mb = fmaxf(mb, mv[u]);
+      const float base = mb == kNegInf ? 0.f : mb;
+      const float a = fast_exp2(M - base);
+      Lsum *= a;
+      o.x *= a;
+      o.y *= a;
+      o.z *= a;
+      o.w *= a;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float wt = fast_exp2(mv[u] - base);
+        Lsum += wt * lv[u];
+        o.x += wt * ov[u].x;
+        o.y += wt * ov[u].y;
+        o.z += wt * ov[u].z;
+        o.w += wt * ov[u].w;
+      }
+      M = mb;
+    }
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    *reinterpret_cast<uint2 *>(P.out + (hq0 + r) * kHeadDim + 4 * q4) =
+        make_uint2(pack_half2(o.x * inv, o.y * inv), pack_half2(o.z * inv, o.w * inv));
+    if (q4 == 0 && P.lse != nullptr) P.lse[hq0 + r] = Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : kNegInf;
+  }
+}
+
+// Ticket of a shared stream: acq_rel at gpu scope, so the release covers this CTA's partial
+// stores (ordered before it by the CTA barrier) and the acquire covers the other CTAs' ones.
+__device__ __forceinline__ uint32_t take_ticket(uint32_t *counter) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;\n" : "=r"(old) : "l"(counter) : "memory");
+  return old;
 }
 
 template <int NSTAGE, bool HIROWS>
@@ -457,26 +487,37 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
   __shared__ int sh_info[3];  // U, batch row of this CTA's first unit (-1: none), that row's first unit
-  __shared__ int sh_flag;
+  __shared__ Pending sh_pend[2];
+  __shared__ int sh_npend, sh_last[2];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x, nctas = gridDim.x;
   const int cap = min(P.cap_k, P.cap_v);
 
-  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts
+  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts (rows up
+  // to 128 are read once, in one round of independent loads, and kept in registers)
   if (warp == 0) {
+    int nrow[4];
     int tot = 0;
-    for (int b0 = 0; b0 < P.B; b0 += 32) {
-      const int b = b0 + lane;
-      tot += b < P.B ? n_chunks(row_len(P, b, cap)) : 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int b = lane + 32 * i;
+      nrow[i] = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
+      tot += nrow[i];
     }
+    for (int b = 128 + lane; b < P.B; b += 32) tot += P.Hkv * n_chunks(row_len(P, b, cap));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    tot *= P.Hkv;
     const int u0 = range_start(cta, tot, nctas);
     int row = -1, row_start = 0, before = 0;
     for (int b0 = 0; b0 < P.B && u0 < tot; b0 += 32) {
       const int b = b0 + lane;
-      const int n = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
+      int n;
+      if (b0 < 128) {
+        const int i = b0 >> 5;
+        n = i == 0 ? nrow[0] : i == 1 ? nrow[1] : i == 2 ? nrow[2] : nrow[3];
+      } else {
+        n = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
+      }
       int incl = n;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -499,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     }
   }
   if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) sh_npend = 0;
   uint8_t *wbase = smem + warp * P.warp_bytes;
   uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // [32 rows][8 half words] u16 prefixes
   const uint32_t bars = smem_addr(htab + 512);     // NSTAGE mbarriers of this warp
@@ -565,32 +607,37 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
 
   // ---- the warp's chunks: units u0 + warp + 4j of the range, through a ring of NSTAGE buffers
   const uint32_t za = smem_addr(zero_slot);
-  const uint32_t stage_bytes_tx = 512 + 32 * (P.keep_k + P.keep_v);
-  Stream ps = first;        // producer: stream of the next unit to copy in
-  int punit = u0 + warp;    // producer: next unit
-  int pitem = 0;            // producer: items issued
-  auto produce = [&]() {
+  // producer state of each warp in shared memory (only lane 0 walks it), to keep registers for
+  // the chunk math: the stream of the next unit to copy in, and that unit
+  __shared__ Stream sh_ps[kWarps];
+  __shared__ int sh_punit[kWarps];
+  if (lane == 0) {
+    sh_ps[warp] = first;
+    sh_punit[warp] = u0 + warp;
+  }
+  __syncwarp();
+  auto produce = [&](int item) {
+    if (lane != 0) return;
+    int punit = sh_punit[warp];
     if (punit >= u1) return;
+    Stream ps = sh_ps[warp];
     while (punit >= ps.end()) next_stream(P, cap, ps);
-    if (lane == 0) {
-      const int slot = pitem % NSTAGE;
-      const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
-      const uint32_t bar = bars + 8 * slot;
-      const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
-      const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
-      const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
-      fence_proxy_async_smem();  // earlier generic writes to this buffer come before the copy
-      mbar_expect_tx(bar, stage_bytes_tx);
-      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
-      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
-      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
-    }
-    ++pitem;
-    punit += kWarps;
+    const int slot = item % NSTAGE;
+    const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
+    const uint32_t bar = bars + 8 * slot;
+    const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
+    const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
+    const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
+    mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
+    bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+    bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+    bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
+    bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
+    sh_ps[warp] = ps;
+    sh_punit[warp] = punit + kWarps;
   };
-#pragma unroll
-  for (int i = 0; i < NSTAGE; ++i) produce();
+#pragma unroll 1
+  for (int i = 0; i < NSTAGE; ++i) produce(i);
 
   Stream cs = first;
   int cunit = u0 + warp, citem = 0;
@@ -610,9 +657,9 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
         timed_out = true;
       consume_chunk<HIROWS>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, lane, qa, acc);
       __syncwarp();
-      produce();  // the unit NSTAGE items ahead goes into the buffer just read
+      produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
     }
-    flush_piece<HIROWS>(P, acc, mer, warp, lane, cs, seg_a, u0, U, cta, nctas, &sh_flag);
+    flush_piece<HIROWS>(P, acc, mer, warp, lane, cs, seg_a, u0, U, cta, nctas, sh_pend, &sh_npend);
     if (seg_e >= u1) break;
     bool more;
     do {
@@ -621,6 +668,21 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     if (!more) break;
   }
   if (timed_out && lane == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_TIMEOUT);
+
+  // ---- tickets for the pieces shared with other CTAs; the last CTA of a stream merges it
+  const int np = sh_npend;  // the partial stores are ordered before this by flush_piece's barrier
+  if (np > 0) {
+    if (threadIdx.x == 0)
+      for (int i = 0; i < np; ++i)
+        sh_last[i] = take_ticket(P.ws_cnt + sh_pend[i].b * P.Hkv + sh_pend[i].g) ==
+                     static_cast<uint32_t>(sh_pend[i].cb - sh_pend[i].ca);
+    __syncthreads();
+    for (int i = 0; i < np; ++i) {
+      if (!sh_last[i]) continue;
+      merge_stream(P, sh_pend[i]);
+      if (threadIdx.x == 0) P.ws_cnt[sh_pend[i].b * P.Hkv + sh_pend[i].g] = 0u;  // ready for the next call
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------ host side
@@ -687,7 +749,11 @@ int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_s
   if (forced_splits > 0) {
     ctas = forced_splits * streams;
   } else {
-    ctas = static_cast<long long>(sms_of_current_device()) * per_sm;
+    // one wave; when a whole number of CTAs per stream fills nearly all of it, take that, so that
+    // (for equal row lengths) no range crosses a stream boundary and no piece needs an extra merge
+    const long long wave = static_cast<long long>(sms_of_current_device()) * per_sm;
+    const long long per_stream = wave / streams;
+    ctas = per_stream >= 1 && per_stream * streams * 20 >= wave * 19 ? per_stream * streams : wave;
     const long long by_len = units / kMinUnitsPerCta;
     ctas = by_len < ctas ? by_len : ctas;
   }

@@ -90,7 +90,7 @@ def decode_algorithmic_bytes(B, Hq, Hkv, d, lens, kK, kV):
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("common.cuh", "select.cuh", "decode_attn.cu"):
+    for f in ("common.cuh", "select.cuh", "decode_sparse.cu"):
         with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -325,6 +325,9 @@ def main(argv=None):
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="ncu case: build the workload, run this many eager fused steps over the rotated "
                          "caches, and exit without timing")
+    ap.add_argument("--profile-shape", default=None,
+                    help="ncu case: 'B,L,sK,sV' -- GQA 32/8 decode over two rotating compressed-cache copies "
+                         "of that shape (larger than L2 for B*L >= 64k), six mustafar_decode_attn launches, no timing")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
@@ -333,6 +336,34 @@ def main(argv=None):
         from unstructured_sparse_kv_b200 import suite
         M.load()
         suite.run(args.suite, measured_peak()[0], tuple(args.suite_parts.split(",")))
+        return 0
+    if args.profile_shape:
+        import torch
+        import unstructured_sparse_kv_b200 as M
+        from unstructured_sparse_kv_b200 import synth
+        M.load()
+        B, L = (int(x) for x in args.profile_shape.split(",")[:2])
+        sK, sV = (float(x) for x in args.profile_shape.split(",")[2:4])
+        Hq, Hkv, d, dev = 32, 8, 128, torch.device("cuda", 0)
+        K, V = synth.keys(B, Hkv, L, d, 5, dev), synth.values(B, Hkv, L, d, 5, dev)
+        q = synth.queries(B, Hq, d, 5, dev)
+        seq = torch.full((B,), L, dtype=torch.int32, device=dev)
+        copies = []
+        for _ in range(2):
+            kc, vc = M.CompressedCache(B, Hkv, L, sK, device=dev), M.CompressedCache(B, Hkv, L, sV, device=dev)
+            M.mustafar_compress(K, L, sK, kc)
+            M.mustafar_compress(V, L, sV, vc)
+            copies.append((kc, vc))
+        del K, V
+        out = torch.empty_like(q)
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+        ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, L), dtype=torch.uint8, device=dev)
+        for i in range(6):
+            kc, vc = copies[i % 2]
+            M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0, out=out, lse=lse, workspace=ws)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": "decode_attn", "batch": B, "context": L, "sparsity_k": sK,
+                          "sparsity_v": sV, "launches": 6}))
         return 0
     if args.profile_launches > 0:
         import torch

@@ -178,7 +178,7 @@ int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t
   if (!dense && (keep_k < 1 || keep_k > kHeadDim || keep_v < 1 || keep_v > kHeadDim)) return -1;
   DecodePlan plan;
   if (dense) {
-    if (plan_decode(false, batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, &plan) != cudaSuccess) return -1;
+    if (plan_dense(batch, num_kv_heads, 4, max_len, 0, &plan) != cudaSuccess) return -1;
     return plan.splits;
   }
   // the sparse kernel cuts the end-to-end chunk sequence into CTA ranges; report the CTAs per stream
@@ -213,7 +213,7 @@ mustafar_status run_decode(bool sparse, DecodeParams &p, int max_len, int num_sp
                            size_t workspace_bytes, const char *name, cudaStream_t stream) {
   if (sparse) return run_sparse(p, max_len, num_splits, workspace, workspace_bytes, name, stream);
   DecodePlan plan;
-  cudaError_t e = plan_decode(sparse, p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, &plan);
+  cudaError_t e = plan_dense(p.B, p.Hkv, p.G, max_len, num_splits, &plan);
   if (e != cudaSuccess) return cuda_fail(e, name);
   p.num_splits = plan.splits;
   p.chunks_per_split = plan.chunks_per_split;
@@ -232,7 +232,7 @@ mustafar_status run_decode(bool sparse, DecodeParams &p, int max_len, int num_sp
     p.ws_ml = reinterpret_cast<float *>(w + cnt);
     p.ws_o = reinterpret_cast<float *>(w + cnt + ml);
   }
-  e = launch_decode(sparse, p, plan, stream);
+  e = launch_dense(p, plan, stream);
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, name);
 }
 

@@ -1,38 +1,25 @@
-// decode_attn.cu - split-K decode attention over the bitmap-compressed caches, and the
-// dense fp16 baseline built on the same skeleton.
+// decode_attn.cu - dense fp16 decode attention: the baseline the pages compare the sparse
+// kernel against (MUSTAFAR summary, atlas.scime.ai, "Experimental setup": dense attention over
+// uncompressed caches).  Same math as the sparse kernel, over [B][Hkv][cap][128] fp16 caches:
+//   out = softmax(scale * q K^T) V
 //
-// Computes, for each batch row b and q head hq (kv head g = hq / G):
-//   out = softmax(scale * q K~^T) V~  over the pruned caches K~, V~
-// directly from the compressed format (Mustafar abstract, catalyzex author page: a custom
-// attention kernel that computes directly over the compressed caches; MUSTAFAR summary,
-// atlas.scime.ai, "Approach": an SpMV-style attention kernel over the bitmap format).
-//
-// Work decomposition (B200-first, not the pages' design):
+// Work decomposition:
 // * grid = (splits, Hkv, B); a CTA owns a contiguous range of 16-token chunks of one
 //   (b, kv head) stream and the whole GQA group of that kv head.
-// * each of the CTA's 4 warps is an independent pipeline over every 4th chunk of the
-//   range: a cp.async ring (NSTAGE deep) stages the chunk's compressed bytes (16 bitmap
-//   rows + 16*k packed values, for K and for V) in the warp's own shared memory, so the
-//   loop needs no CTA barrier.
-// * S = Q K~^T and O^T += V~^T P^T run as mma.sync m16n8k16 (fp16 in, fp32 accumulate):
-//   S has the G q heads (padded to 16) as M and the 16 tokens as N; O^T has the 128
-//   channels as M (8 m-tiles), the heads as N and the tokens as K, so the fp32 accumulator
-//   is 128 x 8 (32 registers per lane) for G <= 8.  Online softmax per head, log2 domain.
-// * no dense tile is ever built: each lane expands, straight into its mma fragment
-//   registers, exactly the (token, channel) elements the fragment layouts give it, with one
-//   predicated 16-bit shared load per channel (the bit of the bitmap is the predicate; the
-//   value pointer advances past each kept value).  The contraction index is permuted so
-//   that a lane's channels are one contiguous bitmap word (K: 32 channels of each of its
-//   2 tokens) or half-word (V: 16 channels of each of its 4 tokens); Q's fragments use the
-//   same permutation and the output columns are put back in order when the warps merge.
-// * warps merge in shared memory; with splits > 1 each CTA writes its (m, l, o) partial to
-//   the workspace and the last CTA of the stream (atomic ticket, no spin-wait) merges all
-//   splits in a fixed order and writes out / lse.
+// * each of the CTA's 4 warps is an independent pipeline over every 4th chunk of the range: a
+//   cp.async ring (NSTAGE deep) stages the chunk's 16 K rows and 16 V rows (padded to 272 B)
+//   in the warp's own shared memory, so the loop needs no CTA barrier.
+// * S = Q K^T and O^T += V^T P^T run as mma.sync m16n8k16 (fp16 in, fp32 accumulate) on
+//   ldmatrix (K) / ldmatrix.trans (V) fragments: S has the G q heads (padded to 16) as M and
+//   the 16 tokens as N; O^T has the 128 channels as M (8 m-tiles), the heads as N and the
+//   tokens as K.  Online softmax per head, log2 domain.
+// * warps merge in shared memory; with splits > 1 each CTA writes its (m, l, o) partial to the
+//   workspace and the last CTA of the stream (atomic ticket, no spin-wait) merges all splits in
+//   a fixed order and writes out / lse.
 #include <cfloat>
 
 #include "common.cuh"
 #include "internal.h"
-#include "select.cuh"
 
 namespace mustafar {
 
@@ -40,99 +27,30 @@ constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = 32 * kDecodeWarps;
 constexpr float kNegInf = -INFINITY;
 
-template <bool SPARSE>
 __device__ __forceinline__ void issue_chunk(const DecodeParams &P, int64_t stream, int c, uint8_t *stage,
                                             int lane) {
-  if constexpr (SPARSE) {
-    const int64_t tk = stream * P.cap_k + static_cast<int64_t>(c) * kChunk;
-    const int64_t tv = stream * P.cap_v + static_cast<int64_t>(c) * kChunk;
-    const uint8_t *src_kb = reinterpret_cast<const uint8_t *>(P.kbm + tk * kWords);
-    const uint8_t *src_vb = reinterpret_cast<const uint8_t *>(P.vbm + tv * kWords);
-    const uint8_t *src_kv = reinterpret_cast<const uint8_t *>(P.kval + tk * P.keep_k);
-    const uint8_t *src_vv = reinterpret_cast<const uint8_t *>(P.vval + tv * P.keep_v);
-    const uint32_t dst = smem_addr(stage);
-    // bitmaps: 16 rows x 16 B for K then V (32 units of 16 B: one per lane)
-    {
-      const uint8_t *src = lane < 16 ? src_kb + lane * 16 : src_vb + (lane - 16) * 16;
-      cp_async16(dst + lane * 16, src);
-    }
-    const int uk = 2 * P.keep_k, uv = 2 * P.keep_v;  // 16-byte units of packed values (16*k*2/16)
-    for (int u = lane; u < uk; u += 32) cp_async16(dst + 512 + u * 16, src_kv + u * 16);
-    for (int u = lane; u < uv; u += 32) cp_async16(dst + 512 + uk * 16 + u * 16, src_vv + u * 16);
-  } else {
-    const int64_t row0 = (stream * P.cap_k + static_cast<int64_t>(c) * kChunk) * kHeadDim;
-    const uint8_t *src_k = reinterpret_cast<const uint8_t *>(P.kd + row0);
-    const uint8_t *src_v = reinterpret_cast<const uint8_t *>(P.vd + row0);
-    const uint32_t dst = smem_addr(stage);
+  const int64_t row0 = (stream * P.cap_k + static_cast<int64_t>(c) * kChunk) * kHeadDim;
+  const uint8_t *src_k = reinterpret_cast<const uint8_t *>(P.kd + row0);
+  const uint8_t *src_v = reinterpret_cast<const uint8_t *>(P.vd + row0);
+  const uint32_t dst = smem_addr(stage);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // 256 units of 16 B per tile, 8 per lane
-      const int u = lane + 32 * i;
-      const int r = u >> 4, j = u & 15;
-      cp_async16(dst + r * kRowBytes + j * 16, src_k + u * 16);
-      cp_async16(dst + kTileBytes + r * kRowBytes + j * 16, src_v + u * 16);
-    }
+  for (int i = 0; i < 8; ++i) {  // 256 units of 16 B per tile, 8 per lane
+    const int u = lane + 32 * i;
+    const int r = u >> 4, j = u & 15;
+    cp_async16(dst + r * kRowBytes + j * 16, src_k + u * 16);
+    cp_async16(dst + kTileBytes + r * kRowBytes + j * 16, src_v + u * 16);
   }
 }
 
-// x = (bits & MASK) ? the fp16 at shared address ra : 0 (read from the CTA's zero slot `za`);
-// ra advances past a taken value.  No branch and no register zeroing: pruned channels load the
-// zero slot, which every pruned lane of a warp reads at the same address (a broadcast).
-template <uint32_t MASK>
-__device__ __forceinline__ uint32_t take(uint32_t bits, uint32_t &ra, uint32_t za) {
-  uint32_t x;
-  asm volatile(
-      "{\n .reg .pred p;\n .reg .b32 t, a;\n and.b32 t, %2, %3;\n setp.ne.u32 p, t, 0;\n"
-      " selp.u32 a, %1, %4, p;\n ld.shared.u16 %0, [a];\n @p add.u32 %1, %1, 2;\n}\n"
-      : "=r"(x), "+r"(ra)
-      : "r"(bits), "n"(MASK), "r"(za)
-      : "memory");
-  return x;
-}
-
-// Expand the 32 channels of one bitmap word into 16 packed fp16 pairs (channels 2i, 2i+1).
-// The low and high half words advance two independent value pointers (ra, rb), interleaved.
-template <int I = 0>
-__device__ __forceinline__ void expand_word(uint32_t bits, uint32_t ra, uint32_t rb, uint32_t za,
-                                            uint32_t (&out)[16]) {
-  if constexpr (I < 8) {
-    const uint32_t a0 = take<(1u << (2 * I))>(bits, ra, za);
-    const uint32_t b0 = take<(1u << (2 * I + 16))>(bits, rb, za);
-    const uint32_t a1 = take<(1u << (2 * I + 1))>(bits, ra, za);
-    const uint32_t b1 = take<(1u << (2 * I + 17))>(bits, rb, za);
-    out[I] = __byte_perm(a0, a1, 0x5410);
-    out[I + 8] = __byte_perm(b0, b1, 0x5410);
-    expand_word<I + 1>(bits, ra, rb, za, out);
-  }
-}
-
-// Expand the 16 channels of a half word (bits 0..15 of `bits`) into 16 separate fp16 values.
-template <int I = 0>
-__device__ __forceinline__ void expand_half(uint32_t bits, uint32_t ra, uint32_t za, uint32_t (&out)[16]) {
-  if constexpr (I < 16) {
-    out[I] = take<(1u << I)>(bits, ra, za);
-    expand_half<I + 1>(bits, ra, za, out);
-  }
-}
-
-template <bool SPARSE, int NSTAGE, bool HIROWS>
-__global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) decode_kernel(const DecodeParams P) {
+template <int NSTAGE, bool HIROWS>
+__global__ void __launch_bounds__(kDecodeThreads, 3) dense_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int G = P.G;
-  const int cap = SPARSE ? min(P.cap_k, P.cap_v) : P.cap_k;
+  const int cap = P.cap_k;
   int L;
-  int append_at = -1;  // slot this CTA compresses the new token into (fused decode step), or -1
-  if (SPARSE && P.pos != nullptr) {
-    const int p = P.pos[b];
-    if (p < 0 || p >= cap) {
-      if (threadIdx.x == 0 && split == 0 && g == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_POS_RANGE);
-      L = p < 0 ? 0 : cap;
-    } else {
-      L = p + 1;
-      if ((p / kChunk) / P.chunks_per_split == split) append_at = p;  // the CTA that will read that chunk
-    }
-  } else {
+  {
     L = P.seq_len[b];
     if (L < 0 || L > cap) {
       if (threadIdx.x == 0 && split == 0 && g == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_LEN_RANGE);
@@ -148,27 +66,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
   const int64_t stream = static_cast<int64_t>(b) * P.Hkv + g;
 
   uint8_t *wbase = smem + warp * P.warp_bytes;
-  uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // sparse: [32 rows][8 half words] u16 prefixes
-  __shared__ __align__(16) uint32_t zero_slot[4];
-  if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
-  if (SPARSE && append_at >= 0 && warp < 2) {
-    // fused decode step: warp 0 compresses the new K token, warp 1 the new V token, into slot
-    // append_at of this stream; the fence makes them visible to the chunk loads below
-    const bool kside = warp == 0;
-    const uint16_t *src = kside ? P.kn + b * P.kn_sb + g * P.kn_sh : P.vn + b * P.vn_sb + g * P.vn_sh;
-    const int keep = kside ? P.keep_k : P.keep_v;
-    const int64_t slot = stream * (kside ? P.cap_k : P.cap_v) + append_at;
-    uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + slot * kWords;
-    uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + slot * keep;
-    warp_compress_vector(src, keep, bm, vals, lane);
-    __threadfence();
-  }
-  __syncthreads();
-  const uint32_t za = smem_addr(zero_slot);
 
-  // Q A-fragments (rows = q heads of the group, zero beyond G), 8 k-steps.  Sparse path: k-step
-  // ks, fragment column 2q+e is channel 32q+4ks+e and column 2q+8+e is 32q+4ks+2+e (the
-  // permutation that gives lane q the 32 channels of bitmap word q); dense path: natural order.
+  // Q A-fragments (rows = q heads of the group, zero beyond G), 8 k-steps, natural channel order.
   const int gq = lane >> 2, qq = lane & 3;
   uint32_t qa[8][4];
   {
@@ -176,8 +75,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     const bool r0 = gq < G, r1 = HIROWS && (gq + 8 < G);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const int c0 = SPARSE ? 32 * qq + 4 * ks : ks * 16 + 2 * qq;
-      const int c1 = SPARSE ? c0 + 2 : c0 + 8;
+      const int c0 = ks * 16 + 2 * qq;
+      const int c1 = c0 + 8;
       qa[ks][0] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + c0) : 0u;
       qa[ks][1] = r1 ? *reinterpret_cast<const uint32_t *>(qb + (gq + 8) * kHeadDim + c0) : 0u;
       qa[ks][2] = r0 ? *reinterpret_cast<const uint32_t *>(qb + gq * kHeadDim + c1) : 0u;
@@ -185,8 +84,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     }
   }
 
-  // O^T accumulators, m-tile mt.  Sparse: rows g / g+8 are channels 16g+2mt / 16g+2mt+1;
-  // dense: channels 16mt+g / 16mt+g+8.  Columns 2q, 2q+1 are heads; oh holds heads 8+2q, 8+2q+1.
+  // O^T accumulators, m-tile mt: rows g / g+8 are channels 16mt+g / 16mt+g+8.  Columns 2q, 2q+1
+  // are heads; oh holds heads 8+2q, 8+2q+1.
   float ot[8][4];
   float oh[HIROWS ? 8 : 1][4];
 #pragma unroll
@@ -198,7 +97,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
 
 #pragma unroll
   for (int i = 0; i < NSTAGE - 1; ++i) {
-    if (i < my_n) issue_chunk<SPARSE>(P, stream, c_begin + warp + kDecodeWarps * i, wbase + i * P.stage_bytes, lane);
+    if (i < my_n) issue_chunk(P, stream, c_begin + warp + kDecodeWarps * i, wbase + i * P.stage_bytes, lane);
     cp_async_commit();
   }
 
@@ -211,7 +110,7 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     {
       const int ni = i + NSTAGE - 1;
       if (ni < my_n)
-        issue_chunk<SPARSE>(P, stream, c_begin + warp + kDecodeWarps * ni, wbase + (ni % NSTAGE) * P.stage_bytes,
+        issue_chunk(P, stream, c_begin + warp + kDecodeWarps * ni, wbase + (ni % NSTAGE) * P.stage_bytes,
                             lane);
       cp_async_commit();
     }
@@ -225,47 +124,15 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     float s[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-    if constexpr (SPARSE) {
-      // per-row table: lane r (K rows 0-15, V rows 16-31) zeroes the bitmap of a token >= L in
-      // place and stores the popcount prefix of each of its row's 8 half words (u16 each)
-      {
-        uint4 *row = reinterpret_cast<uint4 *>(stage + lane * 16);
-        uint4 w = *row;
-        if (!full && t0 + (lane & 15) >= L) {
-          w = make_uint4(0u, 0u, 0u, 0u);
-          *row = w;
-        }
-        const uint32_t h0 = __popc(w.x & 0xFFFFu), c0 = __popc(w.x);
-        const uint32_t h1 = c0 + __popc(w.y & 0xFFFFu), c1 = c0 + __popc(w.y);
-        const uint32_t h2 = c1 + __popc(w.z & 0xFFFFu), c2 = c1 + __popc(w.z);
-        const uint32_t h3 = c2 + __popc(w.w & 0xFFFFu);
-        // half words 0..7 start at 0, h0, c0, h1, c1, h2, c2, h3 kept values
-        *reinterpret_cast<uint4 *>(htab + lane * 16) =
-            make_uint4(h0 << 16, c0 | (h1 << 16), c1 | (h2 << 16), c2 | (h3 << 16));
-      }
-      __syncwarp();
-      const uint32_t kvals = smem_addr(stage + 512);
+    const uint32_t kaddr = smem_addr(stage) + t_off;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
-        const uint32_t word = *reinterpret_cast<const uint32_t *>(stage + T * 16 + qq * 4);
-        const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
-        const uint32_t rbase = kvals + 2 * T * P.keep_k;
-        uint32_t kb[16];
-        expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
-      }
-    } else {
-      const uint32_t kaddr = smem_addr(stage) + t_off;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * 32);
-        mma_f16_16816(s[0], qa[ks], b0, b1);
-        mma_f16_16816(s[1], qa[ks], b2, b3);
-      }
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4(b0, b1, b2, b3, kaddr + ks * 32);
+      mma_f16_16816(s[0], qa[ks], b0, b1);
+      mma_f16_16816(s[1], qa[ks], b2, b3);
     }
+  
 
     // ---- scale into the log2 domain, mask tokens >= L, online softmax per row (= q head)
     float mx[2] = {kNegInf, kNegInf};
@@ -333,44 +200,15 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     const uint32_t pc1 = HIROWS ? pack_half2(s[1][2], s[1][3]) : 0u;
 
     // ---- O^T += V~^T P^T : 8 m-tiles of 16 channels
-    if constexpr (SPARSE) {
-      // this lane's A fragments cover channels 16g..16g+15 (half word g of the bitmap) of
-      // tokens 2q, 2q+1 (k = 2q, 2q+1) and 2q+8, 2q+9 (k = 2q+8, 2q+9)
-      const uint32_t vvals = smem_addr(stage + 512 + 32 * P.keep_k);
-      uint32_t va[8][4];
+    const uint32_t vaddr = smem_addr(stage + kTileBytes) + t_off;
 #pragma unroll
-      for (int pair = 0; pair < 2; ++pair) {
-        uint32_t x0[16], x1[16];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int T = 2 * qq + 8 * pair + e;
-          // half word gq of V row T: its 16 bits and the number of kept values before it
-          const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
-          const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
-          expand_half(bits, vvals + 2 * (T * P.keep_v + pre), za, e ? x1 : x0);
-        }
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          va[mt][2 * pair] = __byte_perm(x0[2 * mt], x1[2 * mt], 0x5410);
-          va[mt][2 * pair + 1] = __byte_perm(x0[2 * mt + 1], x1[2 * mt + 1], 0x5410);
-        }
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const uint32_t a[4] = {va[mt][0], va[mt][1], va[mt][2], va[mt][3]};
-        mma_f16_16816(ot[mt], a, pb0, pb1);
-        if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
-      }
-    } else {
-      const uint32_t vaddr = smem_addr(stage + kTileBytes) + t_off;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t a[4];
-        ldmatrix_x4_trans(a[0], a[1], a[2], a[3], vaddr + mt * 32);
-        mma_f16_16816(ot[mt], a, pb0, pb1);
-        if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
-      }
+    for (int mt = 0; mt < 8; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a[0], a[1], a[2], a[3], vaddr + mt * 32);
+      mma_f16_16816(ot[mt], a, pb0, pb1);
+      if constexpr (HIROWS) mma_f16_16816(oh[mt], a, pc0, pc1);
     }
+  
     __syncwarp();
   }
   cp_async_wait<0>();
@@ -400,8 +238,8 @@ __global__ void __launch_bounds__(kDecodeThreads, (SPARSE && !HIROWS) ? 4 : 3) d
     const int h0 = 2 * qq, h1 = 2 * qq + 1;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      const int ch0 = SPARSE ? 16 * gq + 2 * mt : 16 * mt + gq;  // channel of accumulator rows g
-      const int ch1 = SPARSE ? ch0 + 1 : ch0 + 8;                // and g+8
+      const int ch0 = 16 * mt + gq;  // channel of accumulator rows g
+      const int ch1 = ch0 + 8;       // and g+8
       if (h0 < G) {
         sm_o[(warp * G + h0) * kHeadDim + ch0] = ot[mt][0];
         sm_o[(warp * G + h0) * kHeadDim + ch1] = ot[mt][2];
@@ -503,26 +341,14 @@ namespace {
 
 using KernelFn = void (*)(const DecodeParams);
 
-template <bool SPARSE, int NSTAGE>
+template <int NSTAGE>
 KernelFn pick_rows(bool hirows) {
-  return hirows ? decode_kernel<SPARSE, NSTAGE, true> : decode_kernel<SPARSE, NSTAGE, false>;
+  return hirows ? dense_decode_kernel<NSTAGE, true> : dense_decode_kernel<NSTAGE, false>;
 }
 
-KernelFn pick_kernel(bool sparse, int nstage, bool hirows) {
-  if (sparse) {
-    switch (nstage) {
-      case 2: return pick_rows<true, 2>(hirows);
-      case 3: return pick_rows<true, 3>(hirows);
-      default: return pick_rows<true, 4>(hirows);
-    }
-  }
-  switch (nstage) {
-    case 2: return pick_rows<false, 2>(hirows);
-    default: return pick_rows<false, 3>(hirows);
-  }
-}
+KernelFn pick_kernel(int nstage, bool hirows) { return nstage == 2 ? pick_rows<2>(hirows) : pick_rows<3>(hirows); }
 
-int kernel_slot(bool sparse, int nstage, bool hirows) { return 1 + (sparse ? 0 : 8) + 2 * nstage + (hirows ? 1 : 0); }
+int kernel_slot(int nstage, bool hirows) { return 1 + 2 * nstage + (hirows ? 1 : 0); }
 
 struct DeviceInfo {
   int sms = 0;
@@ -569,7 +395,6 @@ cudaError_t occupancy(KernelFn fn, int slot, int smem, int *per_sm) {
 constexpr int kMaxSplits = 128;
 constexpr int kMinChunksPerCta = 2 * kDecodeWarps;
 constexpr int kMaxCtasPerSm = 4;  // the split bound assumes at most this many resident CTAs
-constexpr int kWarpSmemTarget = 12 * 1024;  // lets 4 CTAs of 4 warps share an SM at the common keep counts
 
 }  // namespace
 
@@ -594,28 +419,19 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int splits) {
   return cnt + ml + o;
 }
 
-cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
-                        DecodePlan *plan) {
+cudaError_t plan_dense(int B, int Hkv, int G, int max_len, int forced_splits, DecodePlan *plan) {
   DeviceInfo info;
   cudaError_t e = device_info(&info);
   if (e != cudaSuccess) return e;
-  int nstage, stage_bytes, warp_bytes;
-  if (sparse) {
-    stage_bytes = 512 + 32 * (keep_k + keep_v);
-    nstage = (kWarpSmemTarget - 512) / stage_bytes;
-    nstage = nstage < 2 ? 2 : (nstage > 4 ? 4 : nstage);
-    warp_bytes = nstage * stage_bytes + 512;  // + the per-row half-word prefix table
-  } else {
-    stage_bytes = 2 * kTileBytes;
-    nstage = 3;
-    warp_bytes = nstage * stage_bytes;
-  }
+  const int stage_bytes = 2 * kTileBytes;
+  const int nstage = 3;
+  const int warp_bytes = nstage * stage_bytes;
   const int merge_bytes = kDecodeWarps * 16 * 2 * 4 + kDecodeWarps * G * kHeadDim * 4;
   int smem = kDecodeWarps * warp_bytes;
   smem = smem < merge_bytes ? merge_bytes : smem;
   const bool hirows = G > 8;
-  KernelFn fn = pick_kernel(sparse, nstage, hirows);
-  e = ensure_smem_limit(reinterpret_cast<const void *>(fn), kernel_slot(sparse, nstage, hirows), smem);
+  KernelFn fn = pick_kernel(nstage, hirows);
+  e = ensure_smem_limit(reinterpret_cast<const void *>(fn), kernel_slot(nstage, hirows), smem);
   if (e != cudaSuccess) return e;
 
   const int nch = (max_len + kChunk - 1) / kChunk;
@@ -624,7 +440,7 @@ cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int kee
     splits = forced_splits;
   } else {
     int per_sm = 0;
-    e = occupancy(fn, kernel_slot(sparse, nstage, hirows), smem, &per_sm);
+    e = occupancy(fn, kernel_slot(nstage, hirows), smem, &per_sm);
     if (e != cudaSuccess) return e;
     per_sm = per_sm < 1 ? 1 : (per_sm > kMaxCtasPerSm ? kMaxCtasPerSm : per_sm);
     const int streams = B * Hkv;
@@ -647,8 +463,8 @@ cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int kee
   return cudaSuccess;
 }
 
-cudaError_t launch_decode(bool sparse, const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
-  KernelFn fn = pick_kernel(sparse, plan.nstage, p.G > 8);
+cudaError_t launch_dense(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
+  KernelFn fn = pick_kernel(plan.nstage, p.G > 8);
   dim3 grid(plan.splits, p.Hkv, p.B);
   fn<<<grid, kDecodeThreads, plan.smem_bytes, stream>>>(p);
   return cudaGetLastError();

@@ -62,12 +62,11 @@ struct DecodePlan {
   int smem_bytes;
 };
 
-// Plan (split count, pipeline depth, shared memory) for one decode call.
-cudaError_t plan_decode(bool sparse, int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
-                        DecodePlan *plan);
+// Dense fp16 baseline: plan (split count, pipeline depth, shared memory) and launch.
+cudaError_t plan_dense(int B, int Hkv, int G, int max_len, int forced_splits, DecodePlan *plan);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int splits);
 int decode_split_bound(int B, int Hkv, int max_len);
-cudaError_t launch_decode(bool sparse, const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
+cudaError_t launch_dense(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
 
 // Sparse decode over the compressed caches (one wave of CTAs over the end-to-end chunk sequence):
 // plan->splits holds the CTA count.

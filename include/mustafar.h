@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define MUSTAFAR_ABI_VERSION 1
+#define MUSTAFAR_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MUSTAFAR_API __attribute__((visibility("default")))
@@ -80,10 +80,17 @@ typedef struct {
   int32_t num_kv_heads;
   int32_t head_dim;
   int32_t capacity;
-  int32_t keep; /* = mustafar_keep_count(head_dim, sparsity) */
+  int32_t keep; /* = mustafar_keep_count(head_dim, sparsity); with head_keep: the largest of them */
   uint32_t *bitmap;
   uint16_t *values;
   uint32_t *tile_offset;
+  /* HOST array [num_kv_heads] (at most 128 heads), or NULL.  Per-head sparsity (the allocation
+   * the MUSTAFAR summary, "Limitations", leaves open): kv head h keeps head_keep[h] channels per
+   * token, each in [1, head_dim].  Stream (b, h)'s packed values then start at element
+   * capacity * (b * sum_h' head_keep[h'] + sum_{h'<h} head_keep[h']), token t's run at + t*head_keep[h],
+   * and its tile offsets are 64*i*head_keep[h].  NULL: every head keeps `keep` (the same layout
+   * with all head_keep[h] = keep).  Read at call time only; the library keeps no pointer to it. */
+  const int32_t *head_keep;
 } mustafar_cache_t;
 
 /* Keep count for a pruning sparsity s (fraction of channels removed, README
@@ -96,13 +103,22 @@ MUSTAFAR_API mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_
                                      int32_t capacity, float sparsity, size_t *bitmap_bytes,
                                      size_t *values_bytes, size_t *offset_bytes);
 
+/* As mustafar_cache_sizes for a cache with a keep count per kv head (host array
+ * head_keep[num_kv_heads], each in [1, head_dim]): values take 2 * batch * capacity *
+ * sum_h head_keep[h] bytes.  Errors: INVALID_ARG. */
+MUSTAFAR_API mustafar_status mustafar_cache_sizes_per_head(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                                                           int32_t capacity, const int32_t *head_keep,
+                                                           size_t *bitmap_bytes, size_t *values_bytes,
+                                                           size_t *offset_bytes);
+
 /* Prune + compress (prefill).  Per-token magnitude pruning followed by the
  * bitmap compression (MUSTAFAR summary, "Approach"; Mustafar abstract).
  *   x        : fp16 dense cache; element (b, h, t, c) at
  *              x[b*stride_b + h*stride_h + t*stride_t + c] (strides in elements,
  *              channels contiguous; x and every stride a multiple of 8 elements).
  *   L        : tokens [0, L) are compressed into slots [0, L); 0 <= L <= capacity.
- *   sparsity : must satisfy c->keep == mustafar_keep_count(c->head_dim, sparsity).
+ *   sparsity : must satisfy c->keep == mustafar_keep_count(c->head_dim, sparsity); ignored
+ *              when c->head_keep is set (each head then keeps c->head_keep[h]).
  *   c        : the destination cache; its whole tile_offset array is written.
  *   d_err    : optional device word (unused by this call today; may be NULL).
  * Slots >= L are not touched.  Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */

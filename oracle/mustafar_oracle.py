@@ -194,6 +194,71 @@ def append(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
 
 
 # --------------------------------------------------------------------------------------
+# a keep count per kv head
+# --------------------------------------------------------------------------------------
+# The pages prune every head to the same sparsity and name per-head allocation as the open
+# next step (MUSTAFAR summary, atlas.scime.ai, "Limitations").  With a keep count head_keep[h]
+# per kv head, each (token, head h) vector is pruned exactly as above with k = head_keep[h]; the
+# library's layout puts the streams batch-major, head h's packed values right after those of the
+# heads before it.
+def value_base_heads(b: int, h: int, head_keep, capacity: int) -> int:
+    """First element of stream (b, h)'s packed values: capacity * (b * sum(k) + sum(k[:h]))."""
+    return capacity * (b * int(sum(head_keep)) + int(sum(head_keep[:h])))
+
+
+def prune_heads(x_bits: np.ndarray, head_keep) -> np.ndarray:
+    """Pruned fp16 bits of a dense cache [B, H, T, d]: head h keeps head_keep[h] channels per token."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    return np.concatenate([prune(x[:, h:h + 1], int(k)) for h, k in enumerate(head_keep)], axis=1)
+
+
+def compress_heads(x_bits: np.ndarray, head_keep, capacity: int, L: int | None = None) -> dict:
+    """``compress`` with a keep count per kv head: bitmap [B, H, capacity, d/32] and tile_offset
+    [B, H, capacity/64] as before (offsets 64*i*head_keep[h]); ``values`` is one flat uint16 array of
+    B * capacity * sum(head_keep) elements, stream (b, h) at ``value_base_heads(b, h, ...)``."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    B, H, T, d = x.shape
+    L = T if L is None else L
+    parts = [compress(x[:, h:h + 1], int(k), capacity, L) for h, k in enumerate(head_keep)]
+    values = np.zeros(B * capacity * int(sum(head_keep)), dtype=np.uint16)
+    for h, k in enumerate(head_keep):
+        for b in range(B):
+            base = value_base_heads(b, h, head_keep, capacity)
+            values[base:base + capacity * int(k)] = parts[h]["values"][b, 0]
+    return {"bitmap": np.concatenate([c["bitmap"] for c in parts], axis=1), "values": values,
+            "tile_offset": np.concatenate([c["tile_offset"] for c in parts], axis=1),
+            "head_keep": [int(k) for k in head_keep], "L": L}
+
+
+def decompress_heads(cache: dict, L: int, d: int) -> np.ndarray:
+    """Dense fp16 bits [B, H, L, d] rebuilt from a per-head compressed cache."""
+    hk = cache["head_keep"]
+    B, H, cap = cache["bitmap"].shape[:3]
+    out = []
+    for h, k in enumerate(hk):
+        vals = np.stack([cache["values"][value_base_heads(b, h, hk, cap):value_base_heads(b, h, hk, cap) + cap * k]
+                         for b in range(B)])[:, None]
+        out.append(decompress(cache["bitmap"][:, h:h + 1], vals, k, L, d))
+    return np.concatenate(out, axis=1)
+
+
+def append_heads(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
+    """``append`` for a per-head cache: the new token of (b, h) keeps head_keep[h] channels."""
+    hk = cache["head_keep"]
+    x = np.asarray(x_new_bits, dtype=np.uint16)  # [B, H, d]
+    B, H, d = x.shape
+    cap = cache["bitmap"].shape[2]
+    for h, k in enumerate(hk):
+        mask = select_sort(x[:, h], k)
+        words = bitmap_words(mask)
+        for b in range(B):
+            p = int(pos[b])
+            cache["bitmap"][b, h, p] = words[b]
+            base = value_base_heads(b, h, hk, cap) + p * k
+            cache["values"][base:base + k] = x[b, h][mask[b]]
+
+
+# --------------------------------------------------------------------------------------
 # attention over the pruned caches
 # --------------------------------------------------------------------------------------
 def f16_to_f64(bits: np.ndarray) -> np.ndarray:

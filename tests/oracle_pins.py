@@ -12,6 +12,9 @@ oracle disagrees with the fact it checks.  Facts used:
 * attention at sparsity 0 against torch's float64 ``scaled_dot_product_attention``;
 * L = 1 gives o = V~_0 exactly; softmax weights sum to 1; token-permutation
   invariance; a GQA group with equal queries gives equal outputs.
+* per-head keep counts: with one keep for every head the per-head layout equals the uniform
+  one byte for byte; the streams tile the value array exactly; brute-force ranks and popcounts
+  per head; round trip to the per-head pruned cache; append == compress.
 """
 from __future__ import annotations
 
@@ -258,9 +261,52 @@ def pin_append_equals_compress(O):
         assert np.array_equal(full[key], part[key]), key
 
 
+# ----------------------------------------------------------------------------- keep count per head
+def pin_heads_layout(O):
+    rng = np.random.default_rng(19)
+    B, H, L, d, cap = 2, 4, 100, 128, 128
+    x = rand_bits(rng, (B, H, L, d))
+    x[1, 2, 7] = rand_bits(rng, (d,), tie_heavy=True)
+    # one keep count for every head: the per-head layout is the uniform layout, byte for byte
+    for k in (39, 64):
+        u, p = O.compress(x, k, cap), O.compress_heads(x, [k] * H, cap)
+        assert np.array_equal(p["values"], u["values"].reshape(-1))
+        assert np.array_equal(p["bitmap"], u["bitmap"]) and np.array_equal(p["tile_offset"], u["tile_offset"])
+    hk = [13, 128, 1, 64]
+    c = O.compress_heads(x, hk, cap)
+    # the streams' value ranges tile the array exactly, batch-major then head order
+    spans = [(O.value_base_heads(b, h, hk, cap), O.value_base_heads(b, h, hk, cap) + cap * hk[h])
+             for b in range(B) for h in range(H)]
+    assert spans[0][0] == 0 and spans[-1][1] == c["values"].size == B * cap * sum(hk)
+    assert all(a[1] == nxt[0] for a, nxt in zip(spans, spans[1:]))
+    # every token of head h keeps exactly hk[h] channels, chosen by the brute-force rank rule
+    pop = np.vectorize(lambda w: bin(int(w)).count("1"))(c["bitmap"][:, :, :L]).sum(-1)
+    for h, k in enumerate(hk):
+        assert (pop[:, h] == k).all()
+        mask = O.bitmap_to_mask(c["bitmap"][:, h:h + 1, :4], d)
+        assert np.array_equal(mask, O.select_rank_bruteforce(x[:, h:h + 1, :4], k))
+        assert all(int(c["tile_offset"][b, h, i]) == 64 * i * k for b in range(B) for i in range(cap // 64))
+    # round trip: the packed values put back by the bitmap give the per-head pruned cache
+    dec = O.decompress_heads(c, L, d)
+    assert np.array_equal(dec, O.prune_heads(x, hk))
+    assert all(np.array_equal(dec[:, h:h + 1], O.prune(x[:, h:h + 1], k)) for h, k in enumerate(hk))
+
+
+def pin_heads_append_equals_compress(O):
+    rng = np.random.default_rng(23)
+    B, H, L, d, cap, hk = 2, 3, 62, 128, 128, [90, 13, 39]
+    x = rand_bits(rng, (B, H, L + 3, d))
+    full = O.compress_heads(x, hk, cap, L + 3)
+    part = O.compress_heads(x, hk, cap, L)
+    for s in range(3):
+        O.append_heads(part, x[:, :, L + s], np.full(B, L + s))
+    for key in ("bitmap", "values", "tile_offset"):
+        assert np.array_equal(full[key], part[key]), key
+
+
 ALL_PINS = [pin_golden_selection, pin_golden_keep_count, pin_bruteforce_selection, pin_threshold_invariant,
             pin_roundtrip_and_popcount, pin_compressed_size, pin_dense_limit_sdpa, pin_golden_attention,
-            pin_attention_invariants, pin_append_equals_compress]
+            pin_attention_invariants, pin_append_equals_compress, pin_heads_layout, pin_heads_append_equals_compress]
 
 
 def failing_pins(O):

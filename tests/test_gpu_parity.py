@@ -272,6 +272,102 @@ def test_decode_step_out_of_range_positions():
     U.assert_attn_close(out, o_ref, lse, l_ref, tag="row longer than max_len")
 
 
+# ------------------------------------------------------------------------------------ keep count per kv head
+def _heads_cache_matches(cache, x_bits, L, streams=None):
+    """Bit-exact check of a per-head cache against the oracle, tokens [0, L) of every (b, h)."""
+    B, H, cap = cache.batch, cache.num_kv_heads, cache.capacity
+    hk = cache.head_keep
+    ref = oracle.compress_heads(x_bits[:, :, :L], hk, cap, L)
+    bm = cache.bitmap.view(B, H, cap, 4).cpu().numpy().view(np.uint32)
+    offs = cache.tile_offset.view(B, H, cap // 64).cpu().numpy().view(np.uint32)
+    vals = cache.values.cpu().numpy().view(np.uint16)
+    assert np.array_equal(bm[:, :, :L], ref["bitmap"][:, :, :L]), "bitmap"
+    assert np.array_equal(offs, ref["tile_offset"]), "tile offsets"
+    for b in range(B):
+        for h in range(H):
+            base = oracle.value_base_heads(b, h, hk, cap)
+            assert cache.value_base(b, h) == base
+            assert np.array_equal(vals[base:base + L * hk[h]], ref["values"][base:base + L * hk[h]]), (b, h)
+
+
+def test_per_head_compress_and_append_bit_exact():
+    B, H, L0, L1, cap = 2, 4, 150, 160, 192
+    hs = [0.0, 0.3, 0.7, 0.9]
+    x = synth.keys(B, H, L1, D, 61, DEV, capacity=cap)
+    c = M.CompressedCache(B, H, cap, hs)
+    assert c.head_keep == [128, 90, 39, 13] and c.keep == 128
+    M.mustafar_compress(x, L0, 0.0, c)  # the sparsity argument is not used by a per-head cache
+    for t in range(L0, L1):
+        M.mustafar_append(x[:, :, t], torch.full((B,), t, dtype=torch.int32, device=DEV), c)
+    _heads_cache_matches(c, U.bits(x), L1)
+
+
+@pytest.mark.parametrize("splits", [0, 3])
+def test_per_head_decode_attn_and_step(splits):
+    B, Hq, Hkv, L, cap = 3, 16, 4, 200, 256
+    sK, sV = [0.5, 0.7, 0.9, 0.3], [0.7, 0.5, 0.7, 0.0]
+    K = synth.keys(B, Hkv, cap, D, 62, DEV)
+    V = synth.values(B, Hkv, cap, D, 62, DEV)
+    kc, vc = M.CompressedCache(B, Hkv, cap, sK), M.CompressedCache(B, Hkv, cap, sV)
+    M.mustafar_compress(K, L, 0.0, kc)
+    M.mustafar_compress(V, L, 0.0, vc)
+    q = synth.queries(B, Hq, D, 62, DEV)
+    seq = synth.seq_lens(B, L, True, 62)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), L, 1.0, num_splits=splits)
+    Kb, Vb = U.bits(K), U.bits(V)
+    kp, vp = oracle.prune_heads(Kb[:, :, :L], kc.head_keep), oracle.prune_heads(Vb[:, :, :L], vc.head_keep)
+    o_ref, l_ref = oracle.attention(U.bits(q), kp, vp, seq.numpy(), 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"per-head decode, splits {splits}")
+    # fused steps with fresh tokens, each row at its own position (overwriting prefill slots of
+    # the shorter rows with different tokens)
+    pos = seq.clone().to(DEV)
+    rows = torch.arange(B, device=DEV)
+    for st in range(2):
+        qs = synth.queries(B, Hq, D, 62, DEV, step=st + 1)
+        kn, vn = synth.step_tokens(B, Hkv, D, 62, st, DEV)
+        K[rows, :, pos.long()] = kn
+        V[rows, :, pos.long()] = vn
+        out, lse = M.mustafar_decode_step(qs, kn, vn, pos, kc, vc, L + 2, 1.0, num_splits=splits)
+        lens = (pos + 1).cpu().numpy()
+        Lm = int(lens.max())
+        Kb, Vb = U.bits(K), U.bits(V)
+        kp = oracle.prune_heads(Kb[:, :, :Lm], kc.head_keep)
+        vp = oracle.prune_heads(Vb[:, :, :Lm], vc.head_keep)
+        o_ref, l_ref = oracle.attention(U.bits(qs), kp, vp, lens, 1.0)
+        U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"per-head step {st}")
+        pos += 1
+    # cache rows now hold tokens [0, seq + 2) of K / V
+    fin = (seq + 2).numpy()
+    for cache, xb in ((kc, Kb), (vc, Vb)):
+        for b in range(B):
+            ref = oracle.compress_heads(xb[b:b + 1, :, :fin[b]], cache.head_keep, cap, int(fin[b]))
+            vals = cache.values.cpu().numpy().view(np.uint16)
+            for h, k in enumerate(cache.head_keep):
+                base = oracle.value_base_heads(b, h, cache.head_keep, cap)
+                rb = oracle.value_base_heads(0, h, cache.head_keep, cap)
+                assert np.array_equal(vals[base:base + fin[b] * k], ref["values"][rb:rb + fin[b] * k]), (b, h)
+
+
+def test_per_head_llama3_gqa_b8_ctx4096_mean_s07():
+    # per-head sparsities spread around 0.7 (their keep counts average the uniform s = 0.7 keep)
+    B, Hq, Hkv, L = 8, 32, 8, 4096
+    sK = [0.5, 0.6, 0.7, 0.8, 0.9, 0.7, 0.6, 0.8]
+    sV = sK[::-1]
+    K = synth.keys(B, Hkv, L, D, 1005, DEV)
+    V = synth.values(B, Hkv, L, D, 1005, DEV)
+    kc, vc = M.CompressedCache(B, Hkv, L, sK), M.CompressedCache(B, Hkv, L, sV)
+    M.mustafar_compress(K, L, 0.0, kc)
+    M.mustafar_compress(V, L, 0.0, vc)
+    q = synth.queries(B, Hq, D, 1005, DEV)
+    seq = torch.full((B,), L, dtype=torch.int32)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), L, 1.0)
+    rows = [0, 3, 7]
+    Kb, Vb = U.bits(K[rows]), U.bits(V[rows])
+    kp, vp = oracle.prune_heads(Kb, kc.head_keep), oracle.prune_heads(Vb, vc.head_keep)
+    o_ref, l_ref = oracle.attention(U.bits(q[rows]), kp, vp, [L] * len(rows), 1.0)
+    U.assert_attn_close(out[rows], o_ref, lse[rows], l_ref, tag="per-head b8 ctx4096")
+
+
 # ------------------------------------------------------------------------------------ the workload shapes
 def test_llama3_gqa_b1_ctx1024_s05():
     B, Hq, Hkv, L = 1, 32, 8, 1024

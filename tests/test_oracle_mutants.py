@@ -59,6 +59,48 @@ def _mutant(**overrides):
                 cache["values"][b, h, p * k:(p + 1) * k] = x[b, h][mask[b, h]]
     if "append" not in overrides:
         ns.append = append
+    # per-head functions, rebound so that they call the (possibly mutated) namespace
+    def prune_heads(x_bits, head_keep):
+        x = np.asarray(x_bits, dtype=np.uint16)
+        return np.concatenate([ns.prune(x[:, h:h + 1], int(k)) for h, k in enumerate(head_keep)], axis=1)
+    if "prune_heads" not in overrides:
+        ns.prune_heads = prune_heads
+    def compress_heads(x_bits, head_keep, capacity, L=None):
+        x = np.asarray(x_bits, dtype=np.uint16)
+        B, H, T, d = x.shape
+        parts = [ns.compress(x[:, h:h + 1], int(k), capacity, L) for h, k in enumerate(head_keep)]
+        values = np.zeros(B * capacity * int(sum(head_keep)), dtype=np.uint16)
+        for h, k in enumerate(head_keep):
+            for b in range(B):
+                base = ns.value_base_heads(b, h, head_keep, capacity)
+                values[max(base, 0):max(base, 0) + capacity * int(k)] = parts[h]["values"][b, 0][: max(0, min(
+                    capacity * int(k), values.size - max(base, 0)))]
+        return {"bitmap": np.concatenate([c["bitmap"] for c in parts], axis=1), "values": values,
+                "tile_offset": np.concatenate([c["tile_offset"] for c in parts], axis=1),
+                "head_keep": [int(k) for k in head_keep], "L": parts[0]["L"]}
+    ns.compress_heads = compress_heads
+    def decompress_heads(cache, L, d):
+        hk = cache["head_keep"]
+        B, H, cap = cache["bitmap"].shape[:3]
+        out = []
+        for h, k in enumerate(hk):
+            vals = np.stack([cache["values"][ns.value_base_heads(b, h, hk, cap):][: cap * k] for b in range(B)])
+            out.append(ns.decompress(cache["bitmap"][:, h:h + 1], vals[:, None], k, L, d))
+        return np.concatenate(out, axis=1)
+    ns.decompress_heads = decompress_heads
+    def append_heads(cache, x_new_bits, pos):
+        hk = cache["head_keep"]
+        x = np.asarray(x_new_bits, dtype=np.uint16)
+        cap = cache["bitmap"].shape[2]
+        for h, k in enumerate(hk):
+            mask = ns.select_sort(x[:, h], k)
+            words = ns.bitmap_words(mask)
+            for b in range(x.shape[0]):
+                p = int(pos[b])
+                cache["bitmap"][b, h, p] = words[b]
+                base = ns.value_base_heads(b, h, hk, cap) + p * k
+                cache["values"][base:base + k] = x[b, h][mask[b]]
+    ns.append_heads = append_heads
     return ns
 
 
@@ -128,7 +170,23 @@ def prune_negzero(x_bits, k):           # pruned slots written as -0 instead of 
     return np.where(real.select_sort(x, k), x, np.uint16(0x8000)).astype(np.uint16)
 
 
+def base_next_head(b, h, head_keep, capacity):      # stream starts after its own head's values
+    return capacity * (b * int(sum(head_keep)) + int(sum(head_keep[:h + 1])))
+
+
+def base_head_major(b, h, head_keep, capacity):     # head-major instead of batch-major streams
+    return capacity * (int(sum(head_keep[:h])) * 2 + b * int(head_keep[h]))
+
+
+def prune_heads_max(x_bits, head_keep):             # every head pruned with the largest keep
+    x = np.asarray(x_bits, dtype=np.uint16)
+    return np.concatenate([real.prune(x[:, h:h + 1], int(max(head_keep))) for h in range(x.shape[1])], axis=1)
+
+
 MUTANTS = {
+    "per-head base after own head": dict(value_base_heads=base_next_head),
+    "per-head streams head-major": dict(value_base_heads=base_head_major),
+    "per-head prune with max keep": dict(prune_heads=prune_heads_max),
     "select ascending": dict(select_sort=sel_ascending),
     "ties to higher index": dict(select_sort=sel_high_index_ties),
     "signed compare": dict(select_sort=sel_signed),

@@ -26,7 +26,7 @@ ABI_SYMBOLS = (
     "mustafar_keep_count", "mustafar_cache_sizes", "mustafar_compress", "mustafar_append",
     "mustafar_decode_workspace_bytes", "mustafar_decode_attn", "mustafar_dense_decode_attn",
     "mustafar_decode_plan_splits", "mustafar_status_string", "mustafar_last_error", "mustafar_abi_version",
-    "mustafar_decode_attn_noalloc", "mustafar_decode_step",
+    "mustafar_decode_attn_noalloc", "mustafar_decode_step", "mustafar_cache_sizes_per_head",
 )
 
 
@@ -40,7 +40,7 @@ class CacheT(C.Structure):
     """Mirror of mustafar_cache_t."""
     _fields_ = [("batch", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
                 ("capacity", C.c_int32), ("keep", C.c_int32), ("bitmap", C.c_void_p),
-                ("values", C.c_void_p), ("tile_offset", C.c_void_p)]
+                ("values", C.c_void_p), ("tile_offset", C.c_void_p), ("head_keep", C.c_void_p)]
 
 
 _lib = None
@@ -59,6 +59,7 @@ def load() -> C.CDLL:
     sig = {
         "mustafar_keep_count": (i32, [i32, f32]),
         "mustafar_cache_sizes": (i32, [i32, i32, i32, i32, f32, P(sz), P(sz), P(sz)]),
+        "mustafar_cache_sizes_per_head": (i32, [i32, i32, i32, i32, vp, P(sz), P(sz), P(sz)]),
         "mustafar_compress": (i32, [vp, i64, i64, i64, i32, f32, P(CacheT), vp, vp]),
         "mustafar_append": (i32, [vp, i64, i64, vp, P(CacheT), vp, vp]),
         "mustafar_decode_workspace_bytes": (i32, [i32, i32, i32, i32, i32, i32, P(sz)]),
@@ -131,30 +132,72 @@ def mustafar_decode_plan_splits(batch, num_kv_heads, max_len, keep_k, keep_v, de
 
 
 # ------------------------------------------------------------------------------------------- caches
-class CompressedCache:
-    """Caller-owned device arrays of one compressed cache (K or V) plus its C descriptor."""
+def mustafar_cache_sizes_per_head(batch, num_kv_heads, capacity, head_keep, head_dim=HEAD_DIM):
+    """(bitmap_bytes, values_bytes, offset_bytes) of a cache with keep count head_keep[h] per kv head."""
+    arr = (C.c_int32 * len(head_keep))(*head_keep)
+    nb, nv, no = C.c_size_t(), C.c_size_t(), C.c_size_t()
+    _check(load().mustafar_cache_sizes_per_head(batch, num_kv_heads, head_dim, capacity, C.cast(arr, C.c_void_p),
+                                                C.byref(nb), C.byref(nv), C.byref(no)))
+    return nb.value, nv.value, no.value
 
-    def __init__(self, batch: int, num_kv_heads: int, capacity: int, sparsity: float, head_dim: int = HEAD_DIM,
+
+class CompressedCache:
+    """Caller-owned device arrays of one compressed cache (K or V) plus its C descriptor.
+
+    ``sparsity`` is one value for every kv head, or a sequence with one sparsity per kv head
+    (then head h keeps ``mustafar_keep_count(head_dim, sparsity[h])`` channels per token)."""
+
+    def __init__(self, batch: int, num_kv_heads: int, capacity: int, sparsity, head_dim: int = HEAD_DIM,
                  device="cuda"):
         self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
-        self.sparsity = float(sparsity)
-        self.keep = mustafar_keep_count(head_dim, sparsity)
-        nb, nv, no = mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity)
+        self._head_keep_arr = None
+        if isinstance(sparsity, (list, tuple)):
+            if len(sparsity) != num_kv_heads:
+                raise ValueError("one sparsity per kv head expected")
+            self.head_sparsity = [float(x) for x in sparsity]
+            self.head_keep = [mustafar_keep_count(head_dim, x) for x in self.head_sparsity]
+            self.sparsity = None
+            self.keep = max(self.head_keep)
+            nb, nv, no = mustafar_cache_sizes_per_head(batch, num_kv_heads, capacity, self.head_keep, head_dim)
+            self._head_keep_arr = (C.c_int32 * num_kv_heads)(*self.head_keep)
+        else:
+            self.sparsity = float(sparsity)
+            self.keep = mustafar_keep_count(head_dim, sparsity)
+            self.head_keep = [self.keep] * num_kv_heads
+            self.head_sparsity = None
+            nb, nv, no = mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity)
         self.bitmap = torch.zeros(nb // 4, dtype=torch.int32, device=device)
         self.values = torch.zeros(nv // 2, dtype=torch.int16, device=device)
         self.tile_offset = torch.zeros(no // 4, dtype=torch.int32, device=device)
+        hk = C.cast(self._head_keep_arr, C.c_void_p).value if self._head_keep_arr is not None else None
         self._struct = CacheT(batch, num_kv_heads, head_dim, capacity, self.keep, self.bitmap.data_ptr(),
-                              self.values.data_ptr(), self.tile_offset.data_ptr())
+                              self.values.data_ptr(), self.tile_offset.data_ptr(), hk)
 
     @property
     def struct(self) -> CacheT:
         return self._struct
 
+    @property
+    def per_head(self) -> bool:
+        return self._head_keep_arr is not None
+
     def nbytes(self) -> int:
         return self.bitmap.numel() * 4 + self.values.numel() * 2 + self.tile_offset.numel() * 4
 
+    def value_base(self, b: int, h: int) -> int:
+        """Element index where stream (b, h)'s packed values start."""
+        return self.capacity * (b * sum(self.head_keep) + sum(self.head_keep[:h]))
+
+    def stream_values(self, b: int, h: int) -> torch.Tensor:
+        """The capacity * head_keep[h] packed values of stream (b, h) (int16 view)."""
+        base = self.value_base(b, h)
+        return self.values[base:base + self.capacity * self.head_keep[h]]
+
     def views(self):
-        """(bitmap [B,H,cap,d/32] int32, values [B,H,cap*k] int16, tile_offset [B,H,cap/64] int32)."""
+        """(bitmap [B,H,cap,d/32] int32, values [B,H,cap*k] int16, tile_offset [B,H,cap/64] int32);
+        uniform caches only (per-head caches: ``stream_values``)."""
+        if self.per_head:
+            raise ValueError("values of a per-head cache have no [B, H, cap*k] view; use stream_values")
         B, H, cap, d = self.batch, self.num_kv_heads, self.capacity, self.head_dim
         return (self.bitmap.view(B, H, cap, d // 32), self.values.view(B, H, cap * self.keep),
                 self.tile_offset.view(B, H, cap // 64))

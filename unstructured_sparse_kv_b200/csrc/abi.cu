@@ -50,6 +50,20 @@ mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: capacity must be a multiple of 64 (got %d)", name, c->capacity);
   if (c->keep < 1 || c->keep > c->head_dim)
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: keep must lie in [1, head_dim] (got %d)", name, c->keep);
+  if (c->head_keep != nullptr) {
+    if (c->num_kv_heads > kMaxKvHeads)
+      return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: per-head keep supports at most %d kv heads", name, kMaxKvHeads);
+    int32_t kmax = 0;
+    for (int h = 0; h < c->num_kv_heads; ++h) {
+      if (c->head_keep[h] < 1 || c->head_keep[h] > c->head_dim)
+        return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: head_keep[%d] = %d outside [1, head_dim]", name, h, c->head_keep[h]);
+      kmax = c->head_keep[h] > kmax ? c->head_keep[h] : kmax;
+    }
+    if (kmax != c->keep)
+      return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: keep must be the largest head_keep (%d), got %d", name, kmax, c->keep);
+  } else if (c->num_kv_heads > kMaxKvHeads) {
+    return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: at most %d kv heads", name, kMaxKvHeads);
+  }
   if (static_cast<int64_t>(c->capacity) * c->keep >= (int64_t(1) << 32))
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: capacity*keep must stay below 2^32 (32-bit tile offsets)", name);
   if (c->bitmap == nullptr || c->values == nullptr || c->tile_offset == nullptr)
@@ -98,6 +112,21 @@ const char *mustafar_status_string(mustafar_status s) {
 
 const char *mustafar_last_error(void) { return g_last_error.c_str(); }
 
+// Keep counts and value placement of every head of a checked cache.
+static HeadKeep head_keep_of(const mustafar_cache_t *c) {
+  HeadKeep hk;
+  hk.pre[0] = 0;
+  for (int h = 0; h < c->num_kv_heads; ++h) {
+    hk.k[h] = c->head_keep != nullptr ? c->head_keep[h] : c->keep;
+    hk.pre[h + 1] = hk.pre[h] + hk.k[h];
+  }
+  for (int h = c->num_kv_heads; h < kMaxKvHeads; ++h) {
+    hk.k[h] = 0;
+    hk.pre[h + 1] = hk.pre[h];
+  }
+  return hk;
+}
+
 int32_t mustafar_keep_count(int32_t head_dim, float sparsity) { return keep_count(head_dim, sparsity); }
 
 mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity,
@@ -114,17 +143,41 @@ mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_heads, int32_
   return MUSTAFAR_OK;
 }
 
+mustafar_status mustafar_cache_sizes_per_head(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                                              int32_t capacity, const int32_t *head_keep, size_t *bitmap_bytes,
+                                              size_t *values_bytes, size_t *offset_bytes) {
+  if (head_keep == nullptr) return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes_per_head: head_keep is NULL");
+  if (head_dim <= 0 || head_dim % 32 != 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes_per_head: head_dim must be a positive multiple of 32");
+  if (batch <= 0 || num_kv_heads <= 0 || capacity <= 0 || capacity % kTileTokens != 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes_per_head: positive shapes and capacity %% 64 == 0 required");
+  size_t ksum = 0;
+  for (int h = 0; h < num_kv_heads; ++h) {
+    if (head_keep[h] < 1 || head_keep[h] > head_dim)
+      return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes_per_head: head_keep[%d] = %d outside [1, head_dim]", h,
+                  head_keep[h]);
+    ksum += static_cast<size_t>(head_keep[h]);
+  }
+  const size_t streams = static_cast<size_t>(batch) * num_kv_heads;
+  if (bitmap_bytes) *bitmap_bytes = streams * capacity * (head_dim / 8);
+  if (values_bytes) *values_bytes = static_cast<size_t>(batch) * capacity * ksum * 2;
+  if (offset_bytes) *offset_bytes = streams * (capacity / kTileTokens) * 4;
+  return MUSTAFAR_OK;
+}
+
 mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t stride_h, int64_t stride_t, int32_t L,
                                   float sparsity, const mustafar_cache_t *c, uint32_t *d_err,
                                   mustafar_stream_t stream) {
   (void)d_err;
   mustafar_status s = check_cache(c, "compress");
   if (s != MUSTAFAR_OK) return s;
-  const int32_t k = keep_count(c->head_dim, sparsity);
-  if (k < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: sparsity must lie in [0, 1)");
-  if (k != c->keep)
-    return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: cache keep %d != keep_count(%d, %g) = %d", c->keep,
-                c->head_dim, static_cast<double>(sparsity), k);
+  if (c->head_keep == nullptr) {
+    const int32_t k = keep_count(c->head_dim, sparsity);
+    if (k < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: sparsity must lie in [0, 1)");
+    if (k != c->keep)
+      return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: cache keep %d != keep_count(%d, %g) = %d", c->keep,
+                  c->head_dim, static_cast<double>(sparsity), k);
+  }
   if (L < 0 || L > c->capacity) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: L must lie in [0, capacity]");
   if (x == nullptr && L > 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: x is NULL");
   if (L > 0) {
@@ -134,8 +187,8 @@ mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t strid
       return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: negative strides are not supported");
   }
   cudaError_t e = launch_compress(static_cast<const uint16_t *>(x), stride_b, stride_h, stride_t, L, c->batch,
-                                  c->num_kv_heads, c->keep, c->capacity, c->bitmap, c->values, c->tile_offset,
-                                  reinterpret_cast<cudaStream_t>(stream));
+                                  c->num_kv_heads, head_keep_of(c), c->keep, c->capacity, c->bitmap, c->values,
+                                  c->tile_offset, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "compress launch");
 }
 
@@ -149,7 +202,7 @@ mustafar_status mustafar_append(const void *x, int64_t stride_b, int64_t stride_
   if (stride_b < 0 || stride_h < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "append: negative strides");
   if (!aligned(d_pos, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "append: pos must be 4-byte aligned");
   cudaError_t e = launch_append(static_cast<const uint16_t *>(x), stride_b, stride_h, d_pos, c->batch,
-                                c->num_kv_heads, c->keep, c->capacity, c->bitmap, c->values, d_err,
+                                c->num_kv_heads, head_keep_of(c), c->capacity, c->bitmap, c->values, d_err,
                                 reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "append launch");
 }
@@ -182,7 +235,7 @@ int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t
     return plan.splits;
   }
   // the sparse kernel cuts the end-to-end chunk sequence into CTA ranges; report the CTAs per stream
-  if (plan_sparse(batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, &plan) != cudaSuccess) return -1;
+  if (plan_sparse(batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, false, &plan) != cudaSuccess) return -1;
   const int streams = batch * num_kv_heads;
   return (plan.splits + streams - 1) / streams;
 }
@@ -192,7 +245,7 @@ namespace {
 mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *workspace, size_t workspace_bytes,
                            const char *name, cudaStream_t stream) {
   DecodePlan plan;
-  cudaError_t e = plan_sparse(p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, &plan);
+  cudaError_t e = plan_sparse(p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, p.perhead != 0, &plan);
   if (e != cudaSuccess) return cuda_fail(e, name);
   p.stage_bytes = plan.stage_bytes;
   p.warp_bytes = plan.warp_bytes;
@@ -276,6 +329,9 @@ mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_heads, const m
   p.vval = v->values;
   p.keep_k = k->keep;
   p.keep_v = v->keep;
+  p.hk_k = head_keep_of(k);
+  p.hk_v = head_keep_of(v);
+  p.perhead = k->head_keep != nullptr || v->head_keep != nullptr;
   p.cap_k = k->capacity;
   p.cap_v = v->capacity;
   p.seq_len = d_seq_len;
@@ -322,6 +378,9 @@ mustafar_status mustafar_decode_step(const void *q, int32_t num_q_heads, const v
   p.vval = v->values;
   p.keep_k = k->keep;
   p.keep_v = v->keep;
+  p.hk_k = head_keep_of(k);
+  p.hk_v = head_keep_of(v);
+  p.perhead = k->head_keep != nullptr || v->head_keep != nullptr;
   p.cap_k = k->capacity;
   p.cap_v = v->capacity;
   p.B = k->batch;

@@ -22,7 +22,7 @@ constexpr int kRowBytesDense = kHeadDim * 2;  // 256
 __device__ __forceinline__ int stage_off(int tok, int j) { return tok * kRowBytesDense + ((j ^ (tok & 15)) << 4); }
 
 __global__ void __launch_bounds__(kCompressThreads)
-compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, int k,
+compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, const HeadKeep hk,
                 int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
                 uint32_t *__restrict__ tile_offset) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -32,6 +32,7 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
   const int tid = threadIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t stream = static_cast<int64_t>(b) * H + h;
+  const int k = hk.k[h];
 
   // tile offsets of the whole stream: the closed form 64*i*k (= popcount prefix sums, every
   // token keeps exactly k channels)
@@ -80,9 +81,9 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
   }
   __syncthreads();
 
-  // coalesced write-out of the CTA's packed run; its start (stream*cap + t0)*k*2 bytes is
-  // 16-byte aligned because cap % 64 == 0 and t0 % 128 == 0
-  uint16_t *vdst = values + (stream * cap + t0) * static_cast<int64_t>(k);
+  // coalesced write-out of the CTA's packed run; its start (value base + t0*k)*2 bytes is
+  // 16-byte aligned because the value base is a multiple of cap, cap % 64 == 0 and t0 % 128 == 0
+  uint16_t *vdst = values + hk.value_base(b, h, H, cap) + static_cast<int64_t>(t0) * k;
   const int n = ntok * k;
   const int nvec = n >> 3;
   for (int i = tid; i < nvec; i += kCompressThreads)
@@ -96,7 +97,7 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
 // largest key T, then the keys equal to T are taken lowest channel first.
 __global__ void __launch_bounds__(128)
 append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int32_t *__restrict__ pos, int B,
-              int H, int k, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
+              int H, const HeadKeep hk, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
               uint32_t *__restrict__ err) {
   const int lane = threadIdx.x & 31;
   const int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -109,29 +110,31 @@ append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int3
   }
   const uint16_t *src = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
   const int64_t stream = static_cast<int64_t>(b) * H + h;
-  warp_compress_vector(src, k, bitmap + (stream * cap + p) * kWords, values + (stream * cap + p) * static_cast<int64_t>(k),
-                       lane);
+  const int k = hk.k[h];
+  warp_compress_vector(src, k, bitmap + (stream * cap + p) * kWords,
+                       values + hk.value_base(b, h, H, cap) + static_cast<int64_t>(p) * k, lane);
 }
 
-cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H, int k,
-                            int cap, uint32_t *bitmap, uint16_t *values, uint32_t *tile_offset,
-                            cudaStream_t stream) {
-  const size_t smem = kCompressThreads * kRowBytesDense + static_cast<size_t>(kCompressThreads) * k * 2;
+cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
+                            const HeadKeep &hk, int kmax, int cap, uint32_t *bitmap, uint16_t *values,
+                            uint32_t *tile_offset, cudaStream_t stream) {
+  const size_t smem = kCompressThreads * kRowBytesDense + static_cast<size_t>(kCompressThreads) * kmax * 2;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(compress_kernel), 0,
                                     kCompressThreads * kRowBytesDense + kCompressThreads * kHeadDim * 2);
   if (e != cudaSuccess) return e;
   const int nbx = L > 0 ? (L + kCompressThreads - 1) / kCompressThreads : 1;
   dim3 grid(nbx, H, B);
-  compress_kernel<<<grid, kCompressThreads, smem, stream>>>(x, sb, sh, st, L, H, k, cap, bitmap, values,
+  compress_kernel<<<grid, kCompressThreads, smem, stream>>>(x, sb, sh, st, L, H, hk, cap, bitmap, values,
                                                             tile_offset);
   return cudaGetLastError();
 }
 
-cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H, int k,
-                          int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err, cudaStream_t stream) {
+cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H,
+                          const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
+                          cudaStream_t stream) {
   const int warps = B * H;
   const int threads = 128;  // 4 vectors per CTA
-  append_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, k, cap,
+  append_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, hk, cap,
                                                                               bitmap, values, err);
   return cudaGetLastError();
 }

@@ -174,10 +174,13 @@ __device__ __forceinline__ void load_q(const DecodeParams &P, int b, int g, int 
 // One 16-token chunk staged at `stage` ([K bitmap rows 16x16 B][V bitmap rows][K values 16*kK]
 // [V values 16*kV]); tokens t0 .. t0+15 of a row of length L.  `htab` is the warp's 512-byte
 // per-row half-word prefix table.
-template <bool HIROWS>
+template <bool HIROWS, bool PERHEAD>
 __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *stage, uint8_t *htab, uint32_t za,
-                                              int t0, int L, int lane, const uint32_t (&qa)[8][4],
+                                              int t0, int L, int kKh, int kVh, int lane, const uint32_t (&qa)[8][4],
                                               Acc<HIROWS> &acc) {
+  // keep counts of this stream; a uniform cache reads them from the kernel parameters here, so that
+  // they hold no register across the chunk loop
+  const int kK = PERHEAD ? kKh : P.keep_k, kV = PERHEAD ? kVh : P.keep_v;
   const int gq = lane >> 2, qq = lane & 3;
   const bool full = t0 + kChunk <= L;
   // lane r (K rows 0-15, V rows 16-31) zeroes the bitmap of a token >= L in place and stores the
@@ -207,7 +210,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
     const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
     const uint32_t word = *reinterpret_cast<const uint32_t *>(stage + T * 16 + qq * 4);
     const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
-    const uint32_t rbase = kvals + 2 * T * P.keep_k;
+    const uint32_t rbase = kvals + 2 * T * kK;
     uint32_t kb[16];
     expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
 #pragma unroll
@@ -281,7 +284,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
 
   // ---- O^T += V~^T P^T : 8 m-tiles of 16 channels.  This lane's A fragments cover channels
   // 16g..16g+15 (half word g of the bitmap) of tokens 2q, 2q+1 and 2q+8, 2q+9.
-  const uint32_t vvals = smem_addr(stage + 512 + 32 * P.keep_k);
+  const uint32_t vvals = smem_addr(stage + 512 + 32 * kK);
   uint32_t va[8][4];
 #pragma unroll
   for (int pair = 0; pair < 2; ++pair) {
@@ -291,7 +294,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
       const int T = 2 * qq + 8 * pair + e;
       const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
       const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
-      expand_half(bits, vvals + 2 * (T * P.keep_v + pre), za, e ? x1 : x0);
+      expand_half(bits, vvals + 2 * (T * kV + pre), za, e ? x1 : x0);
     }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
@@ -482,7 +485,18 @@ __device__ __forceinline__ uint32_t take_ticket(uint32_t *counter) {
   return old;
 }
 
-template <int NSTAGE, bool HIROWS>
+// Keep count and first packed value of stream (b, h) in one cache.  PERHEAD = false is the uniform
+// cache: the keep count is the kernel parameter, so it costs no register across the chunk loop.
+template <bool PERHEAD>
+__device__ __forceinline__ int keep_of(const HeadKeep &hk, int keep, int h) {
+  return PERHEAD ? hk.k[h] : keep;
+}
+template <bool PERHEAD>
+__device__ __forceinline__ int64_t base_of(const HeadKeep &hk, int keep, int b, int h, int H, int cap) {
+  return PERHEAD ? hk.value_base(b, h, H, cap) : (static_cast<int64_t>(b) * H + h) * cap * static_cast<int64_t>(keep);
+}
+
+template <int NSTAGE, bool HIROWS, bool PERHEAD>
 __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
@@ -589,10 +603,13 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
             const bool kside = warp == 0;
             const uint16_t *src =
                 kside ? P.kn + st.b * P.kn_sb + st.g * P.kn_sh : P.vn + st.b * P.vn_sb + st.g * P.vn_sh;
-            const int keep = kside ? P.keep_k : P.keep_v;
-            const int64_t slot = (static_cast<int64_t>(st.b) * P.Hkv + st.g) * (kside ? P.cap_k : P.cap_v) + p;
+            const int capx = kside ? P.cap_k : P.cap_v;
+            const int keep = kside ? keep_of<PERHEAD>(P.hk_k, P.keep_k, st.g) : keep_of<PERHEAD>(P.hk_v, P.keep_v, st.g);
+            const int64_t base = kside ? base_of<PERHEAD>(P.hk_k, P.keep_k, st.b, st.g, P.Hkv, capx)
+                                       : base_of<PERHEAD>(P.hk_v, P.keep_v, st.b, st.g, P.Hkv, capx);
+            const int64_t slot = (static_cast<int64_t>(st.b) * P.Hkv + st.g) * capx + p;
             uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + slot * kWords;
-            uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + slot * keep;
+            uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
             warp_compress_vector(src, keep, bm, vals, lane);
           }
         }
@@ -628,11 +645,20 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
     const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
     const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
-    mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
-    bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
-    bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-    bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
-    bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
+    if constexpr (PERHEAD) {
+      const int kK = P.hk_k.k[ps.g], kV = P.hk_v.k[ps.g];
+      mbar_expect_tx(bar, 512 + 32 * (kK + kV));
+      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      bulk_g2s(dst + 512, P.kval + P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK, 32 * kK, bar);
+      bulk_g2s(dst + 512 + 32 * kK, P.vval + P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV, 32 * kV, bar);
+    } else {  // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
+      mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
+      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
+      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
+    }
     sh_ps[warp] = ps;
     sh_punit[warp] = punit + kWarps;
   };
@@ -647,6 +673,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   for (;;) {
     const int seg_a = max(cs.start, u0), seg_e = min(cs.end(), u1);
     const int L = row_len(P, cs.b, cap);
+    const int kK = keep_of<PERHEAD>(P.hk_k, P.keep_k, cs.g), kV = keep_of<PERHEAD>(P.hk_v, P.keep_v, cs.g);
     load_q<HIROWS>(P, cs.b, cs.g, lane, qa);
     acc.reset();
 #pragma unroll 1
@@ -655,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       uint8_t *stage = wbase + slot * P.stage_bytes;
       if (!mbar_wait(bars + 8 * slot, (citem / NSTAGE) & 1, timed_out ? kWaitCyclesAfter : kWaitCycles))
         timed_out = true;
-      consume_chunk<HIROWS>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, lane, qa, acc);
+      consume_chunk<HIROWS, PERHEAD>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc);
       __syncwarp();
       produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
     }
@@ -688,20 +715,25 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
 // ------------------------------------------------------------------------------------ host side
 using SparseFn = void (*)(const DecodeParams);
 
-template <int NSTAGE>
+template <int NSTAGE, bool PERHEAD>
 SparseFn pick_rows(bool hirows) {
-  return hirows ? sparse_decode_kernel<NSTAGE, true> : sparse_decode_kernel<NSTAGE, false>;
+  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD> : sparse_decode_kernel<NSTAGE, false, PERHEAD>;
 }
 
-SparseFn pick_sparse(int nstage, bool hirows) {
+template <bool PERHEAD>
+SparseFn pick_stages(int nstage, bool hirows) {
   switch (nstage) {
-    case 2: return pick_rows<2>(hirows);
-    case 3: return pick_rows<3>(hirows);
-    default: return pick_rows<4>(hirows);
+    case 2: return pick_rows<2, PERHEAD>(hirows);
+    case 3: return pick_rows<3, PERHEAD>(hirows);
+    default: return pick_rows<4, PERHEAD>(hirows);
   }
 }
 
-int sparse_slot(int nstage, bool hirows) { return 20 + 2 * nstage + (hirows ? 1 : 0); }
+SparseFn pick_sparse(int nstage, bool hirows, bool perhead) {
+  return perhead ? pick_stages<true>(nstage, hirows) : pick_stages<false>(nstage, hirows);
+}
+
+int sparse_slot(int nstage, bool hirows, bool perhead) { return 12 + 2 * nstage + (hirows ? 1 : 0) + (perhead ? 10 : 0); }
 
 constexpr int kMinUnitsPerCta = 2 * kWarps;  // at least two chunks per warp
 constexpr int kMaxCtasPerSm = 4;
@@ -771,7 +803,7 @@ size_t sparse_workspace_bound(int B, int Hkv, int G, int max_len, int forced_spl
   return sparse_workspace_bytes(B, Hkv, G, sparse_decode_ctas(B, Hkv, max_len, forced_splits, kMaxCtasPerSm));
 }
 
-cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
+cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, bool perhead,
                         DecodePlan *plan) {
   const bool hirows = G > 8;
   const int stage_bytes = round_up(512 + 32 * (keep_k + keep_v), 128);
@@ -785,8 +817,8 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
     }
   const int warp_bytes = warp_bytes_of(nstage);
   const int smem = kWarps * warp_bytes + merge_bytes;
-  SparseFn fn = pick_sparse(nstage, hirows);
-  const int slot = sparse_slot(nstage, hirows);
+  SparseFn fn = pick_sparse(nstage, hirows, perhead);
+  const int slot = sparse_slot(nstage, hirows, perhead);
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), slot, smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -799,11 +831,12 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
   plan->stage_bytes = stage_bytes;
   plan->warp_bytes = warp_bytes;
   plan->smem_bytes = smem;
+  plan->perhead = perhead;
   return cudaSuccess;
 }
 
 cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
-  SparseFn fn = pick_sparse(plan.nstage, p.G > 8);
+  SparseFn fn = pick_sparse(plan.nstage, p.G > 8, plan.perhead);
   fn<<<plan.splits, kThreads, plan.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }

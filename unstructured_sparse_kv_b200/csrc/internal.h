@@ -15,11 +15,25 @@ void set_last_error(const char *msg);
 // Set a kernel's dynamic shared-memory limit once per device.
 cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes);
 
-cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H, int k,
-                            int cap, uint32_t *bitmap, uint16_t *values, uint32_t *tile_offset,
-                            cudaStream_t stream);
-cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H, int k,
-                          int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err, cudaStream_t stream);
+// Keep count of every kv head of one cache, and where each stream's packed values start: stream
+// (b, h) keeps k[h] values per token, and its values begin at element cap*(b*pre[H] + pre[h]),
+// pre being the prefix sums of k.  A uniform cache has k[h] = keep for every head.  Passed to the
+// kernels by value.
+constexpr int kMaxKvHeads = 128;
+struct HeadKeep {
+  int32_t k[kMaxKvHeads];
+  int32_t pre[kMaxKvHeads + 1];
+  __host__ __device__ __forceinline__ int64_t value_base(int b, int h, int H, int cap) const {
+    return static_cast<int64_t>(cap) * (static_cast<int64_t>(b) * pre[H] + pre[h]);
+  }
+};
+
+cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
+                            const HeadKeep &hk, int kmax, int cap, uint32_t *bitmap, uint16_t *values,
+                            uint32_t *tile_offset, cudaStream_t stream);
+cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H,
+                          const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
+                          cudaStream_t stream);
 
 struct DecodeParams {
   const uint16_t *q;  // [B][Hq][128]
@@ -28,7 +42,9 @@ struct DecodeParams {
   const uint16_t *kval;
   const uint32_t *vbm;
   const uint16_t *vval;
-  int keep_k, keep_v;
+  int keep_k, keep_v;  // the largest keep of each cache (sizes the staging buffers)
+  HeadKeep hk_k, hk_v;  // per kv head keep counts and value placement
+  int perhead;          // either cache has a keep count per kv head
   // dense caches (baseline kernel), [B][Hkv][cap][128]
   const uint16_t *kd;
   const uint16_t *vd;
@@ -60,6 +76,7 @@ struct DecodePlan {
   int stage_bytes;
   int warp_bytes;
   int smem_bytes;
+  bool perhead;  // sparse kernel: a cache with a keep count per kv head
 };
 
 // Dense fp16 baseline: plan (split count, pipeline depth, shared memory) and launch.
@@ -70,7 +87,7 @@ cudaError_t launch_dense(const DecodeParams &p, const DecodePlan &plan, cudaStre
 
 // Sparse decode over the compressed caches (one wave of CTAs over the end-to-end chunk sequence):
 // plan->splits holds the CTA count.
-cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits,
+cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, bool perhead,
                         DecodePlan *plan);
 cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
 int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_sm);

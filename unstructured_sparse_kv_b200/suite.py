@@ -41,7 +41,11 @@ class Timer:
 
 
 def decode_bytes(B, Hq, Hkv, L, kK, kV):
-    return B * Hkv * L * (32 + 2 * (kK + kV)) + 4 * B * Hq * D
+    """Bitmaps + kept values of K and V for every token-head, plus q and out (fp16); kK and kV are
+    keep counts, or lists with one keep count per kv head."""
+    kK = kK if isinstance(kK, (list, tuple)) else [kK] * Hkv
+    kV = kV if isinstance(kV, (list, tuple)) else [kV] * Hkv
+    return B * L * sum(32 + 2 * (a + b) for a, b in zip(kK, kV)) + 4 * B * Hq * D
 
 
 def dense_bytes(B, Hq, Hkv, L):
@@ -62,16 +66,17 @@ def decode_point(timer, peak, Hq, Hkv, B, L, sK, sV, seed, with_dense=True):
     V = synth.values(B, Hkv, L, D, seed, dev, capacity=cap)
     q = synth.queries(B, Hq, D, seed, dev)
     kc, vc = M.CompressedCache(B, Hkv, cap, sK), M.CompressedCache(B, Hkv, cap, sV)
-    M.mustafar_compress(K, L, sK, kc)
-    M.mustafar_compress(V, L, sV, vc)
+    M.mustafar_compress(K, L, sK if kc.sparsity is not None else 0.0, kc)  # per-head caches ignore it
+    M.mustafar_compress(V, L, sV if vc.sparsity is not None else 0.0, vc)
     seq = torch.full((B,), L, dtype=torch.int32, device=dev)
     out = torch.empty_like(q)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
     ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, L), dtype=torch.uint8, device=dev)
     t_sparse = timer.median_us(lambda: M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0, out=out, lse=lse, workspace=ws))
-    nb = decode_bytes(B, Hq, Hkv, L, kc.keep, vc.keep)
+    nb = decode_bytes(B, Hq, Hkv, L, kc.head_keep, vc.head_keep)
     rec = {"kind": "decode", "q_heads": Hq, "kv_heads": Hkv, "batch": B, "context": L, "sparsity_k": sK,
-           "sparsity_v": sV, "keep_k": kc.keep, "keep_v": vc.keep,
+           "sparsity_v": sV, "keep_k": kc.head_keep if kc.per_head else kc.keep,
+           "keep_v": vc.head_keep if vc.per_head else vc.keep,
            "splits": M.mustafar_decode_plan_splits(B, Hkv, L, kc.keep, vc.keep),
            "sparse_us": t_sparse, "sparse_bytes": nb, "sparse_gbs": nb / t_sparse / 1e3,
            "sparse_frac_of_peak": nb / t_sparse / 1e3 / peak,
@@ -105,7 +110,7 @@ def compress_point(timer, peak, B, L, H, s, seed):
     return rec
 
 
-def run(out_path: str, peak: float, which=("c1", "c3", "c4", "sweep"), log=print):
+def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "sweep"), log=print):
     torch.cuda.set_device(0)
     timer = Timer("cuda")
     recs = []
@@ -123,6 +128,13 @@ def run(out_path: str, peak: float, which=("c1", "c3", "c4", "sweep"), log=print
     if "c4" in which:
         for s in (0.3, 0.5, 0.7):
             emit(dict(compress_point(timer, peak, 8, 16384, 8, s, 1004), workload="compress b8 16k h8"))
+    if "heads" in which:
+        # a sparsity per kv head around 0.7 (K) and its mirror (V), against uniform 0.7 on the same inputs
+        hs = [0.5, 0.6, 0.7, 0.8, 0.9, 0.7, 0.6, 0.8]
+        emit(dict(decode_point(timer, peak, 32, 8, 8, 4096, hs, hs[::-1], 1006, with_dense=False),
+                  workload="b8 ctx4096 per-head sparsity (mean 0.7)"))
+        emit(dict(decode_point(timer, peak, 32, 8, 8, 4096, 0.7, 0.7, 1006, with_dense=False),
+                  workload="b8 ctx4096 uniform 0.7 (same inputs)"))
     if "sweep" in which:
         for Hkv in (8, 32):
             for B in (1, 8, 32):

@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define MUSTAFAR_ABI_VERSION 2
+#define MUSTAFAR_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MUSTAFAR_API __attribute__((visibility("default")))
@@ -91,7 +91,16 @@ typedef struct {
    * and its tile offsets are 64*i*head_keep[h].  NULL: every head keeps `keep` (the same layout
    * with all head_keep[h] = keep).  Read at call time only; the library keeps no pointer to it. */
   const int32_t *head_keep;
+  /* MUSTAFAR_PATTERN_TOPK: per-token top-keep pruning (the method).  MUSTAFAR_PATTERN_2_4: the
+   * 2:4 semi-structured comparison pattern the pages benchmark against (MUSTAFAR summary,
+   * "Experimental setup"): every group of 4 consecutive channels keeps its 2 largest magnitudes
+   * (ties to the lower channel), so keep must be head_dim/2 and head_keep NULL.  Both are stored in
+   * the same bitmap format, and the decode calls read either. */
+  int32_t pattern;
 } mustafar_cache_t;
+
+#define MUSTAFAR_PATTERN_TOPK 0
+#define MUSTAFAR_PATTERN_2_4 1
 
 /* Keep count for a pruning sparsity s (fraction of channels removed, README
  * Part II: a setting of 0.5 prunes half of them).  Returns head_dim - floor(s*head_dim), or -1
@@ -117,8 +126,9 @@ MUSTAFAR_API mustafar_status mustafar_cache_sizes_per_head(int32_t batch, int32_
  *              x[b*stride_b + h*stride_h + t*stride_t + c] (strides in elements,
  *              channels contiguous; x and every stride a multiple of 8 elements).
  *   L        : tokens [0, L) are compressed into slots [0, L); 0 <= L <= capacity.
- *   sparsity : must satisfy c->keep == mustafar_keep_count(c->head_dim, sparsity); ignored
- *              when c->head_keep is set (each head then keeps c->head_keep[h]).
+ *   sparsity : must satisfy c->keep == mustafar_keep_count(c->head_dim, sparsity) (0.5 for a
+ *              2:4 cache); ignored when c->head_keep is set (each head then keeps c->head_keep[h]).
+ * The selection follows c->pattern (per-token top-keep, or 2:4).
  *   c        : the destination cache; its whole tile_offset array is written.
  *   d_err    : optional device word (unused by this call today; may be NULL).
  * Slots >= L are not touched.  Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */

@@ -145,7 +145,12 @@ def compress(x_bits: np.ndarray, k: int, capacity: int, L: int | None = None) ->
     B, H, T, d = x.shape
     L = T if L is None else L
     assert capacity % TILE_TOKENS == 0 and L <= capacity and L <= T
-    mask = select_sort(x[:, :, :L], k)
+    return _compress_mask(x, select_sort(x[:, :, :L], k), k, capacity, L)
+
+
+def _compress_mask(x: np.ndarray, mask: np.ndarray, k: int, capacity: int, L: int) -> dict:
+    """The bitmap format of tokens [0, L) of ``x`` given their kept-mask (k kept per token)."""
+    B, H, T, d = x.shape
     bitmap = np.zeros((B, H, capacity, d // WORD_BITS), dtype=np.uint32)
     bitmap[:, :, :L] = bitmap_words(mask)
     values = np.zeros((B, H, capacity * k), dtype=np.uint16)
@@ -185,6 +190,54 @@ def append(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
     x = np.asarray(x_new_bits, dtype=np.uint16)  # [B, H, d]
     B, H, d = x.shape
     mask = select_sort(x, k)
+    words = bitmap_words(mask)
+    for b in range(B):
+        p = int(pos[b])
+        cache["bitmap"][b, :, p] = words[b]
+        for h in range(H):
+            cache["values"][b, h, p * k:(p + 1) * k] = x[b, h][mask[b, h]]
+
+
+# --------------------------------------------------------------------------------------
+# 2:4 semi-structured pruning (the comparison pattern)
+# --------------------------------------------------------------------------------------
+# The pages compare against 2:4 semi-structured sparsity (MUSTAFAR summary, atlas.scime.ai,
+# "Experimental setup": baselines).  Reading: every group of 4 consecutive channels of a
+# (token, kv head) vector keeps its 2 largest-magnitude elements (same key, ties to the lower
+# channel), so every token keeps exactly d/2 channels (sparsity 0.5) and the result is stored in
+# the same bitmap format.
+GROUP = 4
+GROUP_KEEP = 2
+
+
+def select_24(x_bits: np.ndarray) -> np.ndarray:
+    """Kept-mask of 2:4 pruning over the last axis: the top 2 of each group of 4 consecutive channels."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    d = x.shape[-1]
+    groups = x.reshape(x.shape[:-1] + (d // GROUP, GROUP))
+    return select_sort(groups, GROUP_KEEP).reshape(x.shape)
+
+
+def prune_24(x_bits: np.ndarray) -> np.ndarray:
+    x = np.asarray(x_bits, dtype=np.uint16)
+    return np.where(select_24(x), x, np.uint16(0)).astype(np.uint16)
+
+
+def compress_24(x_bits: np.ndarray, capacity: int, L: int | None = None) -> dict:
+    """2:4-pruned tokens [0, L) of a dense cache [B, H, T, d] in the bitmap format (k = d/2)."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    B, H, T, d = x.shape
+    L = T if L is None else L
+    assert capacity % TILE_TOKENS == 0 and L <= capacity and L <= T
+    return _compress_mask(x, select_24(x[:, :, :L]), d // 2, capacity, L)
+
+
+def append_24(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
+    """2:4-prune + compress one new token per (b, h) into slot pos[b] (in place)."""
+    k = cache["k"]
+    x = np.asarray(x_new_bits, dtype=np.uint16)  # [B, H, d]
+    B, H, d = x.shape
+    mask = select_24(x)
     words = bitmap_words(mask)
     for b in range(B):
         p = int(pos[b])

@@ -15,6 +15,8 @@ oracle disagrees with the fact it checks.  Facts used:
 * per-head keep counts: with one keep for every head the per-head layout equals the uniform
   one byte for byte; the streams tile the value array exactly; brute-force ranks and popcounts
   per head; round trip to the per-head pruned cache; append == compress.
+* 2:4 pattern: a hand-derived 32-channel fixture (selection, bitmap word, packed values);
+  exactly 2 of every 4 channels; brute-force ranks per group; round trip; append == compress.
 """
 from __future__ import annotations
 
@@ -304,9 +306,46 @@ def pin_heads_append_equals_compress(O):
         assert np.array_equal(full[key], part[key]), key
 
 
+# ----------------------------------------------------------------------------- 2:4 comparison pattern
+def pin_golden_24(O):
+    g = _load("select_24.json")
+    x = np.array([int(h, 16) for h in g["x_hex_by_channel"]], dtype=np.uint16).reshape(1, 1, 1, 32)
+    mask = O.select_24(x)[0, 0, 0]
+    assert np.flatnonzero(mask).tolist() == g["kept_channels"]
+    assert int(O.bitmap_words(mask[None])[0, 0]) == int(g["bitmap_word_hex"], 16)
+    comp = O.compress_24(x, 64)
+    assert comp["k"] == 16
+    assert comp["values"][0, 0, :16].tolist() == [int(h, 16) for h in g["packed_values_hex"]]
+
+
+def pin_24_structure(O):
+    rng = np.random.default_rng(29)
+    B, H, L, d, cap = 2, 2, 70, 128, 128
+    x = rand_bits(rng, (B, H, L, d))
+    x[0, 1, 3] = rand_bits(rng, (d,), tie_heavy=True)
+    x[1, 0, 9] = 0x3C00  # every magnitude equal
+    mask = O.select_24(x)
+    groups = mask.reshape(B, H, L, d // 4, 4)
+    assert (groups.sum(-1) == 2).all()  # exactly two of every four, so d/2 per token
+    # brute-force ranks inside each group (independent of the sort-based selection)
+    xg = x.reshape(B, H, L, d // 4, 4)
+    assert np.array_equal(groups, O.select_rank_bruteforce(xg, 2))
+    comp = O.compress_24(x, cap)
+    assert comp["k"] == d // 2
+    dec = O.decompress(comp["bitmap"], comp["values"], d // 2, L, d)
+    assert np.array_equal(dec, O.prune_24(x))
+    assert np.array_equal(O.bitmap_to_mask(comp["bitmap"][:, :, :L], d), mask)
+    part = O.compress_24(x, cap, L - 2)
+    for s in range(2):
+        O.append_24(part, x[:, :, L - 2 + s], np.full(B, L - 2 + s))
+    for key in ("bitmap", "values", "tile_offset"):
+        assert np.array_equal(comp[key], part[key]), key
+
+
 ALL_PINS = [pin_golden_selection, pin_golden_keep_count, pin_bruteforce_selection, pin_threshold_invariant,
             pin_roundtrip_and_popcount, pin_compressed_size, pin_dense_limit_sdpa, pin_golden_attention,
-            pin_attention_invariants, pin_append_equals_compress, pin_heads_layout, pin_heads_append_equals_compress]
+            pin_attention_invariants, pin_append_equals_compress, pin_heads_layout, pin_heads_append_equals_compress,
+            pin_golden_24, pin_24_structure]
 
 
 def failing_pins(O):

@@ -33,7 +33,7 @@ def test_header_lists_the_binding_symbols():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.mustafar_abi_version() == 2
+    assert lib.mustafar_abi_version() == 3
 
 
 def test_keep_count_matches_oracle(lib):
@@ -138,16 +138,16 @@ def test_per_head_keep_checks_and_sizes(lib):
     for kwargs, want, msg in [(dict(keep=39), 1, "largest head_keep"), ]:
         bad = _cache(**kwargs)
         bad.head_keep = c.head_keep
-        st, err = _status(lib, "mustafar_append", 0x5000, 256, 128, 0x6000, C.byref(bad), None, None)
+        st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(bad), None, None)
         assert st == want and msg in err, (st, err)
     zero = (C.c_int32 * 2)(39, 0)
     bad = _cache(keep=39)
     bad.head_keep = C.cast(zero, C.c_void_p).value
-    st, err = _status(lib, "mustafar_append", 0x5000, 256, 128, 0x6000, C.byref(bad), None, None)
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(bad), None, None)
     assert st == 1 and "head_keep[1]" in err
     many = _cache(heads=129)
     many.head_keep = C.cast((C.c_int32 * 129)(*([39] * 129)), C.c_void_p).value
-    st, err = _status(lib, "mustafar_append", 0x5000, 256, 128, 0x6000, C.byref(many), None, None)
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(many), None, None)
     assert st == 2 and "128" in err
     # sizes: bitmap and offsets as for a uniform cache, values 2 * B * cap * sum(head_keep)
     B, H, cap, hk = 3, 4, 192, [13, 39, 64, 128]
@@ -157,6 +157,24 @@ def test_per_head_keep_checks_and_sizes(lib):
         M.mustafar_cache_sizes_per_head(B, H, cap, [13, 39, 64, 129])
     # a uniform head_keep gives exactly the uniform sizes
     assert M.mustafar_cache_sizes_per_head(B, H, cap, [39] * H) == M.mustafar_cache_sizes(B, H, 128, cap, 0.7)
+
+
+def test_pattern_checks(lib):
+    # every call stops in host validation (stride 100 is deliberately misaligned): nothing launches
+    c = _cache(keep=64)
+    c.pattern = 1
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(c), None, None)
+    assert st == 3  # a valid 2:4 descriptor passes the pattern checks
+    bad = _cache(keep=39)
+    bad.pattern = 1
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(bad), None, None)
+    assert st == 1 and "2:4" in err
+    bad = _cache(keep=64)
+    bad.pattern = 7
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(bad), None, None)
+    assert st == 1 and "pattern" in err
+    with pytest.raises(ValueError):
+        M.CompressedCache(1, 1, 64, 0.7, pattern="2:4", device="cpu")
 
 
 def test_workspace_query(lib):

@@ -368,6 +368,85 @@ def test_per_head_llama3_gqa_b8_ctx4096_mean_s07():
     U.assert_attn_close(out[rows], o_ref, lse[rows], l_ref, tag="per-head b8 ctx4096")
 
 
+# ------------------------------------------------------------------------------------ 2:4 comparison pattern
+def test_24_compress_append_bit_exact():
+    B, H, L0, L1, cap = 2, 3, 130, 140, 192
+    rng = np.random.default_rng(71)
+    x = synth.keys(B, H, L1, D, 71, "cpu").permute(0, 2, 1, 3).contiguous()  # [B, L, H, d] storage
+    xb = x.view(torch.int16).numpy().view(np.uint16).copy()
+    xb[0, 3, 1] = rng.choice(TIE_ROWS, D)
+    xb[1, 77, 2] = 0x3C00
+    xb[0, 100, 0, :64] = 0x8000
+    xdev = torch.from_numpy(xb.view(np.int16)).view(torch.float16).to(DEV)
+    view = xdev.permute(0, 2, 1, 3)
+    c = M.CompressedCache(B, H, cap, 0.5, pattern="2:4")
+    M.mustafar_compress(view, L0, 0.5, c)
+    for t in range(L0, L1):
+        M.mustafar_append(view[:, :, t], torch.full((B,), t, dtype=torch.int32, device=DEV), c)
+    ref = oracle.compress_24(np.ascontiguousarray(xb.transpose(0, 2, 1, 3))[:, :, :L1], cap, L1)
+    bm, vals, offs = U.cache_np(c)
+    assert np.array_equal(bm[:, :, :L1], ref["bitmap"][:, :, :L1])
+    assert np.array_equal(vals[:, :, :L1 * 64], ref["values"][:, :, :L1 * 64])
+    assert np.array_equal(offs, ref["tile_offset"])
+
+
+@pytest.mark.parametrize("splits", [0, 2])
+def test_24_decode_attn_and_step(splits):
+    B, Hq, Hkv, L, cap = 2, 8, 2, 300, 320
+    K = synth.keys(B, Hkv, cap, D, 72, DEV)
+    V = synth.values(B, Hkv, cap, D, 72, DEV)
+    kc = M.CompressedCache(B, Hkv, cap, 0.5, pattern="2:4")
+    vc = M.CompressedCache(B, Hkv, cap, 0.5, pattern="2:4")
+    M.mustafar_compress(K, L, 0.5, kc)
+    M.mustafar_compress(V, L, 0.5, vc)
+    q = synth.queries(B, Hq, D, 72, DEV)
+    seq = synth.seq_lens(B, L, True, 72)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), L, 1.0, num_splits=splits)
+    Kb, Vb = U.bits(K), U.bits(V)
+    o_ref, l_ref = oracle.attention(U.bits(q), oracle.prune_24(Kb[:, :, :L]), oracle.prune_24(Vb[:, :, :L]),
+                                    seq.numpy(), 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"2:4 decode splits {splits}")
+    pos = seq.clone().to(DEV)
+    rows = torch.arange(B, device=DEV)
+    kn, vn = synth.step_tokens(B, Hkv, D, 72, 0, DEV)
+    K[rows, :, pos.long()] = kn
+    V[rows, :, pos.long()] = vn
+    out, lse = M.mustafar_decode_step(q, kn, vn, pos, kc, vc, L + 1, 1.0, num_splits=splits)
+    lens = (pos + 1).cpu().numpy()
+    Kb, Vb = U.bits(K), U.bits(V)
+    o_ref, l_ref = oracle.attention(U.bits(q), oracle.prune_24(Kb[:, :, :L + 1]), oracle.prune_24(Vb[:, :, :L + 1]),
+                                    lens, 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"2:4 fused step splits {splits}")
+    for cache, xb in ((kc, Kb), (vc, Vb)):
+        bm, vals, _ = U.cache_np(cache)
+        for b in range(B):
+            ref = oracle.compress_24(xb[b:b + 1, :, :lens[b]], cap, int(lens[b]))
+            assert np.array_equal(bm[b, :, :lens[b]], ref["bitmap"][0, :, :lens[b]])
+            assert np.array_equal(vals[b, :, :lens[b] * 64], ref["values"][0, :, :lens[b] * 64])
+
+
+def test_24_llama3_gqa_b8_ctx4096():
+    B, Hq, Hkv, L = 8, 32, 8, 4096
+    K = synth.keys(B, Hkv, L, D, 1007, DEV)
+    V = synth.values(B, Hkv, L, D, 1007, DEV)
+    kc = M.CompressedCache(B, Hkv, L, 0.5, pattern="2:4")
+    vc = M.CompressedCache(B, Hkv, L, 0.5, pattern="2:4")
+    M.mustafar_compress(K, L, 0.5, kc)
+    M.mustafar_compress(V, L, 0.5, vc)
+    q = synth.queries(B, Hq, D, 1007, DEV)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, torch.full((B,), L, dtype=torch.int32, device=DEV), L, 1.0)
+    rows = [1, 6]
+    streams = [(1, 0), (6, 5)]
+    Kb, Vb = U.bits(K), U.bits(V)
+    bm, vals, _ = U.cache_np(kc)
+    for b, h in streams:
+        ref = oracle.compress_24(Kb[b:b + 1, h:h + 1], L, L)
+        assert np.array_equal(bm[b, h], ref["bitmap"][0, 0]) and np.array_equal(vals[b, h], ref["values"][0, 0])
+    o_ref, l_ref = oracle.attention(U.bits(q[rows]), oracle.prune_24(Kb[rows]), oracle.prune_24(Vb[rows]),
+                                    [L] * len(rows), 1.0)
+    U.assert_attn_close(out[rows], o_ref, lse[rows], l_ref, tag="2:4 b8 ctx4096")
+
+
 # ------------------------------------------------------------------------------------ the workload shapes
 def test_llama3_gqa_b1_ctx1024_s05():
     B, Hq, Hkv, L = 1, 32, 8, 1024

@@ -101,6 +101,43 @@ def _mutant(**overrides):
                 base = ns.value_base_heads(b, h, hk, cap) + p * k
                 cache["values"][base:base + k] = x[b, h][mask[b]]
     ns.append_heads = append_heads
+    # 2:4 functions, rebound to the namespace's select_24 / select_sort
+    if "select_24" not in overrides:
+        def select_24(x_bits):
+            x = np.asarray(x_bits, dtype=np.uint16)
+            d = x.shape[-1]
+            return ns.select_sort(x.reshape(x.shape[:-1] + (d // 4, 4)), 2).reshape(x.shape)
+        ns.select_24 = select_24
+    def prune_24(x_bits):
+        x = np.asarray(x_bits, dtype=np.uint16)
+        return np.where(ns.select_24(x), x, np.uint16(0)).astype(np.uint16)
+    ns.prune_24 = prune_24
+    def compress_24(x_bits, capacity, L=None):
+        x = np.asarray(x_bits, dtype=np.uint16)
+        B, H, T, d = x.shape
+        L = T if L is None else L
+        mask = ns.select_24(x[:, :, :L])
+        k = d // 2
+        bitmap = np.zeros((B, H, capacity, d // 32), dtype=np.uint32)
+        bitmap[:, :, :L] = ns.bitmap_words(mask)
+        values = np.zeros((B, H, capacity * k), dtype=np.uint16)
+        values[:, :, : L * k] = x[:, :, :L][mask].reshape(B, H, -1)[:, :, : L * k]
+        starts = np.arange(capacity // 64, dtype=np.int64) * 64 * k
+        return {"bitmap": bitmap, "values": values,
+                "tile_offset": np.broadcast_to(starts, (B, H, capacity // 64)).astype(np.uint32), "k": k, "L": L}
+    ns.compress_24 = compress_24
+    def append_24(cache, x_new_bits, pos):
+        k = cache["k"]
+        x = np.asarray(x_new_bits, dtype=np.uint16)
+        mask = ns.select_24(x)
+        words = ns.bitmap_words(mask)
+        for b in range(x.shape[0]):
+            p = int(pos[b])
+            cache["bitmap"][b, :, p] = words[b]
+            for h in range(x.shape[1]):
+                v = x[b, h][mask[b, h]]
+                cache["values"][b, h, p * k:p * k + v.size] = v[:k]
+    ns.append_24 = append_24
     return ns
 
 
@@ -183,7 +220,23 @@ def prune_heads_max(x_bits, head_keep):             # every head pruned with the
     return np.concatenate([real.prune(x[:, h:h + 1], int(max(head_keep))) for h in range(x.shape[1])], axis=1)
 
 
+def sel24_strided(x_bits):            # groups of channels c, c+d/4, c+d/2, c+3d/4 instead of 4 neighbours
+    x = np.asarray(x_bits, np.uint16)
+    d = x.shape[-1]
+    g = np.swapaxes(x.reshape(x.shape[:-1] + (4, d // 4)), -1, -2)
+    m = real.select_sort(g, 2)
+    return np.swapaxes(m, -1, -2).reshape(x.shape)
+
+
+def sel24_groups_of_8(x_bits):         # 4 of every 8 instead of 2 of every 4
+    x = np.asarray(x_bits, np.uint16)
+    d = x.shape[-1]
+    return real.select_sort(x.reshape(x.shape[:-1] + (d // 8, 8)), 4).reshape(x.shape)
+
+
 MUTANTS = {
+    "2:4 strided groups": dict(select_24=sel24_strided),
+    "2:4 as 4:8": dict(select_24=sel24_groups_of_8),
     "per-head base after own head": dict(value_base_heads=base_next_head),
     "per-head streams head-major": dict(value_base_heads=base_head_major),
     "per-head prune with max keep": dict(prune_heads=prune_heads_max),

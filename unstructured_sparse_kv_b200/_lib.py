@@ -20,6 +20,8 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "MISALIGNED", 4:
 DEVERR_POS_RANGE = 0x1
 DEVERR_LEN_RANGE = 0x2
 HEAD_DIM = 128
+PATTERN_TOPK = 0   # per-token top-keep pruning (the method)
+PATTERN_2_4 = 1    # 2:4 semi-structured pruning (the comparison pattern)
 
 # every symbol include/mustafar.h declares
 ABI_SYMBOLS = (
@@ -40,7 +42,8 @@ class CacheT(C.Structure):
     """Mirror of mustafar_cache_t."""
     _fields_ = [("batch", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
                 ("capacity", C.c_int32), ("keep", C.c_int32), ("bitmap", C.c_void_p),
-                ("values", C.c_void_p), ("tile_offset", C.c_void_p), ("head_keep", C.c_void_p)]
+                ("values", C.c_void_p), ("tile_offset", C.c_void_p), ("head_keep", C.c_void_p),
+                ("pattern", C.c_int32)]
 
 
 _lib = None
@@ -145,11 +148,17 @@ class CompressedCache:
     """Caller-owned device arrays of one compressed cache (K or V) plus its C descriptor.
 
     ``sparsity`` is one value for every kv head, or a sequence with one sparsity per kv head
-    (then head h keeps ``mustafar_keep_count(head_dim, sparsity[h])`` channels per token)."""
+    (then head h keeps ``mustafar_keep_count(head_dim, sparsity[h])`` channels per token).
+    ``pattern="2:4"`` selects 2:4 semi-structured pruning instead (sparsity 0.5, one value)."""
 
     def __init__(self, batch: int, num_kv_heads: int, capacity: int, sparsity, head_dim: int = HEAD_DIM,
-                 device="cuda"):
+                 device="cuda", pattern: str = "topk"):
         self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
+        if pattern not in ("topk", "2:4"):
+            raise ValueError("pattern must be 'topk' or '2:4'")
+        if pattern == "2:4" and (isinstance(sparsity, (list, tuple)) or float(sparsity) != 0.5):
+            raise ValueError("a 2:4 cache has sparsity 0.5 for every head")
+        self.pattern = pattern
         self._head_keep_arr = None
         if isinstance(sparsity, (list, tuple)):
             if len(sparsity) != num_kv_heads:
@@ -171,7 +180,8 @@ class CompressedCache:
         self.tile_offset = torch.zeros(no // 4, dtype=torch.int32, device=device)
         hk = C.cast(self._head_keep_arr, C.c_void_p).value if self._head_keep_arr is not None else None
         self._struct = CacheT(batch, num_kv_heads, head_dim, capacity, self.keep, self.bitmap.data_ptr(),
-                              self.values.data_ptr(), self.tile_offset.data_ptr(), hk)
+                              self.values.data_ptr(), self.tile_offset.data_ptr(), hk,
+                              PATTERN_2_4 if pattern == "2:4" else PATTERN_TOPK)
 
     @property
     def struct(self) -> CacheT:

@@ -50,6 +50,10 @@ mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: capacity must be a multiple of 64 (got %d)", name, c->capacity);
   if (c->keep < 1 || c->keep > c->head_dim)
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: keep must lie in [1, head_dim] (got %d)", name, c->keep);
+  if (c->pattern != MUSTAFAR_PATTERN_TOPK && c->pattern != MUSTAFAR_PATTERN_2_4)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: pattern must be MUSTAFAR_PATTERN_TOPK or _2_4 (got %d)", name, c->pattern);
+  if (c->pattern == MUSTAFAR_PATTERN_2_4 && (c->keep != c->head_dim / 2 || c->head_keep != nullptr))
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: a 2:4 cache keeps head_dim/2 channels and has no head_keep", name);
   if (c->head_keep != nullptr) {
     if (c->num_kv_heads > kMaxKvHeads)
       return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: per-head keep supports at most %d kv heads", name, kMaxKvHeads);
@@ -188,7 +192,8 @@ mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t strid
   }
   cudaError_t e = launch_compress(static_cast<const uint16_t *>(x), stride_b, stride_h, stride_t, L, c->batch,
                                   c->num_kv_heads, head_keep_of(c), c->keep, c->capacity, c->bitmap, c->values,
-                                  c->tile_offset, reinterpret_cast<cudaStream_t>(stream));
+                                  c->tile_offset, c->pattern == MUSTAFAR_PATTERN_2_4,
+                                  reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "compress launch");
 }
 
@@ -203,7 +208,7 @@ mustafar_status mustafar_append(const void *x, int64_t stride_b, int64_t stride_
   if (!aligned(d_pos, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "append: pos must be 4-byte aligned");
   cudaError_t e = launch_append(static_cast<const uint16_t *>(x), stride_b, stride_h, d_pos, c->batch,
                                 c->num_kv_heads, head_keep_of(c), c->capacity, c->bitmap, c->values, d_err,
-                                reinterpret_cast<cudaStream_t>(stream));
+                                c->pattern == MUSTAFAR_PATTERN_2_4, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "append launch");
 }
 
@@ -332,6 +337,8 @@ mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_heads, const m
   p.hk_k = head_keep_of(k);
   p.hk_v = head_keep_of(v);
   p.perhead = k->head_keep != nullptr || v->head_keep != nullptr;
+  p.p24_k = k->pattern == MUSTAFAR_PATTERN_2_4;
+  p.p24_v = v->pattern == MUSTAFAR_PATTERN_2_4;
   p.cap_k = k->capacity;
   p.cap_v = v->capacity;
   p.seq_len = d_seq_len;
@@ -381,6 +388,8 @@ mustafar_status mustafar_decode_step(const void *q, int32_t num_q_heads, const v
   p.hk_k = head_keep_of(k);
   p.hk_v = head_keep_of(v);
   p.perhead = k->head_keep != nullptr || v->head_keep != nullptr;
+  p.p24_k = k->pattern == MUSTAFAR_PATTERN_2_4;
+  p.p24_v = v->pattern == MUSTAFAR_PATTERN_2_4;
   p.cap_k = k->capacity;
   p.cap_v = v->capacity;
   p.B = k->batch;

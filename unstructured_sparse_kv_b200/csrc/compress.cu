@@ -21,6 +21,7 @@ constexpr int kRowBytesDense = kHeadDim * 2;  // 256
 // byte offset of 16-byte chunk j of staged row `tok` (XOR swizzle: conflict-free row reads)
 __device__ __forceinline__ int stage_off(int tok, int j) { return tok * kRowBytesDense + ((j ^ (tok & 15)) << 4); }
 
+template <bool P24>
 __global__ void __launch_bounds__(kCompressThreads)
 compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, const HeadKeep hk,
                 int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
@@ -64,7 +65,11 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
       raw[4 * j + 3] = v.w;
     }
     uint32_t bm[kWords];
-    topk_bitmap(raw, k, bm);
+    if constexpr (P24) {
+      bitmap_24(raw, bm);
+    } else {
+      topk_bitmap(raw, k, bm);
+    }
     reinterpret_cast<uint4 *>(bitmap)[stream * cap + t0 + tid] = make_uint4(bm[0], bm[1], bm[2], bm[3]);
     // pack the kept values in ascending channel order
     uint16_t *dst = out_stage + tid * k;
@@ -95,6 +100,7 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
 // vectors).  Lane l holds channels l, l+32, l+64, l+96, so a ballot over one of its four keys
 // is directly one bitmap word.  The same selection as topk_bitmap: binary search for the k-th
 // largest key T, then the keys equal to T are taken lowest channel first.
+template <bool P24>
 __global__ void __launch_bounds__(128)
 append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int32_t *__restrict__ pos, int B,
               int H, const HeadKeep hk, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
@@ -111,31 +117,37 @@ append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int3
   const uint16_t *src = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
   const int64_t stream = static_cast<int64_t>(b) * H + h;
   const int k = hk.k[h];
-  warp_compress_vector(src, k, bitmap + (stream * cap + p) * kWords,
-                       values + hk.value_base(b, h, H, cap) + static_cast<int64_t>(p) * k, lane);
+  uint32_t *bm_dst = bitmap + (stream * cap + p) * kWords;
+  uint16_t *val_dst = values + hk.value_base(b, h, H, cap) + static_cast<int64_t>(p) * k;
+  if constexpr (P24) {
+    warp_compress_vector_24(src, bm_dst, val_dst, lane);
+  } else {
+    warp_compress_vector(src, k, bm_dst, val_dst, lane);
+  }
 }
 
 cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
                             const HeadKeep &hk, int kmax, int cap, uint32_t *bitmap, uint16_t *values,
-                            uint32_t *tile_offset, cudaStream_t stream) {
+                            uint32_t *tile_offset, bool p24, cudaStream_t stream) {
+  auto kernel = p24 ? compress_kernel<true> : compress_kernel<false>;
   const size_t smem = kCompressThreads * kRowBytesDense + static_cast<size_t>(kCompressThreads) * kmax * 2;
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(compress_kernel), 0,
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kernel), p24 ? 9 : 0,
                                     kCompressThreads * kRowBytesDense + kCompressThreads * kHeadDim * 2);
   if (e != cudaSuccess) return e;
   const int nbx = L > 0 ? (L + kCompressThreads - 1) / kCompressThreads : 1;
   dim3 grid(nbx, H, B);
-  compress_kernel<<<grid, kCompressThreads, smem, stream>>>(x, sb, sh, st, L, H, hk, cap, bitmap, values,
-                                                            tile_offset);
+  kernel<<<grid, kCompressThreads, smem, stream>>>(x, sb, sh, st, L, H, hk, cap, bitmap, values, tile_offset);
   return cudaGetLastError();
 }
 
 cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H,
                           const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
-                          cudaStream_t stream) {
+                          bool p24, cudaStream_t stream) {
+  auto kernel = p24 ? append_kernel<true> : append_kernel<false>;
   const int warps = B * H;
   const int threads = 128;  // 4 vectors per CTA
-  append_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, hk, cap,
-                                                                              bitmap, values, err);
+  kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, hk, cap, bitmap,
+                                                                       values, err);
   return cudaGetLastError();
 }
 

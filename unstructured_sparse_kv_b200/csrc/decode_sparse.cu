@@ -610,7 +610,10 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
             const int64_t slot = (static_cast<int64_t>(st.b) * P.Hkv + st.g) * capx + p;
             uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + slot * kWords;
             uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
-            warp_compress_vector(src, keep, bm, vals, lane);
+            if (kside ? P.p24_k : P.p24_v)
+              warp_compress_vector_24(src, bm, vals, lane);
+            else
+              warp_compress_vector(src, keep, bm, vals, lane);
           }
         }
       }

@@ -30,10 +30,10 @@ struct HeadKeep {
 
 cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
                             const HeadKeep &hk, int kmax, int cap, uint32_t *bitmap, uint16_t *values,
-                            uint32_t *tile_offset, cudaStream_t stream);
+                            uint32_t *tile_offset, bool p24, cudaStream_t stream);
 cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H,
                           const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
-                          cudaStream_t stream);
+                          bool p24, cudaStream_t stream);
 
 struct DecodeParams {
   const uint16_t *q;  // [B][Hq][128]
@@ -45,6 +45,7 @@ struct DecodeParams {
   int keep_k, keep_v;  // the largest keep of each cache (sizes the staging buffers)
   HeadKeep hk_k, hk_v;  // per kv head keep counts and value placement
   int perhead;          // either cache has a keep count per kv head
+  int p24_k, p24_v;     // the cache is 2:4-pruned (the fused step appends with that rule)
   // dense caches (baseline kernel), [B][Hkv][cap][128]
   const uint16_t *kd;
   const uint16_t *vd;

@@ -137,4 +137,54 @@ __device__ __forceinline__ void warp_compress_vector(const uint16_t *src, int k,
   }
 }
 
+// ---- 2:4 semi-structured pruning (the comparison pattern of the pages' baselines): in every group
+// of 4 consecutive channels keep the 2 largest keys, ties to the lower channel.  An element is kept
+// when fewer than 2 group mates beat it (a mate beats it with a larger key, or an equal key at a
+// lower channel).
+
+// Bitmap of the 2:4 selection of one vector (raw as in topk_bitmap).
+__device__ __forceinline__ void bitmap_24(const uint32_t (&raw)[64], uint32_t (&bm)[kWords]) {
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) bm[w] = 0u;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {  // group j: channels 4j..4j+3 = raw[2j] (lo, hi), raw[2j+1] (lo, hi)
+    const uint32_t a = raw[2 * j] & 0x7FFFu, b = (raw[2 * j] >> 16) & 0x7FFFu;
+    const uint32_t c = raw[2 * j + 1] & 0x7FFFu, d = (raw[2 * j + 1] >> 16) & 0x7FFFu;
+    const int ra = (b > a) + (c > a) + (d > a);
+    const int rb = (a >= b) + (c > b) + (d > b);
+    const int rc = (a >= c) + (b >= c) + (d > c);
+    const int rd = (a >= d) + (b >= d) + (c >= d);
+    const uint32_t nib = (ra < 2 ? 1u : 0u) | (rb < 2 ? 2u : 0u) | (rc < 2 ? 4u : 0u) | (rd < 2 ? 8u : 0u);
+    bm[j >> 3] |= nib << (4 * (j & 7));
+  }
+}
+
+// One warp 2:4-prunes and compresses one 128-channel vector (layout as warp_compress_vector:
+// lane l holds channels l, l+32, l+64, l+96; a group's four channels sit in lanes 4m..4m+3).
+__device__ __forceinline__ void warp_compress_vector_24(const uint16_t *src, uint32_t *bm_dst, uint16_t *val_dst,
+                                                        int lane) {
+  uint32_t raw[kWords], bm[kWords];
+  const int i = lane & 3, g0 = lane & ~3;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    raw[w] = src[32 * w + lane];
+    const uint32_t key = raw[w] & 0x7FFFu;
+    int rank = 0;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t km = __shfl_sync(0xffffffffu, key, g0 + m);
+      rank += (m != i) && (km > key || (km == key && m < i));
+    }
+    bm[w] = __ballot_sync(0xffffffffu, rank < 2);
+  }
+  if (lane < kWords) bm_dst[lane] = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
+  const uint32_t below = (1u << lane) - 1u;
+  int prefix = 0;
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    if ((bm[w] >> lane) & 1u) val_dst[prefix + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[w]);
+    prefix += __popc(bm[w]);
+  }
+}
+
 }  // namespace mustafar

@@ -59,13 +59,14 @@ def fits(B, Hkv, L, s, free_bytes):
     return dense + comp + (2 << 30) < free_bytes
 
 
-def decode_point(timer, peak, Hq, Hkv, B, L, sK, sV, seed, with_dense=True):
+def decode_point(timer, peak, Hq, Hkv, B, L, sK, sV, seed, with_dense=True, pattern="topk"):
     dev = "cuda"
     cap = ((L + 63) // 64) * 64
     K = synth.keys(B, Hkv, L, D, seed, dev, capacity=cap)
     V = synth.values(B, Hkv, L, D, seed, dev, capacity=cap)
     q = synth.queries(B, Hq, D, seed, dev)
-    kc, vc = M.CompressedCache(B, Hkv, cap, sK), M.CompressedCache(B, Hkv, cap, sV)
+    kc = M.CompressedCache(B, Hkv, cap, sK, pattern=pattern)
+    vc = M.CompressedCache(B, Hkv, cap, sV, pattern=pattern)
     M.mustafar_compress(K, L, sK if kc.sparsity is not None else 0.0, kc)  # per-head caches ignore it
     M.mustafar_compress(V, L, sV if vc.sparsity is not None else 0.0, vc)
     seq = torch.full((B,), L, dtype=torch.int32, device=dev)
@@ -74,7 +75,8 @@ def decode_point(timer, peak, Hq, Hkv, B, L, sK, sV, seed, with_dense=True):
     ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, L), dtype=torch.uint8, device=dev)
     t_sparse = timer.median_us(lambda: M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0, out=out, lse=lse, workspace=ws))
     nb = decode_bytes(B, Hq, Hkv, L, kc.head_keep, vc.head_keep)
-    rec = {"kind": "decode", "q_heads": Hq, "kv_heads": Hkv, "batch": B, "context": L, "sparsity_k": sK,
+    rec = {"kind": "decode", "pattern": pattern, "q_heads": Hq, "kv_heads": Hkv, "batch": B, "context": L,
+           "sparsity_k": sK,
            "sparsity_v": sV, "keep_k": kc.head_keep if kc.per_head else kc.keep,
            "keep_v": vc.head_keep if vc.per_head else vc.keep,
            "splits": M.mustafar_decode_plan_splits(B, Hkv, L, kc.keep, vc.keep),
@@ -110,7 +112,7 @@ def compress_point(timer, peak, B, L, H, s, seed):
     return rec
 
 
-def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "sweep"), log=print):
+def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "p24", "sweep"), log=print):
     torch.cuda.set_device(0)
     timer = Timer("cuda")
     recs = []
@@ -135,6 +137,13 @@ def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "sweep"), 
                   workload="b8 ctx4096 per-head sparsity (mean 0.7)"))
         emit(dict(decode_point(timer, peak, 32, 8, 8, 4096, 0.7, 0.7, 1006, with_dense=False),
                   workload="b8 ctx4096 uniform 0.7 (same inputs)"))
+    if "p24" in which:
+        # the 2:4 comparison pattern against unstructured pruning at the same sparsity (0.5) and dense
+        for B, L in ((8, 4096), (4, 32768)):
+            emit(dict(decode_point(timer, peak, 32, 8, B, L, 0.5, 0.5, 1008, pattern="2:4"),
+                      workload=f"b{B} ctx{L} 2:4"))
+            emit(dict(decode_point(timer, peak, 32, 8, B, L, 0.5, 0.5, 1008, with_dense=False),
+                      workload=f"b{B} ctx{L} unstructured s0.5 (same inputs)"))
     if "sweep" in which:
         for Hkv in (8, 32):
             for B in (1, 8, 32):

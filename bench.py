@@ -488,7 +488,7 @@ def main(argv=None):
             "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "traffic": recorded_traffic(),
-                         "kernel": "decode_kernel (sparse, fused append)", "algorithmic_bytes_per_launch": avg_bytes,
+                         "kernel": "sparse_decode_kernel (fused append)", "algorithmic_bytes_per_launch": avg_bytes,
                          "us_per_launch": us_per_step * world, "splits": wl.splits},
             "separate_launches": {"us_per_step": extra_us["separate"], "attend_us_per_launch": att_us,
                                   "attend_frac": avg_bytes / (att_us * 1e-6) / 1e9 / peak,

@@ -240,7 +240,7 @@ int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t
     return plan.splits;
   }
   // the sparse kernel cuts the end-to-end chunk sequence into CTA ranges; report the CTAs per stream
-  if (plan_sparse(batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, false, &plan) != cudaSuccess) return -1;
+  if (plan_sparse(batch, num_kv_heads, 4, max_len, keep_k, keep_v, 0, 0, &plan) != cudaSuccess) return -1;
   const int streams = batch * num_kv_heads;
   return (plan.splits + streams - 1) / streams;
 }
@@ -250,7 +250,8 @@ namespace {
 mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *workspace, size_t workspace_bytes,
                            const char *name, cudaStream_t stream) {
   DecodePlan plan;
-  cudaError_t e = plan_sparse(p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, p.perhead != 0, &plan);
+  const int variant = p.perhead ? 1 : (p.p24_k && p.p24_v ? 2 : 0);
+  cudaError_t e = plan_sparse(p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, variant, &plan);
   if (e != cudaSuccess) return cuda_fail(e, name);
   p.stage_bytes = plan.stage_bytes;
   p.warp_bytes = plan.warp_bytes;

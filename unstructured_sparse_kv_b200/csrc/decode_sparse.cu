@@ -174,10 +174,10 @@ __device__ __forceinline__ void load_q(const DecodeParams &P, int b, int g, int 
 // One 16-token chunk staged at `stage` ([K bitmap rows 16x16 B][V bitmap rows][K values 16*kK]
 // [V values 16*kV]); tokens t0 .. t0+15 of a row of length L.  `htab` is the warp's 512-byte
 // per-row half-word prefix table.
-template <bool HIROWS, bool PERHEAD>
+template <bool HIROWS, bool PERHEAD, bool P24>
 __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *stage, uint8_t *htab, uint32_t za,
                                               int t0, int L, int kKh, int kVh, int lane, const uint32_t (&qa)[8][4],
-                                              Acc<HIROWS> &acc) {
+                                              Acc<HIROWS> &acc, const uint2 *lut24) {
   // keep counts of this stream; a uniform cache reads them from the kernel parameters here, so that
   // they hold no register across the chunk loop
   const int kK = PERHEAD ? kKh : P.keep_k, kV = PERHEAD ? kVh : P.keep_v;
@@ -192,12 +192,14 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
       w = make_uint4(0u, 0u, 0u, 0u);
       *row = w;
     }
-    const uint32_t h0 = __popc(w.x & 0xFFFFu), c0 = __popc(w.x);
-    const uint32_t h1 = c0 + __popc(w.y & 0xFFFFu), c1 = c0 + __popc(w.y);
-    const uint32_t h2 = c1 + __popc(w.z & 0xFFFFu), c2 = c1 + __popc(w.z);
-    const uint32_t h3 = c2 + __popc(w.w & 0xFFFFu);
-    *reinterpret_cast<uint4 *>(htab + lane * 16) =
-        make_uint4(h0 << 16, c0 | (h1 << 16), c1 | (h2 << 16), c2 | (h3 << 16));
+    if constexpr (!P24) {  // 2:4 runs need no prefixes: every word holds 16 values, every nibble 2
+      const uint32_t h0 = __popc(w.x & 0xFFFFu), c0 = __popc(w.x);
+      const uint32_t h1 = c0 + __popc(w.y & 0xFFFFu), c1 = c0 + __popc(w.y);
+      const uint32_t h2 = c1 + __popc(w.z & 0xFFFFu), c2 = c1 + __popc(w.z);
+      const uint32_t h3 = c2 + __popc(w.w & 0xFFFFu);
+      *reinterpret_cast<uint4 *>(htab + lane * 16) =
+          make_uint4(h0 << 16, c0 | (h1 << 16), c1 | (h2 << 16), c2 | (h3 << 16));
+    }
   }
   __syncwarp();
 
@@ -209,10 +211,24 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
     s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
     const int T = gq + 8 * nt;  // this lane's token (the fragment's n index) in n-tile nt
     const uint32_t word = *reinterpret_cast<const uint32_t *>(stage + T * 16 + qq * 4);
-    const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
-    const uint32_t rbase = kvals + 2 * T * kK;
     uint32_t kb[16];
-    expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
+    if constexpr (P24) {
+      // word qq's 16 values: 32 contiguous bytes of the token's 128-byte run, nibble j's two in value
+      // pair j; placed into channel pairs (4j, 4j+1), (4j+2, 4j+3) by the nibble's two selectors
+      const uint4 va = *reinterpret_cast<const uint4 *>(stage + 512 + T * 128 + qq * 32);
+      const uint4 vb = *reinterpret_cast<const uint4 *>(stage + 512 + T * 128 + qq * 32 + 16);
+      const uint32_t x[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint2 sel = lut24[(word >> (4 * j)) & 15u];
+        kb[2 * j] = __byte_perm(x[j], 0u, sel.x);
+        kb[2 * j + 1] = __byte_perm(x[j], 0u, sel.y);
+      }
+    } else {
+      const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
+      const uint32_t rbase = kvals + 2 * T * kK;
+      expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
+    }
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) mma_f16_16816(s[nt], qa[ks], kb[2 * ks], kb[2 * ks + 1]);
   }
@@ -286,20 +302,46 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
   // 16g..16g+15 (half word g of the bitmap) of tokens 2q, 2q+1 and 2q+8, 2q+9.
   const uint32_t vvals = smem_addr(stage + 512 + 32 * kK);
   uint32_t va[8][4];
+  if constexpr (P24) {
+    // half word gq of each token: 8 values, 16 contiguous bytes at 16*gq in the token's run
 #pragma unroll
-  for (int pair = 0; pair < 2; ++pair) {
-    uint32_t x0[16], x1[16];
+    for (int pair = 0; pair < 2; ++pair) {
+      uint32_t y[2][8];  // [token of the pair][channel pair 16g + 2i, +1]
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int T = 2 * qq + 8 * pair + e;
-      const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
-      const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
-      expand_half(bits, vvals + 2 * (T * kV + pre), za, e ? x1 : x0);
+      for (int e = 0; e < 2; ++e) {
+        const int T = 2 * qq + 8 * pair + e;
+        const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + 512 + 2048 + T * 128 + gq * 16);
+        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint2 sel = lut24[(bits >> (4 * m)) & 15u];
+          y[e][2 * m] = __byte_perm(x[m], 0u, sel.x);
+          y[e][2 * m + 1] = __byte_perm(x[m], 0u, sel.y);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        va[mt][2 * pair] = __byte_perm(y[0][mt], y[1][mt], 0x5410);
+        va[mt][2 * pair + 1] = __byte_perm(y[0][mt], y[1][mt], 0x7632);
+      }
     }
+  } else {
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      va[mt][2 * pair] = __byte_perm(x0[2 * mt], x1[2 * mt], 0x5410);
-      va[mt][2 * pair + 1] = __byte_perm(x0[2 * mt + 1], x1[2 * mt + 1], 0x5410);
+    for (int pair = 0; pair < 2; ++pair) {
+      uint32_t x0[16], x1[16];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int T = 2 * qq + 8 * pair + e;
+        const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
+        const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
+        expand_half(bits, vvals + 2 * (T * kV + pre), za, e ? x1 : x0);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        va[mt][2 * pair] = __byte_perm(x0[2 * mt], x1[2 * mt], 0x5410);
+        va[mt][2 * pair + 1] = __byte_perm(x0[2 * mt + 1], x1[2 * mt + 1], 0x5410);
+      }
     }
   }
 #pragma unroll
@@ -496,13 +538,23 @@ __device__ __forceinline__ int64_t base_of(const HeadKeep &hk, int keep, int b, 
   return PERHEAD ? hk.value_base(b, h, H, cap) : (static_cast<int64_t>(b) * H + h) * cap * static_cast<int64_t>(keep);
 }
 
-template <int NSTAGE, bool HIROWS, bool PERHEAD>
+// PRMT selectors that place a 2:4 nibble's two values (one 32-bit pair, lower channel first) at
+// their channels: .x builds channels (0, 1), .y channels (2, 3); bytes 4-7 are the zero operand.
+// Index = the nibble's 4 bits; the six 2-of-4 patterns, and 0 (a masked tail token) -> zeros.
+__constant__ uint2 kLut24[16] = {
+    {0x5454u, 0x5454u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}, {0x3210u, 0x5454u},  // 0, 1, 2, 0011
+    {0x5454u, 0x5454u}, {0x5410u, 0x5432u}, {0x1054u, 0x5432u}, {0x5454u, 0x5454u},  // 4, 0101, 0110, 7
+    {0x5454u, 0x5454u}, {0x5410u, 0x3254u}, {0x1054u, 0x3254u}, {0x5454u, 0x5454u},  // 8, 1001, 1010, 11
+    {0x5454u, 0x3210u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}};  // 1100, 13, 14, 15
+
+template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24>
 __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
   __shared__ int sh_info[3];  // U, batch row of this CTA's first unit (-1: none), that row's first unit
   __shared__ Pending sh_pend[2];
   __shared__ int sh_npend, sh_last[2];
+  __shared__ uint2 lut24[16];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x, nctas = gridDim.x;
   const int cap = min(P.cap_k, P.cap_v);
@@ -555,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   }
   if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
   if (threadIdx.x == 0) sh_npend = 0;
+  if (P24 && threadIdx.x < 16) lut24[threadIdx.x] = kLut24[threadIdx.x];
   uint8_t *wbase = smem + warp * P.warp_bytes;
   uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // [32 rows][8 half words] u16 prefixes
   const uint32_t bars = smem_addr(htab + 512);     // NSTAGE mbarriers of this warp
@@ -685,7 +738,8 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       uint8_t *stage = wbase + slot * P.stage_bytes;
       if (!mbar_wait(bars + 8 * slot, (citem / NSTAGE) & 1, timed_out ? kWaitCyclesAfter : kWaitCycles))
         timed_out = true;
-      consume_chunk<HIROWS, PERHEAD>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc);
+      consume_chunk<HIROWS, PERHEAD, P24>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
+                                          lut24);
       __syncwarp();
       produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
     }
@@ -718,25 +772,32 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
 // ------------------------------------------------------------------------------------ host side
 using SparseFn = void (*)(const DecodeParams);
 
-template <int NSTAGE, bool PERHEAD>
+template <int NSTAGE, bool PERHEAD, bool P24>
 SparseFn pick_rows(bool hirows) {
-  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD> : sparse_decode_kernel<NSTAGE, false, PERHEAD>;
+  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD, P24> : sparse_decode_kernel<NSTAGE, false, PERHEAD, P24>;
 }
 
-template <bool PERHEAD>
+template <bool PERHEAD, bool P24>
 SparseFn pick_stages(int nstage, bool hirows) {
   switch (nstage) {
-    case 2: return pick_rows<2, PERHEAD>(hirows);
-    case 3: return pick_rows<3, PERHEAD>(hirows);
-    default: return pick_rows<4, PERHEAD>(hirows);
+    case 2: return pick_rows<2, PERHEAD, P24>(hirows);
+    case 3: return pick_rows<3, PERHEAD, P24>(hirows);
+    default: return pick_rows<4, PERHEAD, P24>(hirows);
   }
 }
 
-SparseFn pick_sparse(int nstage, bool hirows, bool perhead) {
-  return perhead ? pick_stages<true>(nstage, hirows) : pick_stages<false>(nstage, hirows);
+// variant: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4
+SparseFn pick_sparse(int nstage, bool hirows, int variant) {
+  switch (variant) {
+    case 1: return pick_stages<true, false>(nstage, hirows);
+    case 2: return pick_stages<false, true>(nstage, hirows);
+    default: return pick_stages<false, false>(nstage, hirows);
+  }
 }
 
-int sparse_slot(int nstage, bool hirows, bool perhead) { return 12 + 2 * nstage + (hirows ? 1 : 0) + (perhead ? 10 : 0); }
+// ensure_smem_limit / occupancy cache slots 12..29, one per kernel (compress and the dense kernel
+// use 0..9)
+int sparse_slot(int nstage, bool hirows, int variant) { return 12 + 6 * variant + 2 * (nstage - 2) + (hirows ? 1 : 0); }
 
 constexpr int kMinUnitsPerCta = 2 * kWarps;  // at least two chunks per warp
 constexpr int kMaxCtasPerSm = 4;
@@ -806,7 +867,7 @@ size_t sparse_workspace_bound(int B, int Hkv, int G, int max_len, int forced_spl
   return sparse_workspace_bytes(B, Hkv, G, sparse_decode_ctas(B, Hkv, max_len, forced_splits, kMaxCtasPerSm));
 }
 
-cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, bool perhead,
+cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, int variant,
                         DecodePlan *plan) {
   const bool hirows = G > 8;
   const int stage_bytes = round_up(512 + 32 * (keep_k + keep_v), 128);
@@ -820,8 +881,8 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
     }
   const int warp_bytes = warp_bytes_of(nstage);
   const int smem = kWarps * warp_bytes + merge_bytes;
-  SparseFn fn = pick_sparse(nstage, hirows, perhead);
-  const int slot = sparse_slot(nstage, hirows, perhead);
+  SparseFn fn = pick_sparse(nstage, hirows, variant);
+  const int slot = sparse_slot(nstage, hirows, variant);
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(fn), slot, smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
@@ -834,12 +895,12 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
   plan->stage_bytes = stage_bytes;
   plan->warp_bytes = warp_bytes;
   plan->smem_bytes = smem;
-  plan->perhead = perhead;
+  plan->variant = variant;
   return cudaSuccess;
 }
 
 cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
-  SparseFn fn = pick_sparse(plan.nstage, p.G > 8, plan.perhead);
+  SparseFn fn = pick_sparse(plan.nstage, p.G > 8, plan.variant);
   fn<<<plan.splits, kThreads, plan.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }

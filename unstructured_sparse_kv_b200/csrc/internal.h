@@ -77,7 +77,7 @@ struct DecodePlan {
   int stage_bytes;
   int warp_bytes;
   int smem_bytes;
-  bool perhead;  // sparse kernel: a cache with a keep count per kv head
+  int variant;  // sparse kernel: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4
 };
 
 // Dense fp16 baseline: plan (split count, pipeline depth, shared memory) and launch.
@@ -88,7 +88,8 @@ cudaError_t launch_dense(const DecodeParams &p, const DecodePlan &plan, cudaStre
 
 // Sparse decode over the compressed caches (one wave of CTAs over the end-to-end chunk sequence):
 // plan->splits holds the CTA count.
-cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, bool perhead,
+// variant: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4
+cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, int variant,
                         DecodePlan *plan);
 cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);
 int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_sm);

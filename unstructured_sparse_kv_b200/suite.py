@@ -3,7 +3,7 @@
 Each record is one JSON object: the shape, the sparse decode-attention time per launch, its
 algorithmic bytes and GB/s as a fraction of the HBM peak, the dense fp16 baseline on the same
 inputs, or the compress kernel's throughput and compressed size.  Times are the median of
-CUDA-event-timed launches with the 126 MB L2 flushed (a 256 MiB write) before each launch.
+CUDA-event-timed launches with the 126 MB L2 flushed (a 256 MiB read) before each launch.
 """
 from __future__ import annotations
 
@@ -21,15 +21,18 @@ FLUSH_BYTES = 256 << 20
 
 
 class Timer:
+    """Median of single launches, each after a read of a buffer larger than L2.  The flush only
+    reads (its lines stay clean), so the timed launch pays no write-back of flush data."""
+
     def __init__(self, device):
-        self.flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
 
     def median_us(self, fn, reps: int = 15, warmup: int = 3) -> float:
         for _ in range(warmup):
             fn()
         times = []
         for _ in range(reps):
-            self.flush.fill_(1)
+            torch.amax(self.flush)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             fn()

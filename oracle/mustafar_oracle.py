@@ -14,6 +14,9 @@ What it computes, and from which passage:
   positions, the kept fp16 values are packed, and per-tile offsets locate them.
   The pages give no layout; this oracle follows the library's own choices, which
   are written out in ``keep_count``, ``compress`` and ``compressed_bytes`` below.
+* Channel-wise magnitude pruning, the other pruning direction the README names
+  (Part II, the K/V [t/c] naming): each channel is pruned across the tokens of
+  16-token windows; the readings it takes are written out above ``WINDOW`` below.
 * Decode attention over the pruned caches (the abstract: the kernel computes
   "directly over compressed caches"): the exact result it must reach is plain
   softmax attention over the pruned K and V, computed here in float64.
@@ -309,6 +312,132 @@ def append_heads(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
             cache["bitmap"][b, h, p] = words[b]
             base = value_base_heads(b, h, hk, cap) + p * k
             cache["values"][base:base + k] = x[b, h][mask[b]]
+
+
+# --------------------------------------------------------------------------------------
+# channel-wise magnitude pruning (the Kc_Mag / Vc_Mag direction)
+# --------------------------------------------------------------------------------------
+# The README (Part II, the K/V [t/c] naming) names a channel-wise pruning direction next to the
+# token-wise one and says no more.  Reading: each channel of a kv head is pruned across tokens,
+# over consecutive windows of WINDOW tokens counted from token 0.  A full window prunes
+# F = floor(s*WINDOW) of its tokens per channel (s as a float32, product in double, as in
+# ``keep_count``) and keeps the WINDOW - F of largest magnitude (same key; ties go to the lower
+# token index); a window of n < WINDOW tokens (the newest tokens of a row) prunes floor(n*F/WINDOW).
+# Storage reuses the token bitmap format: bit c of token t marks a kept (t, c); the kept values of
+# a window are packed token after token, each token's in ascending channel order, and window j of
+# a stream starts at element j*WINDOW*keep, keep = (d/WINDOW)*(WINDOW - F) being the stream's values
+# per token slot (so tile i of 64 tokens starts at 64*i*keep, as in the token format).  A dense copy
+# of each stream's last, incomplete window is kept beside the cache, because an appended token
+# changes which of that window's entries are kept.
+WINDOW = 16
+
+
+def window_prune_count(sparsity: float) -> int:
+    """F = floor(s * WINDOW): tokens a full window prunes in every channel."""
+    s = float(np.float32(sparsity))
+    if not (0.0 <= s < 1.0):
+        raise ValueError("sparsity must lie in [0, 1)")
+    return int(math.floor(s * WINDOW))
+
+
+def window_keep(n: int, F: int) -> int:
+    """Tokens a window of n tokens keeps in every channel: n - floor(n*F/WINDOW)."""
+    return n - (n * F) // WINDOW
+
+
+def keep_count_channel(d: int, sparsity: float) -> int:
+    """Values per token slot of a channel-wise cache: (d/WINDOW) * (WINDOW - F)."""
+    return (d // WINDOW) * (WINDOW - window_prune_count(sparsity))
+
+
+def select_channel(x_bits: np.ndarray, F: int) -> np.ndarray:
+    """Kept-mask of channel-wise pruning of [..., T, d]: in every window of tokens, every channel
+    keeps its ``window_keep(n, F)`` largest keys, the lower token first on ties."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    T = x.shape[-2]
+    mask = np.zeros(x.shape, dtype=bool)
+    for t0 in range(0, T, WINDOW):
+        n = min(WINDOW, T - t0)
+        win = np.swapaxes(x[..., t0:t0 + n, :], -1, -2)  # [..., d, n]: a channel's tokens on the last axis
+        mask[..., t0:t0 + n, :] = np.swapaxes(select_sort(win, window_keep(n, F)), -1, -2)
+    return mask
+
+
+def prune_channel(x_bits: np.ndarray, sparsity: float) -> np.ndarray:
+    """Channel-wise pruned fp16 bits of [..., T, d] (pruned entries become +0)."""
+    x = np.asarray(x_bits, dtype=np.uint16)
+    return np.where(select_channel(x, window_prune_count(sparsity)), x, np.uint16(0)).astype(np.uint16)
+
+
+def compress_channel(x_bits: np.ndarray, sparsity: float, capacity: int, L: int | None = None) -> dict:
+    """Channel-wise pruned tokens [0, L) of a dense cache [B, H, T, d] in the bitmap format.
+
+    ``bitmap`` [B, H, capacity, d/32] and ``tile_offset`` [B, H, capacity/64] (= 64*i*keep) as in
+    ``compress``; ``values`` [B, H, capacity*keep] with window j at element j*WINDOW*keep;
+    ``window`` [B, H, WINDOW, d]: tokens [WINDOW*floor(L/WINDOW), L) in slots 0.. (the rest zero).
+    """
+    x = np.asarray(x_bits, dtype=np.uint16)
+    B, H, T, d = x.shape
+    L = T if L is None else L
+    assert capacity % TILE_TOKENS == 0 and L <= capacity and L <= T
+    F = window_prune_count(sparsity)
+    keep = keep_count_channel(d, sparsity)
+    mask = select_channel(x[:, :, :L], F)
+    bitmap = np.zeros((B, H, capacity, d // WORD_BITS), dtype=np.uint32)
+    bitmap[:, :, :L] = bitmap_words(mask)
+    values = np.zeros((B, H, capacity * keep), dtype=np.uint16)
+    for b in range(B):
+        for h in range(H):
+            for t0 in range(0, L, WINDOW):
+                n = min(WINDOW, L - t0)
+                kept = x[b, h, t0:t0 + n][mask[b, h, t0:t0 + n]]  # token-major, channels ascending
+                values[b, h, t0 * keep:t0 * keep + kept.size] = kept
+    tile_offset = np.broadcast_to(np.arange(capacity // TILE_TOKENS, dtype=np.int64) * TILE_TOKENS * keep,
+                                  (B, H, capacity // TILE_TOKENS)).astype(np.uint32)
+    window = np.zeros((B, H, WINDOW, d), dtype=np.uint16)
+    r = L % WINDOW
+    window[:, :, :r] = x[:, :, L - r:L]
+    return {"bitmap": bitmap, "values": values, "tile_offset": tile_offset, "window": window, "F": F,
+            "keep": keep, "L": L}
+
+
+def decompress_channel(cache: dict, L: int, d: int) -> np.ndarray:
+    """Dense fp16 bits [B, H, L, d] rebuilt from a channel-wise cache (pruned positions are +0)."""
+    mask = bitmap_to_mask(cache["bitmap"][:, :, :L], d)
+    B, H = mask.shape[:2]
+    keep = cache["keep"]
+    out = np.zeros((B, H, L, d), dtype=np.uint16)
+    for b in range(B):
+        for h in range(H):
+            for t0 in range(0, L, WINDOW):
+                m = mask[b, h, t0:t0 + WINDOW]
+                cnt = int(m.sum())
+                blk = np.zeros(m.shape, dtype=np.uint16)
+                blk[m] = cache["values"][b, h, t0 * keep:t0 * keep + cnt]
+                out[b, h, t0:t0 + m.shape[0]] = blk
+    return out
+
+
+def append_channel(cache: dict, x_new_bits: np.ndarray, pos: np.ndarray) -> None:
+    """Append one new token per (b, h) at slot pos[b] of a channel-wise cache (in place).
+
+    The token joins its window's dense copy; the window (tokens WINDOW*floor(p/WINDOW) .. p) is
+    pruned again as a window of p % WINDOW + 1 tokens, and its bitmaps and packed values are
+    rewritten.  Appends must come in token order.
+    """
+    x = np.asarray(x_new_bits, dtype=np.uint16)  # [B, H, d]
+    B, H, d = x.shape
+    F, keep = cache["F"], cache["keep"]
+    for b in range(B):
+        p = int(pos[b])
+        t0, r = p - p % WINDOW, p % WINDOW
+        cache["window"][b, :, r] = x[b]
+        dense = cache["window"][b, :, :r + 1]  # [H, r+1, d]
+        mask = select_channel(dense, F)
+        cache["bitmap"][b, :, t0:p + 1] = bitmap_words(mask)
+        for h in range(H):
+            kept = dense[h][mask[h]]
+            cache["values"][b, h, t0 * keep:t0 * keep + kept.size] = kept
 
 
 # --------------------------------------------------------------------------------------

@@ -17,6 +17,10 @@ oracle disagrees with the fact it checks.  Facts used:
   per head; round trip to the per-head pruned cache; append == compress.
 * 2:4 pattern: a hand-derived 32-channel fixture (selection, bitmap word, packed values);
   exactly 2 of every 4 channels; brute-force ranks per group; round trip; append == compress.
+* channel-wise direction: a hand-derived fixture (window counts, a partial window with ties, a
+  full window with a tie at the keep boundary); counts and pairwise dominance per (window,
+  channel); a full window equals brute-force token ranks of the transposed window; the window
+  slots and the round trip; sparsity 0 equals the token format with k = d; append == compress.
 """
 from __future__ import annotations
 
@@ -342,10 +346,130 @@ def pin_24_structure(O):
         assert np.array_equal(comp[key], part[key]), key
 
 
+# ----------------------------------------------------------------------------- channel-wise direction
+def _channel_partial_fixture():
+    g = _load("select_channel.json")["partial_window"]
+    x = np.zeros((1, 1, 4, 32), dtype=np.uint16)
+    for t in range(4):
+        for c in range(32):
+            x[0, 0, t, c] = int(g["x_hex_by_token_and_class"][t][c % 4], 16)
+    return x, g
+
+
+def pin_golden_channel(O):
+    g = _load("select_channel.json")
+    for case in g["window_counts"]["cases"]:
+        F = O.window_prune_count(case["s"])
+        assert F == case["F"], case
+        assert O.window_keep(case["n"], F) == case["window_keep"], case
+    for case in g["window_counts"]["keep_count_channel"]:
+        assert O.keep_count_channel(case["d"], case["s"]) == case["keep"], case
+    # a partial window: selection with ties, bitmap words, token-major packing, the dense copy
+    x, p = _channel_partial_fixture()
+    c = O.compress_channel(x, p["s"], 64)
+    assert [int(w) for w in c["bitmap"][0, 0, :4, 0]] == [int(h, 16) for h in p["bitmap_words_hex"]]
+    expect = []
+    for t, grp in enumerate(p["packed_values_hex_per_token_group"]):
+        assert 8 * len(grp) == p["values_per_token"][t]
+        expect += [int(h, 16) for h in grp] * 8
+    assert c["values"][0, 0, :64].tolist() == expect
+    assert not c["values"][0, 0, 64:].any()
+    assert np.array_equal(c["window"][0, 0, :4], x[0, 0])
+    # a full window: the tie at the keep boundary goes to the lower token
+    f = g["full_window"]
+    t = np.arange(16)
+    col = np.where(t % 2 == 1, -(t % 5), t % 5).astype(np.float16).view(np.uint16)
+    xf = np.repeat(col[:, None], 32, axis=1)[None, None]
+    cf = O.compress_channel(xf, f["s"], 64)
+    assert cf["keep"] == f["keep"]
+    words = cf["bitmap"][0, 0, :16, 0]
+    assert np.flatnonzero(words).tolist() == f["kept_tokens"]
+    assert all(int(words[i]) == 0xFFFFFFFF for i in f["kept_tokens"])
+    assert cf["values"][0, 0, :16 * f["keep"]].tolist() == sum([[int(h, 16)] * 32 for h in f["kept_value_hex"]], [])
+    assert not cf["window"].any()  # 16 tokens: no incomplete window
+
+
+def pin_channel_selection_rules(O):
+    """Counts per (window, channel) and the dominance rule, by brute force over token pairs."""
+    rng = np.random.default_rng(31)
+    for s in (0.7, 0.5, 0.3, 0.9375, 0.0):
+        F = O.window_prune_count(s)
+        for T, ties in ((16, False), (37, True), (5, True)):
+            x = rand_bits(rng, (2, T, 8), tie_heavy=ties)
+            mask = O.select_channel(x, F)
+            m = O.magnitude_key(x)
+            for t0 in range(0, T, 16):
+                n = min(16, T - t0)
+                for b in range(2):
+                    for c in range(8):
+                        kept = [t0 + i for i in range(n) if mask[b, t0 + i, c]]
+                        drop = [t0 + i for i in range(n) if not mask[b, t0 + i, c]]
+                        assert len(kept) == O.window_keep(n, F)
+                        for i in kept:
+                            for j in drop:
+                                assert m[b, i, c] > m[b, j, c] or (m[b, i, c] == m[b, j, c] and i < j)
+        # a full window is a token-wise selection of the transposed window (brute-force ranks)
+        x = rand_bits(rng, (3, 16, 8), tie_heavy=True)
+        assert np.array_equal(np.swapaxes(O.select_channel(x, F), -1, -2),
+                              O.select_rank_bruteforce(np.swapaxes(x, -1, -2), 16 - F))
+
+
+def pin_channel_layout_roundtrip(O):
+    rng = np.random.default_rng(37)
+    B, H, L, d, cap = 2, 3, 70, 128, 128
+    x = rand_bits(rng, (B, H, L, d))
+    x[1, 2, 40:56] = rand_bits(rng, (16, d), tie_heavy=True)
+    for s in (0.7, 0.3):
+        F = O.window_prune_count(s)
+        c = O.compress_channel(x, s, cap)
+        keep = c["keep"]
+        assert keep * 16 == d * (16 - F)
+        dec = O.decompress_channel(c, L, d)
+        assert np.array_equal(dec, O.prune_channel(x, s))
+        # every window's values fill its slot from the start: a full window exactly, the last one
+        # d * window_keep(n) of its 16 * keep
+        bits = O.bitmap_to_mask(c["bitmap"][:, :, :L], d)
+        for t0 in range(0, L, 16):
+            n = min(16, L - t0)
+            per_ch = bits[:, :, t0:t0 + n].sum(axis=2)
+            assert (per_ch == O.window_keep(n, F)).all()
+            used = d * O.window_keep(n, F)
+            assert used <= 16 * keep and (n < 16 or used == 16 * keep)
+            # the packed run is exactly the window's kept entries, token by token
+            for b in range(B):
+                for h in range(H):
+                    assert np.array_equal(c["values"][b, h, t0 * keep:t0 * keep + used],
+                                          x[b, h, t0:t0 + n][bits[b, h, t0:t0 + n]])
+        assert all(int(c["tile_offset"][b, h, i]) == 64 * i * keep
+                   for b in range(B) for h in range(H) for i in range(cap // 64))
+        assert np.array_equal(c["window"][:, :, :L % 16], x[:, :, L - L % 16:L])
+    # nothing pruned: the channel-wise cache is the token format with k = d, byte for byte
+    c0, t0c = O.compress_channel(x, 0.0, cap), O.compress(x, d, cap)
+    for key in ("bitmap", "values", "tile_offset"):
+        assert np.array_equal(c0[key], t0c[key]), key
+
+
+def pin_channel_append_equals_compress(O):
+    rng = np.random.default_rng(41)
+    B, H, d, cap = 2, 2, 128, 128
+    x = rand_bits(rng, (B, H, 70, d))
+    for s, L0 in ((0.7, 37), (0.5, 16), (0.3, 0)):
+        part = O.compress_channel(x, s, cap, L0)
+        for p in range(L0, 70):  # crosses the window edges at 48 and 64
+            O.append_channel(part, x[:, :, p], np.full(B, p))
+            if p in (47, 50, 69):
+                full = O.compress_channel(x, s, cap, p + 1)
+                for key in ("bitmap", "values", "tile_offset"):
+                    assert np.array_equal(full[key], part[key]), (s, p, key)
+                r = (p + 1) % 16
+                assert np.array_equal(full["window"][:, :, :r], part["window"][:, :, :r])
+
+
 ALL_PINS = [pin_golden_selection, pin_golden_keep_count, pin_bruteforce_selection, pin_threshold_invariant,
             pin_roundtrip_and_popcount, pin_compressed_size, pin_dense_limit_sdpa, pin_golden_attention,
             pin_attention_invariants, pin_append_equals_compress, pin_heads_layout, pin_heads_append_equals_compress,
-            pin_golden_24, pin_24_structure]
+            pin_golden_24, pin_24_structure, pin_golden_channel, pin_channel_selection_rules,
+            pin_channel_layout_roundtrip, pin_channel_append_equals_compress]
 
 
 def failing_pins(O):

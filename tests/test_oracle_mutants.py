@@ -2,6 +2,7 @@
 
 Mistakes are planted in the oracle only, on the CPU.
 """
+import builtins
 import types
 
 import numpy as np
@@ -138,6 +139,14 @@ def _mutant(**overrides):
                 v = x[b, h][mask[b, h]]
                 cache["values"][b, h, p * k:p * k + v.size] = v[:k]
     ns.append_24 = append_24
+    # channel-wise functions: the real code, its global names looked up in the namespace
+    glb = vars(ns)
+    glb["__builtins__"] = builtins
+    for name in ("window_prune_count", "window_keep", "keep_count_channel", "select_channel", "prune_channel",
+                 "compress_channel", "decompress_channel", "append_channel"):
+        if name not in overrides:
+            fn = getattr(real, name)
+            setattr(ns, name, types.FunctionType(fn.__code__, glb, name, fn.__defaults__))
     return ns
 
 
@@ -234,7 +243,91 @@ def sel24_groups_of_8(x_bits):         # 4 of every 8 instead of 2 of every 4
     return real.select_sort(x.reshape(x.shape[:-1] + (d // 8, 8)), 4).reshape(x.shape)
 
 
+def selch_high_ties(x_bits, F):          # channel-wise ties go to the later token
+    x = np.asarray(x_bits, np.uint16)
+    return real.select_channel(x[..., ::-1, :], F)[..., ::-1, :] if x.shape[-2] % 16 == 0 else \
+        _selch_windows(x, F, lambda w, k: real.select_sort(w[..., ::-1], k)[..., ::-1])
+
+
+def _selch_windows(x, F, select):
+    T = x.shape[-2]
+    mask = np.zeros(x.shape, bool)
+    for t0 in range(0, T, 16):
+        n = min(16, T - t0)
+        w = np.swapaxes(x[..., t0:t0 + n, :], -1, -2)
+        mask[..., t0:t0 + n, :] = np.swapaxes(select(w, real.window_keep(n, F)), -1, -2)
+    return mask
+
+
+def selch_from_end(x_bits, F):           # windows counted back from the newest token
+    x = np.asarray(x_bits, np.uint16)
+    return _selch_windows(x[..., ::-1, :], F, lambda w, k: real.select_sort(w[..., ::-1], k)[..., ::-1])[..., ::-1, :]
+
+
+def selch_over_channels(x_bits, F):      # prunes across the channels of a token (the token direction)
+    x = np.asarray(x_bits, np.uint16)
+    d = x.shape[-1]
+    return real.select_sort(x, d - (d * F) // 16)
+
+
+def wkeep_ceil(n, F):                    # rounds the pruned count up
+    return n - -(-n * F // 16)
+
+
+def keepch_token_rule(d, s):             # token-wise keep count instead of (d/16)*(16-F)
+    return real.keep_count(d, s)
+
+
+def compress_channel_major(x_bits, sparsity, capacity, L=None):   # a window's values channel by channel
+    c = real.compress_channel(x_bits, sparsity, capacity, L)
+    x = np.asarray(x_bits, np.uint16)
+    keep, L = c["keep"], c["L"]
+    mask = real.bitmap_to_mask(c["bitmap"][:, :, :L], x.shape[-1])
+    for b in range(x.shape[0]):
+        for h in range(x.shape[1]):
+            for t0 in range(0, L, 16):
+                xm = x[b, h, t0:t0 + 16][:L - t0].T
+                kept = xm[mask[b, h, t0:t0 + 16][:L - t0].T]
+                c["values"][b, h, t0 * keep:t0 * keep + kept.size] = kept
+    return c
+
+
+def append_channel_no_window(cache, x_new_bits, pos):   # forgets to keep the window's dense copy
+    saved = cache["window"].copy()
+    real.append_channel(cache, x_new_bits, pos)
+    x = np.asarray(x_new_bits, np.uint16)
+    for b in range(x.shape[0]):
+        p = int(pos[b])
+        cache["window"][b] = saved[b]
+        if p % 16 == 0:
+            cache["window"][b] = 0
+
+
+def append_channel_new_only(cache, x_new_bits, pos):    # prunes the new token alone, old bits kept
+    x = np.asarray(x_new_bits, np.uint16)
+    for b in range(x.shape[0]):
+        p = int(pos[b])
+        r = p % 16
+        cache["window"][b, :, r] = x[b]
+        mask = real.select_channel(cache["window"][b, :, :r + 1], cache["F"])
+        cache["bitmap"][b, :, p] = real.bitmap_words(mask[:, r])
+        t0, keep = p - r, cache["keep"]
+        for h in range(x.shape[1]):
+            old = real.bitmap_to_mask(cache["bitmap"][b, h, t0:p + 1], x.shape[-1])
+            dense = cache["window"][b, h, :r + 1]
+            kept = dense[old]
+            cache["values"][b, h, t0 * keep:t0 * keep + kept.size] = kept
+
+
 MUTANTS = {
+    "channel ties to later token": dict(select_channel=selch_high_ties),
+    "channel windows from the end": dict(select_channel=selch_from_end),
+    "channel pruned across channels": dict(select_channel=selch_over_channels),
+    "channel window count rounded up": dict(window_keep=wkeep_ceil),
+    "channel keep by the token rule": dict(keep_count_channel=keepch_token_rule),
+    "channel values channel-major": dict(compress_channel=compress_channel_major),
+    "channel append keeps no window": dict(append_channel=append_channel_no_window),
+    "channel append prunes new token only": dict(append_channel=append_channel_new_only),
     "2:4 strided groups": dict(select_24=sel24_strided),
     "2:4 as 4:8": dict(select_24=sel24_groups_of_8),
     "per-head base after own head": dict(value_base_heads=base_next_head),

@@ -37,6 +37,18 @@
  *              of each 64-token tile (the popcount prefix sum, = 64*i*k).
  *   Pruned positions read back as +0.  Bytes per stream:
  *              16*L + 2*k*L + 4*capacity/64 for L stored tokens (head_dim 128).
+ *
+ * Channel-wise caches (pattern MUSTAFAR_PATTERN_CHANNEL: the channel-wise pruning
+ * direction of the README, Part II, K/V [t/c] naming) use the same arrays with the
+ * selection turned across tokens: tokens are grouped in windows of 16 from token 0;
+ * a full window prunes F = floor(16 * sparsity) tokens of every channel and keeps
+ * the 16 - F largest magnitudes (ties: the lower token index wins); a window of
+ * n < 16 tokens (the newest ones) prunes floor(n*F/16).  keep is then
+ * (head_dim/16) * (16 - F) (mustafar_keep_count_channel): window j of a stream
+ * owns the 16*keep elements from j*16*keep, its kept values packed token after
+ * token, each token's in ascending channel order, so tokens carry varying counts.
+ * A fourth array, window (fp16 [streams][16][head_dim]), holds the dense copy of
+ * each stream's newest incomplete window, which an append prunes again.
  */
 #ifndef MUSTAFAR_H_
 #define MUSTAFAR_H_
@@ -48,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MUSTAFAR_ABI_VERSION 3
+#define MUSTAFAR_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MUSTAFAR_API __attribute__((visibility("default")))
@@ -97,15 +109,35 @@ typedef struct {
    * (ties to the lower channel), so keep must be head_dim/2 and head_keep NULL.  Both are stored in
    * the same bitmap format, and the decode calls read either. */
   int32_t pattern;
+  /* MUSTAFAR_PATTERN_CHANNEL caches only (NULL otherwise): fp16 [batch][num_kv_heads][16][head_dim],
+   * 16-byte aligned, caller-owned like the other arrays.  Slots 0 .. n-1 hold the n tokens of each
+   * stream's newest window when n < 16; mustafar_compress writes them and every append adds one. */
+  uint16_t *window;
 } mustafar_cache_t;
 
 #define MUSTAFAR_PATTERN_TOPK 0
 #define MUSTAFAR_PATTERN_2_4 1
+/* channel-wise pruning over 16-token windows; keep = mustafar_keep_count_channel(head_dim, s),
+ * head_keep NULL and window non-NULL */
+#define MUSTAFAR_PATTERN_CHANNEL 2
 
 /* Keep count for a pruning sparsity s (fraction of channels removed, README
  * Part II: a setting of 0.5 prunes half of them).  Returns head_dim - floor(s*head_dim), or -1
  * when head_dim <= 0, head_dim % 32 != 0 or s is outside [0, 1). */
 MUSTAFAR_API int32_t mustafar_keep_count(int32_t head_dim, float sparsity);
+
+/* Values per token slot of a channel-wise cache: (head_dim/16) * (16 - floor(16*s)), s rounded
+ * to float and the product formed in double.  -1 when head_dim <= 0, head_dim % 32 != 0 or s is
+ * outside [0, 1). */
+MUSTAFAR_API int32_t mustafar_keep_count_channel(int32_t head_dim, float sparsity);
+
+/* Bytes of the four arrays of a channel-wise cache (host outputs, any may be NULL): bitmap and
+ * tile_offset as mustafar_cache_sizes, values 2*streams*capacity*keep with keep from
+ * mustafar_keep_count_channel, window 2*streams*16*head_dim.  Errors: INVALID_ARG. */
+MUSTAFAR_API mustafar_status mustafar_cache_sizes_channel(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
+                                                          int32_t capacity, float sparsity, size_t *bitmap_bytes,
+                                                          size_t *values_bytes, size_t *offset_bytes,
+                                                          size_t *window_bytes);
 
 /* Bytes of the three arrays of one cache (host outputs, any may be NULL). */
 MUSTAFAR_API mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
@@ -127,8 +159,11 @@ MUSTAFAR_API mustafar_status mustafar_cache_sizes_per_head(int32_t batch, int32_
  *              channels contiguous; x and every stride a multiple of 8 elements).
  *   L        : tokens [0, L) are compressed into slots [0, L); 0 <= L <= capacity.
  *   sparsity : must satisfy c->keep == mustafar_keep_count(c->head_dim, sparsity) (0.5 for a
- *              2:4 cache); ignored when c->head_keep is set (each head then keeps c->head_keep[h]).
- * The selection follows c->pattern (per-token top-keep, or 2:4).
+ *              2:4 cache; mustafar_keep_count_channel for a channel-wise one); ignored when
+ *              c->head_keep is set (each head then keeps c->head_keep[h]).
+ * The selection follows c->pattern (per-token top-keep, 2:4, or channel-wise over 16-token
+ * windows; a channel-wise compress also copies the tokens of an incomplete last window,
+ * [16*floor(L/16), L), into slots 0.. of c->window).
  *   c        : the destination cache; its whole tile_offset array is written.
  *   d_err    : optional device word (unused by this call today; may be NULL).
  * Slots >= L are not touched.  Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */
@@ -144,7 +179,11 @@ MUSTAFAR_API mustafar_status mustafar_compress(const void *x, int64_t stride_b, 
  *   d_pos : int32 [batch] device array of slots; a slot outside [0, capacity)
  *           skips that row and sets MUSTAFAR_DEVERR_POS_RANGE in *d_err.
  * The caller advances its lengths (e.g. seq_len = pos + 1) itself; the library
- * keeps no state.  Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */
+ * keeps no state beyond the caches.  A channel-wise cache stores the token in slot
+ * pos % 16 of c->window and prunes its window (tokens 16*floor(pos/16) .. pos) again,
+ * rewriting those tokens' bitmaps and the window's packed values: appends to a row must
+ * come in token order, each after the previous one.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA. */
 MUSTAFAR_API mustafar_status mustafar_append(const void *x, int64_t stride_b, int64_t stride_h,
                                 const int32_t *d_pos, const mustafar_cache_t *c, uint32_t *d_err,
                                 mustafar_stream_t stream);

@@ -33,7 +33,7 @@ def test_header_lists_the_binding_symbols():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.mustafar_abi_version() == 3
+    assert lib.mustafar_abi_version() == 4
 
 
 def test_keep_count_matches_oracle(lib):
@@ -189,3 +189,36 @@ def test_workspace_query(lib):
     assert M.mustafar_decode_workspace_bytes(8, 32, 8, 4160) >= n1
     with pytest.raises(M.MustafarError):
         M.mustafar_decode_workspace_bytes(8, 30, 8, 4160)
+
+
+def test_channel_keep_count_sizes_and_checks(lib):
+    for d in (32, 128, 256):
+        for s in np.concatenate([np.linspace(0, 0.999, 61), [0.3, 0.5, 0.7, 0.75, 0.9375]]):
+            assert M.mustafar_keep_count_channel(d, float(s)) == oracle.keep_count_channel(d, float(s)), (d, s)
+    assert lib.mustafar_keep_count_channel(128, 1.0) == -1 and lib.mustafar_keep_count_channel(100, 0.5) == -1
+    B, H, cap = 3, 4, 192
+    nb, nv, no, nw = M.mustafar_cache_sizes_channel(B, H, 128, cap, 0.7)
+    assert (nb, nv, no, nw) == (B * H * cap * 16, 2 * B * H * cap * 40, B * H * (cap // 64) * 4, B * H * 16 * 128 * 2)
+    # descriptor checks stop in host validation (stride 100 is misaligned: nothing launches)
+    good = _cache(keep=40)
+    good.pattern, good.window = 2, 0x4000
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(good), None, None)
+    assert st == 3  # a valid channel-wise descriptor passes the pattern checks
+    for change, want, msg in [(dict(window=None), 1, "window"), (dict(window=0x4008), 3, "window"),
+                              (dict(keep=39), 1, "multiple of head_dim/16")]:
+        bad = _cache(keep=40)
+        bad.pattern, bad.window = 2, 0x4000
+        for k, v in change.items():
+            setattr(bad, k, v)
+        st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(bad), None, None)
+        assert st == want and msg in err, (change, st, err)
+    # compress: keep must follow the channel rule for that sparsity
+    st, err = _status(lib, "mustafar_compress", 0x5000, 4096, 2048, 128, 64, 0.7, C.byref(_cache(keep=40)), None, None)
+    assert st == 1 and "keep_count(" in err
+    ch = _cache(keep=48)
+    ch.pattern, ch.window = 2, 0x4000
+    st, err = _status(lib, "mustafar_compress", 0x5000, 4096, 2048, 128, 64, 0.7, C.byref(ch), None, None)
+    assert st == 1 and "keep_count_channel" in err
+    with pytest.raises(ValueError):
+        M.CompressedCache(1, 2, 64, [0.5, 0.7], pattern="channel", device="cpu")
+

@@ -447,6 +447,195 @@ def test_24_llama3_gqa_b8_ctx4096():
     U.assert_attn_close(out[rows], o_ref, lse[rows], l_ref, tag="2:4 b8 ctx4096")
 
 
+# ------------------------------------------------------------------------------------ channel-wise direction
+def _channel_matches(cache, x_bits, lens):
+    """Row b of a channel-wise cache against the oracle's compression of its first lens[b] tokens:
+    bitmaps, the whole packed value run of every window, tile offsets and the window copy."""
+    bm, vals, offs = U.cache_np(cache)
+    win = cache.window_view().cpu().numpy().view(np.uint16)
+    for b, Lb in enumerate(lens):
+        ref = oracle.compress_channel(x_bits[b:b + 1, :, :Lb], cache.sparsity, cache.capacity, int(Lb))
+        assert ref["keep"] == cache.keep
+        assert np.array_equal(bm[b, :, :Lb], ref["bitmap"][0, :, :Lb]), ("bitmap", b)
+        assert np.array_equal(vals[b], ref["values"][0]), ("values", b)
+        assert np.array_equal(offs[b], ref["tile_offset"][0]), ("offsets", b)
+        r = int(Lb) % 16
+        assert np.array_equal(win[b, :, :r], ref["window"][0, :, :r]), ("window", b)
+
+
+@pytest.mark.parametrize("s", [0.0, 0.3, 0.7, 0.9375])
+def test_channel_compress_append_bit_exact(s):
+    B, H, L0, L1, cap = 2, 3, 37, 100, 128
+    rng = np.random.default_rng(81)
+    x = synth.keys(B, H, L1, D, 81, "cpu").permute(0, 2, 1, 3).contiguous()  # [B, L, H, d] storage: strided
+    xb = x.view(torch.int16).numpy().view(np.uint16).copy()
+    xb[0, 16:32, 1] = rng.choice(TIE_ROWS, (16, D))  # a whole window of ties
+    xb[1, 40:48, 2] = 0x3C00                          # equal magnitudes across tokens
+    xb[0, 50, 0, :64] = 0x8000
+    xdev = torch.from_numpy(xb.view(np.int16)).view(torch.float16).to(DEV)
+    view = xdev.permute(0, 2, 1, 3)
+    truth = np.ascontiguousarray(xb.transpose(0, 2, 1, 3))
+    c = M.CompressedCache(B, H, cap, s, pattern="channel")
+    M.mustafar_compress(view, L0, s, c)
+    _channel_matches(c, truth, [L0] * B)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for t in range(L0, L1):  # crosses the window edges at 48, 64, 80, 96
+        M.mustafar_append(view[:, :, t], torch.full((B,), t, dtype=torch.int32, device=DEV), c, err=err)
+        if t in (47, 48, 63, 77):
+            _channel_matches(c, truth, [t + 1] * B)
+    _channel_matches(c, truth, [L1] * B)
+    assert int(err.item()) == 0
+    # a full prefill of the same tokens gives the same bytes
+    c2 = M.CompressedCache(B, H, cap, s, pattern="channel")
+    M.mustafar_compress(view, L1, s, c2)
+    assert torch.equal(c.bitmap, c2.bitmap) and torch.equal(c.values, c2.values)
+    assert torch.equal(c.tile_offset, c2.tile_offset)
+
+
+def test_channel_compress_empty_and_full_capacity():
+    B, H, cap = 1, 2, 64
+    x = synth.keys(B, H, cap, D, 82, DEV)
+    c = M.CompressedCache(B, H, cap, 0.7, pattern="channel")
+    M.mustafar_compress(x, 0, 0.7, c)
+    assert not c.bitmap.any() and not c.values.any() and not c.window.any()
+    assert c.tile_offset.tolist() == [0] * H
+    M.mustafar_compress(x, cap, 0.7, c)
+    _channel_matches(c, U.bits(x), [cap])
+    assert not c.window.any()  # 64 tokens: no incomplete window
+
+
+def test_channel_append_out_of_range_skips_row():
+    B, H, L, cap = 2, 2, 20, 64
+    x = synth.keys(B, H, L + 1, D, 83, DEV, capacity=cap)
+    c = M.CompressedCache(B, H, cap, 0.7, pattern="channel")
+    M.mustafar_compress(x, L, 0.7, c)
+    before = (c.bitmap.clone(), c.values.clone(), c.window.clone())
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    M.mustafar_append(x[:, :, L].contiguous(), torch.tensor([-1, cap], dtype=torch.int32, device=DEV), c, err=err)
+    assert int(err.item()) & M.DEVERR_POS_RANGE
+    assert torch.equal(c.bitmap, before[0]) and torch.equal(c.values, before[1]) and torch.equal(c.window, before[2])
+
+
+@pytest.mark.parametrize("v_pat,splits", [("channel", 0), ("topk", 0), ("channel", 3)])
+def test_channel_decode_attn_ragged_lengths(v_pat, splits):
+    # the caches hold 300 tokens; rows attend over fewer, so their last chunk ends inside a window
+    # that was pruned with more tokens (its runs are read by popcount prefixes)
+    B, Hq, Hkv, L, cap = 3, 8, 2, 300, 320
+    sK, sV = 0.7, 0.5
+    K = synth.keys(B, Hkv, L, D, 84, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L, D, 84, DEV, capacity=cap)
+    kc = M.CompressedCache(B, Hkv, cap, sK, pattern="channel")
+    vc = M.CompressedCache(B, Hkv, cap, sV, pattern=v_pat)
+    M.mustafar_compress(K, L, sK, kc)
+    M.mustafar_compress(V, L, sV, vc)
+    q = synth.queries(B, Hq, D, 84, DEV)
+    seq = torch.tensor([L, 203, 17], dtype=torch.int32)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), L, 0.088, num_splits=splits)
+    Kb, Vb = U.bits(K)[:, :, :L], U.bits(V)[:, :, :L]
+    kp = oracle.prune_channel(Kb, sK)
+    vp = oracle.prune_channel(Vb, sV) if v_pat == "channel" else oracle.prune(Vb, oracle.keep_count(D, sV))
+    o_ref, l_ref = oracle.attention(U.bits(q), kp, vp, seq.numpy(), 0.088)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"channel K, {v_pat} V, splits {splits}")
+
+
+@pytest.mark.parametrize("v_pat", ["channel", "2:4"])
+def test_channel_decode_step_ragged_rows(v_pat):
+    # rows move through their windows at different phases: row b skips its first lag[b] steps
+    # (an out-of-range slot: no append, the row attends over nothing), then appends in order
+    B, Hq, Hkv, L0, cap, steps = 3, 8, 2, 40, 128, 30
+    lag = [0, 5, 11]
+    sK, sV = 0.7, 0.5
+    K = synth.keys(B, Hkv, L0, D, 85, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L0, D, 85, DEV, capacity=cap)
+    kc = M.CompressedCache(B, Hkv, cap, sK, pattern="channel")
+    vc = M.CompressedCache(B, Hkv, cap, sV, pattern=v_pat)
+    M.mustafar_compress(K, L0, sK, kc)
+    M.mustafar_compress(V, L0, sV, vc)
+    lens = [L0] * B
+    for st in range(steps):
+        p = [L0 + st - lag[b] if st >= lag[b] else -1 for b in range(B)]
+        kn, vn = synth.step_tokens(B, Hkv, D, 85, st, DEV)
+        for b in range(B):
+            if p[b] >= 0:
+                K[b, :, p[b]] = kn[b]
+                V[b, :, p[b]] = vn[b]
+                lens[b] = p[b] + 1
+        qs = synth.queries(B, Hq, D, 85, DEV, step=st)
+        pos = torch.tensor(p, dtype=torch.int32, device=DEV)
+        out, lse = M.mustafar_decode_step(qs, kn, vn, pos, kc, vc, L0 + steps, 1.0)
+        if st in (0, 7, 8, 12, 29):
+            live = [b for b in range(B) if p[b] >= 0]
+            Kb, Vb = U.bits(K), U.bits(V)
+            o_ref, l_ref = [], []
+            for b in live:
+                kp = oracle.prune_channel(Kb[b:b + 1, :, :lens[b]], sK)
+                vp = (oracle.prune_channel(Vb[b:b + 1, :, :lens[b]], sV) if v_pat == "channel"
+                      else oracle.prune_24(Vb[b:b + 1, :, :lens[b]]))
+                o, l = oracle.attention(U.bits(qs[b:b + 1]), kp, vp, [lens[b]], 1.0)
+                o_ref.append(o)
+                l_ref.append(l)
+            U.assert_attn_close(out[live], np.concatenate(o_ref), lse[live], np.concatenate(l_ref),
+                                tag=f"channel step {st}")
+    _channel_matches(kc, U.bits(K), lens)
+    if v_pat == "channel":
+        _channel_matches(vc, U.bits(V), lens)
+
+
+def test_channel_decode_step_same_bits_as_append_then_attend():
+    B, Hq, Hkv, L0, cap = 4, 32, 8, 250, 320
+    K = synth.keys(B, Hkv, L0, D, 86, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L0, D, 86, DEV, capacity=cap)
+    caches = []
+    for _ in range(2):
+        kc = M.CompressedCache(B, Hkv, cap, 0.7, pattern="channel")
+        vc = M.CompressedCache(B, Hkv, cap, 0.7, pattern="channel")
+        M.mustafar_compress(K, L0, 0.7, kc)
+        M.mustafar_compress(V, L0, 0.7, vc)
+        caches.append((kc, vc))
+    (kc, vc), (kc2, vc2) = caches
+    for st in range(8):
+        kn, vn = synth.step_tokens(B, Hkv, D, 86, st, DEV)
+        pos = torch.full((B,), L0 + st, dtype=torch.int32, device=DEV)
+        qs = synth.queries(B, Hq, D, 86, DEV, step=st)
+        o1, l1 = M.mustafar_decode_step(qs, kn, vn, pos, kc, vc, cap, 1.0)
+        M.mustafar_append(kn, pos, kc2)
+        M.mustafar_append(vn, pos, vc2)
+        o2, l2 = M.mustafar_decode_attn(qs, kc2, vc2, pos + 1, cap, 1.0)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {st}"
+    for a, b in ((kc, kc2), (vc, vc2)):
+        assert torch.equal(a.bitmap, b.bitmap) and torch.equal(a.values, b.values) and torch.equal(a.window, b.window)
+
+
+def test_channel_llama3_gqa_b8_ctx4096_s07():
+    B, Hq, Hkv, L, cap = 8, 32, 8, 4096, 4160
+    K = synth.keys(B, Hkv, L, D, 1009, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L, D, 1009, DEV, capacity=cap)
+    kc = M.CompressedCache(B, Hkv, cap, 0.7, pattern="channel")
+    vc = M.CompressedCache(B, Hkv, cap, 0.7, pattern="channel")
+    M.mustafar_compress(K, L, 0.7, kc)
+    M.mustafar_compress(V, L, 0.7, vc)
+    q = synth.queries(B, Hq, D, 1009, DEV)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, torch.full((B,), L, dtype=torch.int32, device=DEV), L, 0.088)
+    rows = [2, 7]
+    Kb, Vb = U.bits(K)[:, :, :L], U.bits(V)[:, :, :L]
+    bm, vals, _ = U.cache_np(kc)
+    for b, h in ((2, 1), (7, 6)):
+        ref = oracle.compress_channel(Kb[b:b + 1, h:h + 1], 0.7, cap, L)
+        assert np.array_equal(bm[b, h], ref["bitmap"][0, 0]) and np.array_equal(vals[b, h], ref["values"][0, 0])
+    o_ref, l_ref = oracle.attention(U.bits(q[rows]), oracle.prune_channel(Kb[rows], 0.7),
+                                    oracle.prune_channel(Vb[rows], 0.7), [L] * len(rows), 0.088)
+    U.assert_attn_close(out[rows], o_ref, lse[rows], l_ref, tag="channel b8 ctx4096")
+    # one fused step opens a new window (a lone token keeps every channel)
+    kn, vn = synth.step_tokens(B, Hkv, D, 1009, 0, DEV)
+    pos = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    out, lse = M.mustafar_decode_step(q, kn, vn, pos, kc, vc, L + 1, 0.088)
+    K[:, :, L], V[:, :, L] = kn, vn
+    Kb, Vb = U.bits(K)[:, :, :L + 1], U.bits(V)[:, :, :L + 1]
+    o_ref, l_ref = oracle.attention(U.bits(q[rows]), oracle.prune_channel(Kb[rows], 0.7),
+                                    oracle.prune_channel(Vb[rows], 0.7), [L + 1] * len(rows), 0.088)
+    U.assert_attn_close(out[rows], o_ref, lse[rows], l_ref, tag="channel b8 ctx4096 fused step")
+
+
 # ------------------------------------------------------------------------------------ the workload shapes
 def test_llama3_gqa_b1_ctx1024_s05():
     B, Hq, Hkv, L = 1, 32, 8, 1024

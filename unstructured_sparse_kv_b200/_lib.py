@@ -22,6 +22,8 @@ DEVERR_LEN_RANGE = 0x2
 HEAD_DIM = 128
 PATTERN_TOPK = 0   # per-token top-keep pruning (the method)
 PATTERN_2_4 = 1    # 2:4 semi-structured pruning (the comparison pattern)
+PATTERN_CHANNEL = 2  # channel-wise pruning over 16-token windows
+WINDOW_TOKENS = 16
 
 # every symbol include/mustafar.h declares
 ABI_SYMBOLS = (
@@ -29,6 +31,7 @@ ABI_SYMBOLS = (
     "mustafar_decode_workspace_bytes", "mustafar_decode_attn", "mustafar_dense_decode_attn",
     "mustafar_decode_plan_splits", "mustafar_status_string", "mustafar_last_error", "mustafar_abi_version",
     "mustafar_decode_attn_noalloc", "mustafar_decode_step", "mustafar_cache_sizes_per_head",
+    "mustafar_keep_count_channel", "mustafar_cache_sizes_channel",
 )
 
 
@@ -43,7 +46,7 @@ class CacheT(C.Structure):
     _fields_ = [("batch", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
                 ("capacity", C.c_int32), ("keep", C.c_int32), ("bitmap", C.c_void_p),
                 ("values", C.c_void_p), ("tile_offset", C.c_void_p), ("head_keep", C.c_void_p),
-                ("pattern", C.c_int32)]
+                ("pattern", C.c_int32), ("window", C.c_void_p)]
 
 
 _lib = None
@@ -61,6 +64,8 @@ def load() -> C.CDLL:
     P = C.POINTER
     sig = {
         "mustafar_keep_count": (i32, [i32, f32]),
+        "mustafar_keep_count_channel": (i32, [i32, f32]),
+        "mustafar_cache_sizes_channel": (i32, [i32, i32, i32, i32, f32, P(sz), P(sz), P(sz), P(sz)]),
         "mustafar_cache_sizes": (i32, [i32, i32, i32, i32, f32, P(sz), P(sz), P(sz)]),
         "mustafar_cache_sizes_per_head": (i32, [i32, i32, i32, i32, vp, P(sz), P(sz), P(sz)]),
         "mustafar_compress": (i32, [vp, i64, i64, i64, i32, f32, P(CacheT), vp, vp]),
@@ -113,6 +118,22 @@ def mustafar_keep_count(head_dim: int, sparsity: float) -> int:
     return k
 
 
+def mustafar_keep_count_channel(head_dim: int, sparsity: float) -> int:
+    """Values per token slot of a channel-wise cache: (head_dim/16) * (16 - floor(16*s))."""
+    k = load().mustafar_keep_count_channel(head_dim, sparsity)
+    if k < 0:
+        raise ValueError("head_dim must be a positive multiple of 32 and sparsity in [0, 1)")
+    return k
+
+
+def mustafar_cache_sizes_channel(batch, num_kv_heads, head_dim, capacity, sparsity):
+    """(bitmap_bytes, values_bytes, offset_bytes, window_bytes) of a channel-wise cache."""
+    a, b, c, w = C.c_size_t(), C.c_size_t(), C.c_size_t(), C.c_size_t()
+    _check(load().mustafar_cache_sizes_channel(batch, num_kv_heads, head_dim, capacity, sparsity, C.byref(a),
+                                               C.byref(b), C.byref(c), C.byref(w)))
+    return a.value, b.value, c.value, w.value
+
+
 def mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity):
     a, b, c = C.c_size_t(), C.c_size_t(), C.c_size_t()
     _check(load().mustafar_cache_sizes(batch, num_kv_heads, head_dim, capacity, sparsity,
@@ -149,13 +170,17 @@ class CompressedCache:
 
     ``sparsity`` is one value for every kv head, or a sequence with one sparsity per kv head
     (then head h keeps ``mustafar_keep_count(head_dim, sparsity[h])`` channels per token).
-    ``pattern="2:4"`` selects 2:4 semi-structured pruning instead (sparsity 0.5, one value)."""
+    ``pattern="2:4"`` selects 2:4 semi-structured pruning instead (sparsity 0.5, one value), and
+    ``pattern="channel"`` channel-wise pruning over 16-token windows (one sparsity; the cache then
+    also holds ``window``, the dense copy of each stream's newest incomplete window)."""
 
     def __init__(self, batch: int, num_kv_heads: int, capacity: int, sparsity, head_dim: int = HEAD_DIM,
                  device="cuda", pattern: str = "topk"):
         self.batch, self.num_kv_heads, self.head_dim, self.capacity = batch, num_kv_heads, head_dim, capacity
-        if pattern not in ("topk", "2:4"):
-            raise ValueError("pattern must be 'topk' or '2:4'")
+        if pattern not in ("topk", "2:4", "channel"):
+            raise ValueError("pattern must be 'topk', '2:4' or 'channel'")
+        if pattern == "channel" and isinstance(sparsity, (list, tuple)):
+            raise ValueError("a channel-wise cache has one sparsity for every head")
         if pattern == "2:4" and (isinstance(sparsity, (list, tuple)) or float(sparsity) != 0.5):
             raise ValueError("a 2:4 cache has sparsity 0.5 for every head")
         self.pattern = pattern
@@ -169,6 +194,12 @@ class CompressedCache:
             self.keep = max(self.head_keep)
             nb, nv, no = mustafar_cache_sizes_per_head(batch, num_kv_heads, capacity, self.head_keep, head_dim)
             self._head_keep_arr = (C.c_int32 * num_kv_heads)(*self.head_keep)
+        elif pattern == "channel":
+            self.sparsity = float(sparsity)
+            self.keep = mustafar_keep_count_channel(head_dim, sparsity)
+            self.head_keep = [self.keep] * num_kv_heads
+            self.head_sparsity = None
+            nb, nv, no, nw = mustafar_cache_sizes_channel(batch, num_kv_heads, head_dim, capacity, sparsity)
         else:
             self.sparsity = float(sparsity)
             self.keep = mustafar_keep_count(head_dim, sparsity)
@@ -178,10 +209,12 @@ class CompressedCache:
         self.bitmap = torch.zeros(nb // 4, dtype=torch.int32, device=device)
         self.values = torch.zeros(nv // 2, dtype=torch.int16, device=device)
         self.tile_offset = torch.zeros(no // 4, dtype=torch.int32, device=device)
+        self.window = (torch.zeros(nw // 2, dtype=torch.int16, device=device) if pattern == "channel" else None)
         hk = C.cast(self._head_keep_arr, C.c_void_p).value if self._head_keep_arr is not None else None
+        code = {"topk": PATTERN_TOPK, "2:4": PATTERN_2_4, "channel": PATTERN_CHANNEL}[pattern]
         self._struct = CacheT(batch, num_kv_heads, head_dim, capacity, self.keep, self.bitmap.data_ptr(),
-                              self.values.data_ptr(), self.tile_offset.data_ptr(), hk,
-                              PATTERN_2_4 if pattern == "2:4" else PATTERN_TOPK)
+                              self.values.data_ptr(), self.tile_offset.data_ptr(), hk, code,
+                              self.window.data_ptr() if self.window is not None else None)
 
     @property
     def struct(self) -> CacheT:
@@ -192,7 +225,8 @@ class CompressedCache:
         return self._head_keep_arr is not None
 
     def nbytes(self) -> int:
-        return self.bitmap.numel() * 4 + self.values.numel() * 2 + self.tile_offset.numel() * 4
+        extra = self.window.numel() * 2 if self.window is not None else 0
+        return self.bitmap.numel() * 4 + self.values.numel() * 2 + self.tile_offset.numel() * 4 + extra
 
     def value_base(self, b: int, h: int) -> int:
         """Element index where stream (b, h)'s packed values start."""
@@ -211,6 +245,12 @@ class CompressedCache:
         B, H, cap, d = self.batch, self.num_kv_heads, self.capacity, self.head_dim
         return (self.bitmap.view(B, H, cap, d // 32), self.values.view(B, H, cap * self.keep),
                 self.tile_offset.view(B, H, cap // 64))
+
+    def window_view(self):
+        """window [B, H, 16, d] int16 of a channel-wise cache."""
+        if self.window is None:
+            raise ValueError("only a channel-wise cache has a window")
+        return self.window.view(self.batch, self.num_kv_heads, WINDOW_TOKENS, self.head_dim)
 
 
 # ------------------------------------------------------------------------------------------- calls

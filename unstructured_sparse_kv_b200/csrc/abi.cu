@@ -38,6 +38,17 @@ int32_t keep_count(int32_t d, float s) {
   return d - static_cast<int32_t>(pruned);
 }
 
+// Values per token slot of a channel-wise cache: (d/16) * (16 - floor(16 s)).
+int32_t keep_count_channel(int32_t d, float s) {
+  if (d <= 0 || d % 32 != 0) return -1;
+  if (!(s >= 0.0f && s < 1.0f)) return -1;
+  const int32_t F = static_cast<int32_t>(std::floor(static_cast<double>(s) * kWindowTokens));
+  return (d / kWindowTokens) * (kWindowTokens - F);
+}
+
+// The prune count F of a full window of a checked channel-wise cache (keep = (d/16) * (16 - F)).
+int channel_prune_count(const mustafar_cache_t *c) { return kWindowTokens - c->keep / (c->head_dim / kWindowTokens); }
+
 mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
   if (c == nullptr) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: cache descriptor is NULL", name);
   if (c->batch <= 0 || c->num_kv_heads <= 0 || c->capacity <= 0)
@@ -50,8 +61,18 @@ mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: capacity must be a multiple of 64 (got %d)", name, c->capacity);
   if (c->keep < 1 || c->keep > c->head_dim)
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: keep must lie in [1, head_dim] (got %d)", name, c->keep);
-  if (c->pattern != MUSTAFAR_PATTERN_TOPK && c->pattern != MUSTAFAR_PATTERN_2_4)
-    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: pattern must be MUSTAFAR_PATTERN_TOPK or _2_4 (got %d)", name, c->pattern);
+  if (c->pattern != MUSTAFAR_PATTERN_TOPK && c->pattern != MUSTAFAR_PATTERN_2_4 &&
+      c->pattern != MUSTAFAR_PATTERN_CHANNEL)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: pattern must be MUSTAFAR_PATTERN_TOPK, _2_4 or _CHANNEL (got %d)", name,
+                c->pattern);
+  if (c->pattern == MUSTAFAR_PATTERN_CHANNEL) {
+    if (c->keep % (c->head_dim / kWindowTokens) != 0 || c->head_keep != nullptr)
+      return fail(MUSTAFAR_ERR_INVALID_ARG,
+                  "%s: a channel-wise cache keeps a multiple of head_dim/16 values per token and has no head_keep",
+                  name);
+    if (c->window == nullptr) return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: a channel-wise cache needs its window array", name);
+    if (!aligned(c->window, 16)) return fail(MUSTAFAR_ERR_MISALIGNED, "%s: window needs 16-byte alignment", name);
+  }
   if (c->pattern == MUSTAFAR_PATTERN_2_4 && (c->keep != c->head_dim / 2 || c->head_keep != nullptr))
     return fail(MUSTAFAR_ERR_INVALID_ARG, "%s: a 2:4 cache keeps head_dim/2 channels and has no head_keep", name);
   if (c->head_keep != nullptr) {
@@ -82,11 +103,11 @@ mustafar_status check_cache(const mustafar_cache_t *c, const char *name) {
 void set_last_error(const char *msg) { g_last_error = msg; }
 
 cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes) {
-  static int done[64][32];  // bytes already granted per (device, kernel slot)
+  static int done[64][kKernelSlots];  // bytes already granted per (device, kernel slot)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || slot < 0 || slot >= 32)
+  if (dev < 0 || dev >= 64 || slot < 0 || slot >= kKernelSlots)
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (done[dev][slot] >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -133,6 +154,24 @@ static HeadKeep head_keep_of(const mustafar_cache_t *c) {
 
 int32_t mustafar_keep_count(int32_t head_dim, float sparsity) { return keep_count(head_dim, sparsity); }
 
+int32_t mustafar_keep_count_channel(int32_t head_dim, float sparsity) { return keep_count_channel(head_dim, sparsity); }
+
+mustafar_status mustafar_cache_sizes_channel(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity,
+                                             float sparsity, size_t *bitmap_bytes, size_t *values_bytes,
+                                             size_t *offset_bytes, size_t *window_bytes) {
+  const int32_t k = keep_count_channel(head_dim, sparsity);
+  if (k < 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes_channel: head_dim %% 32 != 0 or sparsity outside [0,1)");
+  if (batch <= 0 || num_kv_heads <= 0 || capacity <= 0 || capacity % kTileTokens != 0)
+    return fail(MUSTAFAR_ERR_INVALID_ARG, "cache_sizes_channel: positive shapes and capacity %% 64 == 0 required");
+  const size_t streams = static_cast<size_t>(batch) * num_kv_heads;
+  if (bitmap_bytes) *bitmap_bytes = streams * capacity * (head_dim / 8);
+  if (values_bytes) *values_bytes = streams * capacity * static_cast<size_t>(k) * 2;
+  if (offset_bytes) *offset_bytes = streams * (capacity / kTileTokens) * 4;
+  if (window_bytes) *window_bytes = streams * kWindowTokens * static_cast<size_t>(head_dim) * 2;
+  return MUSTAFAR_OK;
+}
+
 mustafar_status mustafar_cache_sizes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity,
                                      float sparsity, size_t *bitmap_bytes, size_t *values_bytes,
                                      size_t *offset_bytes) {
@@ -176,11 +215,12 @@ mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t strid
   mustafar_status s = check_cache(c, "compress");
   if (s != MUSTAFAR_OK) return s;
   if (c->head_keep == nullptr) {
-    const int32_t k = keep_count(c->head_dim, sparsity);
+    const bool chan = c->pattern == MUSTAFAR_PATTERN_CHANNEL;
+    const int32_t k = chan ? keep_count_channel(c->head_dim, sparsity) : keep_count(c->head_dim, sparsity);
     if (k < 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: sparsity must lie in [0, 1)");
     if (k != c->keep)
-      return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: cache keep %d != keep_count(%d, %g) = %d", c->keep,
-                  c->head_dim, static_cast<double>(sparsity), k);
+      return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: cache keep %d != %s(%d, %g) = %d", c->keep,
+                  chan ? "keep_count_channel" : "keep_count", c->head_dim, static_cast<double>(sparsity), k);
   }
   if (L < 0 || L > c->capacity) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: L must lie in [0, capacity]");
   if (x == nullptr && L > 0) return fail(MUSTAFAR_ERR_INVALID_ARG, "compress: x is NULL");
@@ -192,7 +232,8 @@ mustafar_status mustafar_compress(const void *x, int64_t stride_b, int64_t strid
   }
   cudaError_t e = launch_compress(static_cast<const uint16_t *>(x), stride_b, stride_h, stride_t, L, c->batch,
                                   c->num_kv_heads, head_keep_of(c), c->keep, c->capacity, c->bitmap, c->values,
-                                  c->tile_offset, c->pattern == MUSTAFAR_PATTERN_2_4,
+                                  c->tile_offset, static_cast<Pattern>(c->pattern), c->window,
+                                  c->pattern == MUSTAFAR_PATTERN_CHANNEL ? channel_prune_count(c) : 0,
                                   reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "compress launch");
 }
@@ -208,7 +249,9 @@ mustafar_status mustafar_append(const void *x, int64_t stride_b, int64_t stride_
   if (!aligned(d_pos, 4)) return fail(MUSTAFAR_ERR_MISALIGNED, "append: pos must be 4-byte aligned");
   cudaError_t e = launch_append(static_cast<const uint16_t *>(x), stride_b, stride_h, d_pos, c->batch,
                                 c->num_kv_heads, head_keep_of(c), c->capacity, c->bitmap, c->values, d_err,
-                                c->pattern == MUSTAFAR_PATTERN_2_4, reinterpret_cast<cudaStream_t>(stream));
+                                static_cast<Pattern>(c->pattern), c->window,
+                                c->pattern == MUSTAFAR_PATTERN_CHANNEL ? channel_prune_count(c) : 0,
+                                reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, "append launch");
 }
 
@@ -250,7 +293,10 @@ namespace {
 mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *workspace, size_t workspace_bytes,
                            const char *name, cudaStream_t stream) {
   DecodePlan plan;
-  const int variant = p.perhead ? 1 : (p.p24_k && p.p24_v ? 2 : 0);
+  const bool chan = p.kwin != nullptr || p.vwin != nullptr;
+  if (chan && p.perhead)
+    return fail(MUSTAFAR_ERR_UNSUPPORTED, "%s: a channel-wise cache cannot be paired with a per-head cache", name);
+  const int variant = chan ? 3 : p.perhead ? 1 : (p.p24_k && p.p24_v ? 2 : 0);
   cudaError_t e = plan_sparse(p.B, p.Hkv, p.G, max_len, p.keep_k, p.keep_v, num_splits, variant, &plan);
   if (e != cudaSuccess) return cuda_fail(e, name);
   p.stage_bytes = plan.stage_bytes;
@@ -293,6 +339,15 @@ mustafar_status run_decode(bool sparse, DecodeParams &p, int max_len, int num_sp
   }
   e = launch_dense(p, plan, stream);
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, name);
+}
+
+// Channel-wise caches of a decode call: their window copies and full-window prune counts.
+void set_channel(DecodeParams &p, const mustafar_cache_t *k, const mustafar_cache_t *v) {
+  const bool ck = k->pattern == MUSTAFAR_PATTERN_CHANNEL, cv = v->pattern == MUSTAFAR_PATTERN_CHANNEL;
+  p.kwin = ck ? k->window : nullptr;
+  p.vwin = cv ? v->window : nullptr;
+  p.chF_k = ck ? channel_prune_count(k) : 0;
+  p.chF_v = cv ? channel_prune_count(v) : 0;
 }
 
 mustafar_status check_decode_common(const void *q, int32_t Hq, int32_t B, int32_t Hkv, const int32_t *d_seq_len,
@@ -340,6 +395,7 @@ mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_heads, const m
   p.perhead = k->head_keep != nullptr || v->head_keep != nullptr;
   p.p24_k = k->pattern == MUSTAFAR_PATTERN_2_4;
   p.p24_v = v->pattern == MUSTAFAR_PATTERN_2_4;
+  set_channel(p, k, v);
   p.cap_k = k->capacity;
   p.cap_v = v->capacity;
   p.seq_len = d_seq_len;
@@ -391,6 +447,7 @@ mustafar_status mustafar_decode_step(const void *q, int32_t num_q_heads, const v
   p.perhead = k->head_keep != nullptr || v->head_keep != nullptr;
   p.p24_k = k->pattern == MUSTAFAR_PATTERN_2_4;
   p.p24_v = v->pattern == MUSTAFAR_PATTERN_2_4;
+  set_channel(p, k, v);
   p.cap_k = k->capacity;
   p.cap_v = v->capacity;
   p.B = k->batch;

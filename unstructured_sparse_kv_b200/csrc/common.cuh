@@ -11,6 +11,8 @@ constexpr int kHeadDim = 128;          // channels per (token, kv head) vector
 constexpr int kWords = kHeadDim / 32;  // bitmap words per token
 constexpr int kTileTokens = 64;        // tokens per tile_offset entry
 constexpr int kChunk = 16;             // tokens per warp work item in decode attention
+constexpr int kWindowTokens = 16;      // tokens per channel-wise pruning window
+static_assert(kWindowTokens == kChunk, "a channel-wise window must be exactly one decode chunk");
 constexpr int kRowHalves = 136;        // padded fp16 row of a dense smem tile (272 B, conflict-free ldmatrix)
 constexpr int kRowBytes = kRowHalves * 2;
 constexpr int kTileBytes = kChunk * kRowBytes;  // one dense 16 x 128 fp16 tile in smem (4352 B)

@@ -10,6 +10,8 @@
 //   own row, writes its 16-byte bitmap, packs its kept values into a shared staging
 //   run, and the CTA writes the 128*k packed values with coalesced 16-byte stores.
 // append: one warp per (b, kv head) vector of the new token.
+// channel-wise caches: one warp per 16-token window (compress) or per stream's newest window
+//   (append), through warp_compress_window.
 #include "internal.h"
 #include "select.cuh"
 
@@ -126,9 +128,62 @@ append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int3
   }
 }
 
+// Channel-wise compress: warp w of CTA x takes window 4x + w of stream (b = z, h = y), and the
+// warp of an incomplete last window also keeps its tokens in the stream's dense window copy.
+__global__ void __launch_bounds__(128)
+compress_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, int keep,
+                        int F, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
+                        uint32_t *__restrict__ tile_offset, uint16_t *__restrict__ window) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t stream = static_cast<int64_t>(b) * H + h;
+  // tile i starts at 64*i*keep: window j owns the 16*keep elements from j*16*keep
+  const int ntiles = cap / kTileTokens;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ntiles; i += gridDim.x * blockDim.x)
+    tile_offset[stream * ntiles + i] = static_cast<uint32_t>(i) * kTileTokens * static_cast<uint32_t>(keep);
+  const int t0 = (blockIdx.x * 4 + warp) * kWindowTokens;
+  if (t0 >= L) return;
+  const int n = min(kWindowTokens, L - t0);
+  const uint16_t *xs = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh + static_cast<int64_t>(t0) * st;
+  uint16_t *win = n < kWindowTokens ? window + stream * kWindowTokens * kHeadDim : nullptr;
+  warp_compress_window([=](int t) { return xs + static_cast<int64_t>(t) * st; }, n, F,
+                       bitmap + (stream * cap + t0) * kWords, values + (stream * cap + t0) * keep, win, 0, lane);
+}
+
+// Channel-wise append: one warp per (b, kv head).  The new token goes to slot pos % 16 of the
+// stream's window copy, and the window (tokens 16*floor(pos/16) .. pos) is pruned again.
+__global__ void __launch_bounds__(128)
+append_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int32_t *__restrict__ pos, int B,
+                      int H, int keep, int F, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
+                      uint16_t *window, uint32_t *__restrict__ err) {
+  const int lane = threadIdx.x & 31;
+  const int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (v >= B * H) return;
+  const int b = v / H, h = v - b * H;
+  const int p = pos[b];
+  if (p < 0 || p >= cap) {
+    if (lane == 0 && err != nullptr) atomicOr(err, MUSTAFAR_DEVERR_POS_RANGE);
+    return;
+  }
+  const int r = p % kWindowTokens, t0 = p - r;
+  const int64_t stream = static_cast<int64_t>(b) * H + h;
+  const uint16_t *xn = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
+  uint16_t *win = window + stream * kWindowTokens * kHeadDim;
+  warp_compress_window([=](int t) -> const uint16_t * { return t < r ? win + t * kHeadDim : xn; }, r + 1, F,
+                       bitmap + (stream * cap + t0) * kWords, values + (stream * cap + t0) * keep, win, r, lane);
+}
+
 cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
                             const HeadKeep &hk, int kmax, int cap, uint32_t *bitmap, uint16_t *values,
-                            uint32_t *tile_offset, bool p24, cudaStream_t stream) {
+                            uint32_t *tile_offset, Pattern pat, uint16_t *window, int chF, cudaStream_t stream) {
+  if (pat == Pattern::kChannel) {
+    const int windows = (L + kWindowTokens - 1) / kWindowTokens;
+    dim3 grid(windows > 0 ? (windows + 3) / 4 : 1, H, B);
+    compress_channel_kernel<<<grid, 128, 0, stream>>>(x, sb, sh, st, L, H, kmax, chF, cap, bitmap, values,
+                                                      tile_offset, window);
+    return cudaGetLastError();
+  }
+  const bool p24 = pat == Pattern::k24;
   auto kernel = p24 ? compress_kernel<true> : compress_kernel<false>;
   const size_t smem = kCompressThreads * kRowBytesDense + static_cast<size_t>(kCompressThreads) * kmax * 2;
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(kernel), p24 ? 9 : 0,
@@ -142,10 +197,15 @@ cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t s
 
 cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H,
                           const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
-                          bool p24, cudaStream_t stream) {
-  auto kernel = p24 ? append_kernel<true> : append_kernel<false>;
+                          Pattern pat, uint16_t *window, int chF, cudaStream_t stream) {
   const int warps = B * H;
   const int threads = 128;  // 4 vectors per CTA
+  if (pat == Pattern::kChannel) {
+    append_channel_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(
+        x, sb, sh, pos, B, H, hk.k[0], chF, cap, bitmap, values, window, err);
+    return cudaGetLastError();
+  }
+  auto kernel = pat == Pattern::k24 ? append_kernel<true> : append_kernel<false>;
   kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, hk, cap, bitmap,
                                                                        values, err);
   return cudaGetLastError();

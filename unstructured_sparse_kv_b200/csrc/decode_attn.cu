@@ -374,12 +374,12 @@ cudaError_t device_info(DeviceInfo *info) {
 // resident CTAs per SM for a kernel and dynamic smem size, cached per device (the query is
 // made once, outside any stream capture, so planning stays capture-safe afterwards)
 cudaError_t occupancy(KernelFn fn, int slot, int smem, int *per_sm) {
-  static int cache_smem[64][32];
-  static int cache_val[64][32];
+  static int cache_smem[64][kKernelSlots];
+  static int cache_val[64][kKernelSlots];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const bool cacheable = dev >= 0 && dev < 64 && slot >= 0 && slot < 32;
+  const bool cacheable = dev >= 0 && dev < 64 && slot >= 0 && slot < kKernelSlots;
   if (cacheable && cache_smem[dev][slot] == smem && cache_val[dev][slot] > 0) {
     *per_sm = cache_val[dev][slot];
     return cudaSuccess;

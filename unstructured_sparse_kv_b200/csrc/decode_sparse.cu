@@ -173,8 +173,10 @@ __device__ __forceinline__ void load_q(const DecodeParams &P, int b, int g, int 
 
 // One 16-token chunk staged at `stage` ([K bitmap rows 16x16 B][V bitmap rows][K values 16*kK]
 // [V values 16*kV]); tokens t0 .. t0+15 of a row of length L.  `htab` is the warp's 512-byte
-// per-row half-word prefix table.
-template <bool HIROWS, bool PERHEAD, bool P24>
+// per-row half-word prefix table.  SCAN: token runs of varying length (a channel-wise cache), each
+// found by the kept counts of the tokens before it in the chunk; otherwise token T's run starts at
+// T*keep.
+template <bool HIROWS, bool PERHEAD, bool P24, bool SCAN>
 __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *stage, uint8_t *htab, uint32_t za,
                                               int t0, int L, int kKh, int kVh, int lane, const uint32_t (&qa)[8][4],
                                               Acc<HIROWS> &acc, const uint2 *lut24) {
@@ -197,8 +199,23 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
       const uint32_t h1 = c0 + __popc(w.y & 0xFFFFu), c1 = c0 + __popc(w.y);
       const uint32_t h2 = c1 + __popc(w.z & 0xFFFFu), c2 = c1 + __popc(w.z);
       const uint32_t h3 = c2 + __popc(w.w & 0xFFFFu);
+      uint32_t base = 0u;
+      if constexpr (SCAN) {
+        // the row's run start: an exclusive prefix sum of the kept counts over the chunk's 16 rows
+        // of its cache (lanes 0-15 K, 16-31 V), capped at the staged run length so that a row never
+        // reads outside the staging buffers, whatever its bitmap holds
+        const uint32_t tot = c2 + __popc(w.w);
+        uint32_t inc = tot;
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o, 16);
+          if ((lane & 15) >= o) inc += y;
+        }
+        base = min(inc - tot, static_cast<uint32_t>(kChunk * (lane < 16 ? kK : kV)));
+        base |= base << 16;
+      }
       *reinterpret_cast<uint4 *>(htab + lane * 16) =
-          make_uint4(h0 << 16, c0 | (h1 << 16), c1 | (h2 << 16), c2 | (h3 << 16));
+          make_uint4((h0 << 16) + base, (c0 | (h1 << 16)) + base, (c1 | (h2 << 16)) + base, (c2 | (h3 << 16)) + base);
     }
   }
   __syncwarp();
@@ -226,7 +243,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
       }
     } else {
       const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
-      const uint32_t rbase = kvals + 2 * T * kK;
+      const uint32_t rbase = SCAN ? kvals : kvals + 2 * T * kK;
       expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
     }
 #pragma unroll
@@ -335,7 +352,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
         const int T = 2 * qq + 8 * pair + e;
         const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
         const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
-        expand_half(bits, vvals + 2 * (T * kV + pre), za, e ? x1 : x0);
+        expand_half(bits, vvals + 2 * ((SCAN ? 0 : T * kV) + pre), za, e ? x1 : x0);
       }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
@@ -547,7 +564,7 @@ __constant__ uint2 kLut24[16] = {
     {0x5454u, 0x5454u}, {0x5410u, 0x3254u}, {0x1054u, 0x3254u}, {0x5454u, 0x5454u},  // 8, 1001, 1010, 11
     {0x5454u, 0x3210u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}};  // 1100, 13, 14, 15
 
-template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24>
+template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24, bool SCAN>
 __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
@@ -660,13 +677,26 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
             const int keep = kside ? keep_of<PERHEAD>(P.hk_k, P.keep_k, st.g) : keep_of<PERHEAD>(P.hk_v, P.keep_v, st.g);
             const int64_t base = kside ? base_of<PERHEAD>(P.hk_k, P.keep_k, st.b, st.g, P.Hkv, capx)
                                        : base_of<PERHEAD>(P.hk_v, P.keep_v, st.b, st.g, P.Hkv, capx);
-            const int64_t slot = (static_cast<int64_t>(st.b) * P.Hkv + st.g) * capx + p;
-            uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + slot * kWords;
-            uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
-            if (kside ? P.p24_k : P.p24_v)
-              warp_compress_vector_24(src, bm, vals, lane);
-            else
-              warp_compress_vector(src, keep, bm, vals, lane);
+            const int64_t sid = static_cast<int64_t>(st.b) * P.Hkv + st.g;
+            uint16_t *win = SCAN ? (kside ? P.kwin : P.vwin) : nullptr;
+            if (SCAN && win != nullptr) {
+              // channel-wise cache: the new token joins its window's dense copy and the whole window
+              // (which is this chunk) is pruned again
+              const int r = p % kWindowTokens, tw = p - r;
+              win += sid * kWindowTokens * kHeadDim;
+              uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + (sid * capx + tw) * kWords;
+              uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(tw) * keep;
+              const uint16_t *wsrc = win;
+              warp_compress_window([=](int t) -> const uint16_t * { return t < r ? wsrc + t * kHeadDim : src; }, r + 1,
+                                   kside ? P.chF_k : P.chF_v, bm, vals, win, r, lane);
+            } else {
+              uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + (sid * capx + p) * kWords;
+              uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
+              if (kside ? P.p24_k : P.p24_v)
+                warp_compress_vector_24(src, bm, vals, lane);
+              else
+                warp_compress_vector(src, keep, bm, vals, lane);
+            }
           }
         }
       }
@@ -738,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       uint8_t *stage = wbase + slot * P.stage_bytes;
       if (!mbar_wait(bars + 8 * slot, (citem / NSTAGE) & 1, timed_out ? kWaitCyclesAfter : kWaitCycles))
         timed_out = true;
-      consume_chunk<HIROWS, PERHEAD, P24>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
+      consume_chunk<HIROWS, PERHEAD, P24, SCAN>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
                                           lut24);
       __syncwarp();
       produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
@@ -772,30 +802,33 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
 // ------------------------------------------------------------------------------------ host side
 using SparseFn = void (*)(const DecodeParams);
 
-template <int NSTAGE, bool PERHEAD, bool P24>
+template <int NSTAGE, bool PERHEAD, bool P24, bool SCAN>
 SparseFn pick_rows(bool hirows) {
-  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD, P24> : sparse_decode_kernel<NSTAGE, false, PERHEAD, P24>;
+  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD, P24, SCAN>
+                : sparse_decode_kernel<NSTAGE, false, PERHEAD, P24, SCAN>;
 }
 
-template <bool PERHEAD, bool P24>
+template <bool PERHEAD, bool P24, bool SCAN>
 SparseFn pick_stages(int nstage, bool hirows) {
   switch (nstage) {
-    case 2: return pick_rows<2, PERHEAD, P24>(hirows);
-    case 3: return pick_rows<3, PERHEAD, P24>(hirows);
-    default: return pick_rows<4, PERHEAD, P24>(hirows);
+    case 2: return pick_rows<2, PERHEAD, P24, SCAN>(hirows);
+    case 3: return pick_rows<3, PERHEAD, P24, SCAN>(hirows);
+    default: return pick_rows<4, PERHEAD, P24, SCAN>(hirows);
   }
 }
 
-// variant: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4
+// variant: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4, 3 token runs found by
+// popcount prefixes (a channel-wise cache; either cache may also be token-wise or 2:4)
 SparseFn pick_sparse(int nstage, bool hirows, int variant) {
   switch (variant) {
-    case 1: return pick_stages<true, false>(nstage, hirows);
-    case 2: return pick_stages<false, true>(nstage, hirows);
-    default: return pick_stages<false, false>(nstage, hirows);
+    case 1: return pick_stages<true, false, false>(nstage, hirows);
+    case 2: return pick_stages<false, true, false>(nstage, hirows);
+    case 3: return pick_stages<false, false, true>(nstage, hirows);
+    default: return pick_stages<false, false, false>(nstage, hirows);
   }
 }
 
-// ensure_smem_limit / occupancy cache slots 12..29, one per kernel (compress and the dense kernel
+// ensure_smem_limit / occupancy cache slots 12..35, one per kernel (compress and the dense kernel
 // use 0..9)
 int sparse_slot(int nstage, bool hirows, int variant) { return 12 + 6 * variant + 2 * (nstage - 2) + (hirows ? 1 : 0); }
 
@@ -818,12 +851,12 @@ int sms_of_current_device() {
 
 // resident CTAs per SM, cached per (device, kernel, smem) so that planning stays capture-safe
 cudaError_t resident_ctas(SparseFn fn, int slot, int smem, int *per_sm) {
-  static int cache_smem[64][32];
-  static int cache_val[64][32];
+  static int cache_smem[64][kKernelSlots];
+  static int cache_val[64][kKernelSlots];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const bool cacheable = dev >= 0 && dev < 64 && slot >= 0 && slot < 32;
+  const bool cacheable = dev >= 0 && dev < 64 && slot >= 0 && slot < kKernelSlots;
   if (cacheable && cache_smem[dev][slot] == smem && cache_val[dev][slot] > 0) {
     *per_sm = cache_val[dev][slot];
     return cudaSuccess;

@@ -12,7 +12,9 @@ namespace mustafar {
 // Record the message mustafar_last_error() returns on this thread.
 void set_last_error(const char *msg);
 
-// Set a kernel's dynamic shared-memory limit once per device.
+// Set a kernel's dynamic shared-memory limit once per device; `slot` (< kKernelSlots) names the
+// kernel in the per-device caches.
+constexpr int kKernelSlots = 48;
 cudaError_t ensure_smem_limit(const void *kernel, int slot, int bytes);
 
 // Keep count of every kv head of one cache, and where each stream's packed values start: stream
@@ -28,12 +30,21 @@ struct HeadKeep {
   }
 };
 
+// Selection rule of a cache (mustafar_cache_t::pattern).
+enum class Pattern { kTopK = 0, k24 = 1, kChannel = 2 };
+
+// Tokens a window of n tokens keeps in every channel of a channel-wise cache, F being the prune
+// count of a full 16-token window.
+__host__ __device__ __forceinline__ int window_keep(int n, int F) { return n - (n * F) / 16; }
+
+// window (channel-wise caches): fp16 [B][H][16][128] dense copy of each stream's newest window;
+// chF: the prune count F of a full window.
 cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
                             const HeadKeep &hk, int kmax, int cap, uint32_t *bitmap, uint16_t *values,
-                            uint32_t *tile_offset, bool p24, cudaStream_t stream);
+                            uint32_t *tile_offset, Pattern pat, uint16_t *window, int chF, cudaStream_t stream);
 cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32_t *pos, int B, int H,
                           const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
-                          bool p24, cudaStream_t stream);
+                          Pattern pat, uint16_t *window, int chF, cudaStream_t stream);
 
 struct DecodeParams {
   const uint16_t *q;  // [B][Hq][128]
@@ -46,6 +57,8 @@ struct DecodeParams {
   HeadKeep hk_k, hk_v;  // per kv head keep counts and value placement
   int perhead;          // either cache has a keep count per kv head
   int p24_k, p24_v;     // the cache is 2:4-pruned (the fused step appends with that rule)
+  uint16_t *kwin, *vwin;  // channel-wise caches: the dense newest-window copies (else nullptr)
+  int chF_k, chF_v;       // channel-wise caches: the prune count F of a full 16-token window
   // dense caches (baseline kernel), [B][Hkv][cap][128]
   const uint16_t *kd;
   const uint16_t *vd;
@@ -77,7 +90,8 @@ struct DecodePlan {
   int stage_bytes;
   int warp_bytes;
   int smem_bytes;
-  int variant;  // sparse kernel: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4
+  int variant;  // sparse kernel: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4,
+                // 3 token runs located by popcount prefixes (a channel-wise cache)
 };
 
 // Dense fp16 baseline: plan (split count, pipeline depth, shared memory) and launch.
@@ -88,7 +102,7 @@ cudaError_t launch_dense(const DecodeParams &p, const DecodePlan &plan, cudaStre
 
 // Sparse decode over the compressed caches (one wave of CTAs over the end-to-end chunk sequence):
 // plan->splits holds the CTA count.
-// variant: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4
+// variant: as DecodePlan::variant
 cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, int variant,
                         DecodePlan *plan);
 cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream);

@@ -15,6 +15,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace mustafar {
 
@@ -184,6 +185,109 @@ __device__ __forceinline__ void warp_compress_vector_24(const uint16_t *src, uin
   for (int w = 0; w < kWords; ++w) {
     if ((bm[w] >> lane) & 1u) val_dst[prefix + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[w]);
     prefix += __popc(bm[w]);
+  }
+}
+
+// ---- channel-wise pruning (the channel direction of the README's K/V [t/c] naming): each channel
+// of a stream is pruned across the tokens of a 16-token window.  A window of n tokens keeps, in
+// every channel, its window_keep(n, F) largest keys, the lower token index first on ties.
+
+// Descending bitonic sort of 16 keys (every index is a compile-time constant once unrolled).
+__device__ __forceinline__ void sort16_desc(uint32_t (&a)[16]) {
+#pragma unroll
+  for (int k = 2; k <= 16; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const uint32_t hi = max(a[i], a[l]), lo = min(a[i], a[l]);
+          a[i] = (i & k) == 0 ? hi : lo;
+          a[l] = (i & k) == 0 ? lo : hi;
+        }
+      }
+    }
+  }
+}
+
+// One warp prunes and compresses one window of n (1..16) tokens of a stream, channel-wise.
+// src(t) points at token t's 128 fp16 channels (device memory).  Writes the n tokens' bitmap rows
+// from bm_dst (4 words a token) and the window's packed values from val_dst, token after token,
+// each token's kept channels in ascending order.  When win_dst is not null, tokens win_from .. n-1
+// are also copied, dense, to win_dst + 128 t.  Lane l holds channels l, l+32, l+64, l+96 of every
+// token, so a ballot over one of them is one bitmap word.  All 32 lanes must call it.
+template <class Src>
+__device__ __forceinline__ void warp_compress_window(Src src, int n, int F, uint32_t *bm_dst, uint16_t *val_dst,
+                                                     uint16_t *win_dst, int win_from, int lane) {
+  const int kc = window_keep(n, F);
+  const uint32_t valid = n >= 16 ? 0xFFFFu : (1u << n) - 1u;
+  uint32_t raw[16][kWords];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    if (t < n) {
+      const uint16_t *row = src(t);
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) raw[t][w] = row[32 * w + lane];
+    } else {
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) raw[t][w] = 0u;
+    }
+  }
+  if (win_dst != nullptr) {
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      if (t >= win_from && t < n) {
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) win_dst[kHeadDim * t + 32 * w + lane] = static_cast<uint16_t>(raw[t][w]);
+      }
+  }
+  // per channel: bit t of kept[w] marks token t of channel 32w + lane as kept.  Keys are shifted
+  // up by one so that the missing tokens of a short window (key 0) sort below every real one.
+  uint32_t kept[kWords];
+#pragma unroll
+  for (int w = 0; w < kWords; ++w) {
+    uint32_t a[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) a[t] = t < n ? (raw[t][w] & 0x7FFFu) + 1u : 0u;
+    sort16_desc(a);
+    uint32_t T = a[0];  // the kc-th largest key
+#pragma unroll
+    for (int i = 1; i < 16; ++i) T = i == kc - 1 ? a[i] : T;
+    uint32_t gt = 0u, eq = 0u;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const uint32_t key = (raw[t][w] & 0x7FFFu) + 1u;
+      gt |= (key > T ? 1u : 0u) << t;
+      eq |= (key == T ? 1u : 0u) << t;
+    }
+    gt &= valid;
+    eq &= valid;
+    int need = kc - __popc(gt);  // keys equal to T that survive, lowest tokens first
+    uint32_t take = gt;
+    while (eq != 0u && need > 0) {
+      const uint32_t low = eq & (0u - eq);
+      take |= low;
+      eq ^= low;
+      --need;
+    }
+    kept[w] = take;
+  }
+  const uint32_t below = (1u << lane) - 1u;
+  int pre = 0;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    if (t < n) {  // n is the same in every lane
+      uint32_t bm[kWords];
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) bm[w] = __ballot_sync(0xffffffffu, (kept[w] >> t) & 1u);
+      if (lane < kWords) bm_dst[kWords * t + lane] = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) {
+        if ((bm[w] >> lane) & 1u) val_dst[pre + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[t][w]);
+        pre += __popc(bm[w]);
+      }
+    }
   }
 }
 

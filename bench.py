@@ -321,7 +321,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--suite", default=None, help="write the workload-shape suite (JSONL) to this path and exit")
-    ap.add_argument("--suite-parts", default="c1,c3,c4,heads,p24,sweep")
+    ap.add_argument("--suite-parts", default="c1,c3,c4,heads,p24,channel,sweep")
     ap.add_argument("--profile-launches", type=int, default=0,
                     help="ncu case: build the workload, run this many eager fused steps over the rotated "
                          "caches, and exit without timing")

@@ -677,19 +677,10 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
             const int keep = kside ? keep_of<PERHEAD>(P.hk_k, P.keep_k, st.g) : keep_of<PERHEAD>(P.hk_v, P.keep_v, st.g);
             const int64_t base = kside ? base_of<PERHEAD>(P.hk_k, P.keep_k, st.b, st.g, P.Hkv, capx)
                                        : base_of<PERHEAD>(P.hk_v, P.keep_v, st.b, st.g, P.Hkv, capx);
-            const int64_t sid = static_cast<int64_t>(st.b) * P.Hkv + st.g;
-            uint16_t *win = SCAN ? (kside ? P.kwin : P.vwin) : nullptr;
-            if (SCAN && win != nullptr) {
-              // channel-wise cache: the new token joins its window's dense copy and the whole window
-              // (which is this chunk) is pruned again
-              const int r = p % kWindowTokens, tw = p - r;
-              win += sid * kWindowTokens * kHeadDim;
-              uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + (sid * capx + tw) * kWords;
-              uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(tw) * keep;
-              const uint16_t *wsrc = win;
-              warp_compress_window([=](int t) -> const uint16_t * { return t < r ? wsrc + t * kHeadDim : src; }, r + 1,
-                                   kside ? P.chF_k : P.chF_v, bm, vals, win, r, lane);
-            } else {
+            // a channel-wise cache got its new token from a separate launch before this one (its whole
+            // window is pruned again, which would weigh on this kernel's registers)
+            if (!SCAN || (kside ? P.kwin : P.vwin) == nullptr) {
+              const int64_t sid = static_cast<int64_t>(st.b) * P.Hkv + st.g;
               uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + (sid * capx + p) * kWords;
               uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
               if (kside ? P.p24_k : P.p24_v)

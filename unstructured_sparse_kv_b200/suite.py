@@ -21,8 +21,10 @@ FLUSH_BYTES = 256 << 20
 
 
 class Timer:
-    """Median of single launches, each after a read of a buffer larger than L2.  The flush only
-    reads (its lines stay clean), so the timed launch pays no write-back of flush data."""
+    """Median of single calls, each after a read of a buffer larger than L2.  The flush only reads
+    (its lines stay clean), so the timed call pays no write-back of flush data.  A short device
+    sleep after the flush keeps the GPU busy while the host enqueues the timed call, so that host
+    time spent between the call's launches never shows up as device idle time inside the events."""
 
     def __init__(self, device):
         self.flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
@@ -33,6 +35,7 @@ class Timer:
         times = []
         for _ in range(reps):
             torch.amax(self.flush)
+            torch.cuda._sleep(200_000)  # about 100 us at the B200's clocks
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             fn()
@@ -98,16 +101,18 @@ def decode_point(timer, peak, Hq, Hkv, B, L, sK, sV, seed, with_dense=True, patt
     return rec
 
 
-def compress_point(timer, peak, B, L, H, s, seed):
+def compress_point(timer, peak, B, L, H, s, seed, pattern="topk"):
     dev = "cuda"
     g = torch.Generator(device=dev)
     g.manual_seed(seed)
     x = torch.randn(B, L, H, D, generator=g, device=dev).to(torch.float16)  # [B, L, H, d] storage
-    c = M.CompressedCache(B, H, L, s)
+    c = M.CompressedCache(B, H, L, s, pattern=pattern)
     view = x.permute(0, 2, 1, 3)
     t = timer.median_us(lambda: M.mustafar_compress(view, L, s, c))
-    nbytes = 2 * B * L * H * D + c.nbytes()
-    rec = {"kind": "compress", "batch": B, "tokens": L, "kv_heads": H, "sparsity": s, "keep": c.keep, "us": t,
+    # dense read + compressed arrays written (a full-window prefill writes no window copy)
+    nbytes = 2 * B * L * H * D + c.nbytes() - (c.window.numel() * 2 if c.window is not None else 0)
+    rec = {"kind": "compress", "pattern": pattern, "batch": B, "tokens": L, "kv_heads": H, "sparsity": s,
+           "keep": c.keep, "us": t,
            "bytes_read_plus_written": nbytes, "gbs": nbytes / t / 1e3, "frac_of_peak": nbytes / t / 1e3 / peak,
            "compressed_bytes": c.nbytes(), "compressed_fraction_of_dense": c.nbytes() / (2 * B * L * H * D)}
     del x, c
@@ -115,7 +120,35 @@ def compress_point(timer, peak, B, L, H, s, seed):
     return rec
 
 
-def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "p24", "sweep"), log=print):
+def step_point(timer, peak, Hq, Hkv, B, L, s, seed, pattern="topk"):
+    """One fused decode step (compress the new K/V token into slot L, attend over L + 1 tokens)."""
+    dev = "cuda"
+    cap = ((L + 1 + 63) // 64) * 64
+    K = synth.keys(B, Hkv, L, D, seed, dev, capacity=cap)
+    V = synth.values(B, Hkv, L, D, seed, dev, capacity=cap)
+    q = synth.queries(B, Hq, D, seed, dev)
+    kc = M.CompressedCache(B, Hkv, cap, s, pattern=pattern)
+    vc = M.CompressedCache(B, Hkv, cap, s, pattern=pattern)
+    M.mustafar_compress(K, L, s, kc)
+    M.mustafar_compress(V, L, s, vc)
+    kn, vn = synth.step_tokens(B, Hkv, D, seed, 0, dev)
+    pos = torch.full((B,), L, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, L + 1), dtype=torch.uint8, device=dev)
+    # the same slot every time: a repeated step writes the same bytes
+    t = timer.median_us(lambda: M.mustafar_decode_step(q, kn, vn, pos, kc, vc, L + 1, 1.0, out=out, lse=lse,
+                                                       workspace=ws))
+    nb = decode_bytes(B, Hq, Hkv, L + 1, kc.keep, vc.keep)
+    rec = {"kind": "decode_step", "pattern": pattern, "q_heads": Hq, "kv_heads": Hkv, "batch": B, "context": L + 1,
+           "sparsity": s, "keep_k": kc.keep, "keep_v": vc.keep, "step_us": t, "bytes": nb,
+           "gbs": nb / t / 1e3, "frac_of_peak": nb / t / 1e3 / peak}
+    del K, V, kc, vc
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "p24", "channel", "sweep"), log=print):
     torch.cuda.set_device(0)
     timer = Timer("cuda")
     recs = []
@@ -147,6 +180,19 @@ def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "p24", "sw
                       workload=f"b{B} ctx{L} 2:4"))
             emit(dict(decode_point(timer, peak, 32, 8, B, L, 0.5, 0.5, 1008, with_dense=False),
                       workload=f"b{B} ctx{L} unstructured s0.5 (same inputs)"))
+    if "channel" in which:
+        # channel-wise pruning over 16-token windows against token-wise pruning on the same inputs
+        # (keep 40 vs 39 values per token at s = 0.7)
+        for B, L in ((8, 4096), (4, 32768)):
+            emit(dict(decode_point(timer, peak, 32, 8, B, L, 0.7, 0.7, 1010, pattern="channel"),
+                      workload=f"b{B} ctx{L} channel-wise s0.7"))
+            emit(dict(decode_point(timer, peak, 32, 8, B, L, 0.7, 0.7, 1010, with_dense=False),
+                      workload=f"b{B} ctx{L} token-wise s0.7 (same inputs)"))
+        for pattern in ("channel", "topk"):
+            emit(dict(step_point(timer, peak, 32, 8, 8, 4096, 0.7, 1010, pattern=pattern),
+                      workload=f"fused decode step b8 ctx4096 s0.7 {pattern}"))
+        emit(dict(compress_point(timer, peak, 8, 16384, 8, 0.7, 1004, pattern="channel"),
+                  workload="compress b8 16k h8 channel-wise"))
     if "sweep" in which:
         for Hkv in (8, 32):
             for B in (1, 8, 32):

@@ -310,19 +310,19 @@ mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *w
   const size_t cnt = ((static_cast<size_t>(p.B) * p.Hkv * 4 + 255) / 256) * 256;
   p.ws_cnt = reinterpret_cast<uint32_t *>(w);
   p.ws_part = reinterpret_cast<float *>(w + cnt);
-  if (p.pos != nullptr) {
-    // a decode step: a channel-wise cache takes its new token in a launch of its own before the
-    // attention (its whole newest window is pruned again); the attention kernel appends the rest
-    if (p.kwin != nullptr) {
-      e = launch_append(p.kn, p.kn_sb, p.kn_sh, p.pos, p.B, p.Hkv, p.hk_k, p.cap_k, const_cast<uint32_t *>(p.kbm),
-                        const_cast<uint16_t *>(p.kval), p.err, Pattern::kChannel, p.kwin, p.chF_k, stream);
-      if (e != cudaSuccess) return cuda_fail(e, name);
-    }
-    if (p.vwin != nullptr) {
-      e = launch_append(p.vn, p.vn_sb, p.vn_sh, p.pos, p.B, p.Hkv, p.hk_v, p.cap_v, const_cast<uint32_t *>(p.vbm),
-                        const_cast<uint16_t *>(p.vval), p.err, Pattern::kChannel, p.vwin, p.chF_v, stream);
-      if (e != cudaSuccess) return cuda_fail(e, name);
-    }
+  if (p.pos != nullptr && (p.kwin != nullptr || p.vwin != nullptr)) {
+    // a decode step: the channel-wise caches take their new token in one launch of their own before
+    // the attention (each newest window is pruned again); the attention kernel appends the rest
+    ChannelAppend c[2];
+    int n = 0;
+    if (p.kwin != nullptr)
+      c[n++] = ChannelAppend{p.kn, p.kn_sb, p.kn_sh, p.keep_k, p.chF_k, p.cap_k, const_cast<uint32_t *>(p.kbm),
+                             const_cast<uint16_t *>(p.kval), p.kwin};
+    if (p.vwin != nullptr)
+      c[n++] = ChannelAppend{p.vn, p.vn_sb, p.vn_sh, p.keep_v, p.chF_v, p.cap_v, const_cast<uint32_t *>(p.vbm),
+                             const_cast<uint16_t *>(p.vval), p.vwin};
+    e = launch_append_channel(c, n, p.pos, p.B, p.Hkv, p.err, stream);
+    if (e != cudaSuccess) return cuda_fail(e, name);
   }
   e = launch_sparse(p, plan, stream);
   return e == cudaSuccess ? MUSTAFAR_OK : cuda_fail(e, name);

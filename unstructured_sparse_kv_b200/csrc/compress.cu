@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(128)
 compress_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, int keep,
                         int F, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
                         uint32_t *__restrict__ tile_offset, uint16_t *__restrict__ window) {
+  __shared__ uint32_t scratch[4][128];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t stream = static_cast<int64_t>(b) * H + h;
@@ -147,30 +148,45 @@ compress_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, 
   const uint16_t *xs = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh + static_cast<int64_t>(t0) * st;
   uint16_t *win = n < kWindowTokens ? window + stream * kWindowTokens * kHeadDim : nullptr;
   warp_compress_window([=](int t) { return xs + static_cast<int64_t>(t) * st; }, n, F,
-                       bitmap + (stream * cap + t0) * kWords, values + (stream * cap + t0) * keep, win, 0, lane);
+                       bitmap + (stream * cap + t0) * kWords, values + (stream * cap + t0) * keep, win, 0,
+                       scratch[warp], lane);
 }
 
-// Channel-wise append: one warp per (b, kv head).  The new token goes to slot pos % 16 of the
-// stream's window copy, and the window (tokens 16*floor(pos/16) .. pos) is pruned again.
+// Channel-wise append: one warp per (cache, b, kv head), for one or two caches (a decode step's K
+// and V) in one launch.  The new token goes to slot pos % 16 of the stream's window copy, and the
+// window (tokens 16*floor(pos/16) .. pos) is pruned again.
 __global__ void __launch_bounds__(128)
-append_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int32_t *__restrict__ pos, int B,
-                      int H, int keep, int F, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
-                      uint16_t *window, uint32_t *__restrict__ err) {
+append_channel_kernel(const ChannelAppend c0, const ChannelAppend c1, const int32_t *__restrict__ pos, int B, int H,
+                      int ncaches, uint32_t *__restrict__ err) {
+  __shared__ uint32_t scratch[4][128];
   const int lane = threadIdx.x & 31;
-  const int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (v >= B * H) return;
+  int v = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (v >= ncaches * B * H) return;
+  const bool second = v >= B * H;
+  const ChannelAppend &c = second ? c1 : c0;
+  v -= second ? B * H : 0;
   const int b = v / H, h = v - b * H;
   const int p = pos[b];
-  if (p < 0 || p >= cap) {
+  if (p < 0 || p >= c.cap) {
     if (lane == 0 && err != nullptr) atomicOr(err, MUSTAFAR_DEVERR_POS_RANGE);
     return;
   }
   const int r = p % kWindowTokens, t0 = p - r;
   const int64_t stream = static_cast<int64_t>(b) * H + h;
-  const uint16_t *xn = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
-  uint16_t *win = window + stream * kWindowTokens * kHeadDim;
-  warp_compress_window([=](int t) -> const uint16_t * { return t < r ? win + t * kHeadDim : xn; }, r + 1, F,
-                       bitmap + (stream * cap + t0) * kWords, values + (stream * cap + t0) * keep, win, r, lane);
+  const uint16_t *xn = c.x + static_cast<int64_t>(b) * c.sb + static_cast<int64_t>(h) * c.sh;
+  uint16_t *win = c.window + stream * kWindowTokens * kHeadDim;
+  warp_compress_window([=](int t) -> const uint16_t * { return t < r ? win + t * kHeadDim : xn; }, r + 1, c.F,
+                       c.bitmap + (stream * c.cap + t0) * kWords, c.values + (stream * c.cap + t0) * c.keep, win, r,
+                       scratch[threadIdx.x >> 5], lane);
+}
+
+cudaError_t launch_append_channel(const ChannelAppend *c, int ncaches, const int32_t *pos, int B, int H,
+                                  uint32_t *err, cudaStream_t stream) {
+  const int threads = 128;  // 4 windows per CTA
+  const int warps = ncaches * B * H;
+  append_channel_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(
+      c[0], ncaches > 1 ? c[1] : c[0], pos, B, H, ncaches, err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_compress(const uint16_t *x, int64_t sb, int64_t sh, int64_t st, int L, int B, int H,
@@ -201,9 +217,8 @@ cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32
   const int warps = B * H;
   const int threads = 128;  // 4 vectors per CTA
   if (pat == Pattern::kChannel) {
-    append_channel_kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(
-        x, sb, sh, pos, B, H, hk.k[0], chF, cap, bitmap, values, window, err);
-    return cudaGetLastError();
+    const ChannelAppend c{x, sb, sh, hk.k[0], chF, cap, bitmap, values, window};
+    return launch_append_channel(&c, 1, pos, B, H, err, stream);
   }
   auto kernel = pat == Pattern::k24 ? append_kernel<true> : append_kernel<false>;
   kernel<<<(warps * 32 + threads - 1) / threads, threads, 0, stream>>>(x, sb, sh, pos, B, H, hk, cap, bitmap,

@@ -46,6 +46,20 @@ cudaError_t launch_append(const uint16_t *x, int64_t sb, int64_t sh, const int32
                           const HeadKeep &hk, int cap, uint32_t *bitmap, uint16_t *values, uint32_t *err,
                           Pattern pat, uint16_t *window, int chF, cudaStream_t stream);
 
+// One channel-wise cache's share of an append launch: the new tokens (x, strided [B][H][128]) and
+// the cache arrays; F is the prune count of a full window.
+struct ChannelAppend {
+  const uint16_t *x;
+  int64_t sb, sh;
+  int keep, F, cap;
+  uint32_t *bitmap;
+  uint16_t *values;
+  uint16_t *window;
+};
+// Append one token per (b, kv head) to each of `ncaches` (1 or 2) channel-wise caches in one launch.
+cudaError_t launch_append_channel(const ChannelAppend *c, int ncaches, const int32_t *pos, int B, int H,
+                                  uint32_t *err, cudaStream_t stream);
+
 struct DecodeParams {
   const uint16_t *q;  // [B][Hq][128]
   // compressed caches (sparse kernel)

@@ -215,41 +215,37 @@ __device__ __forceinline__ void sort16_desc(uint32_t (&a)[16]) {
 // src(t) points at token t's 128 fp16 channels (device memory).  Writes the n tokens' bitmap rows
 // from bm_dst (4 words a token) and the window's packed values from val_dst, token after token,
 // each token's kept channels in ascending order.  When win_dst is not null, tokens win_from .. n-1
-// are also copied, dense, to win_dst + 128 t.  Lane l holds channels l, l+32, l+64, l+96 of every
-// token, so a ballot over one of them is one bitmap word.  All 32 lanes must call it.
+// are also copied, dense, to win_dst + 128 t.  `scratch` is 128 words of this warp's shared
+// memory.  Lane l holds channels l, l+32, l+64, l+96 of every token, so a ballot over one of them
+// is one bitmap word.  All 32 lanes must call it.
+// The loops over words and tokens stay rolled: the routine often runs once per warp (an append),
+// where a long unrolled body would be fetched from a cold instruction cache.
 template <class Src>
 __device__ __forceinline__ void warp_compress_window(Src src, int n, int F, uint32_t *bm_dst, uint16_t *val_dst,
-                                                     uint16_t *win_dst, int win_from, int lane) {
+                                                     uint16_t *win_dst, int win_from, uint32_t *scratch, int lane) {
   const int kc = window_keep(n, F);
   const uint32_t valid = n >= 16 ? 0xFFFFu : (1u << n) - 1u;
-  uint32_t raw[16][kWords];
-#pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    if (t < n) {
-      const uint16_t *row = src(t);
-#pragma unroll
-      for (int w = 0; w < kWords; ++w) raw[t][w] = row[32 * w + lane];
-    } else {
-#pragma unroll
-      for (int w = 0; w < kWords; ++w) raw[t][w] = 0u;
-    }
+  // the window's rows (two 128-byte lines each) are requested up front
+  if (lane < 2 * n) {
+    const uint16_t *line = src(lane >> 1) + 64 * (lane & 1);
+    asm volatile("prefetch.global.L1 [%0];\n" ::"l"(line));
   }
-  if (win_dst != nullptr) {
-#pragma unroll
-    for (int t = 0; t < 16; ++t)
-      if (t >= win_from && t < n) {
-#pragma unroll
-        for (int w = 0; w < kWords; ++w) win_dst[kHeadDim * t + 32 * w + lane] = static_cast<uint16_t>(raw[t][w]);
-      }
-  }
-  // per channel: bit t of kept[w] marks token t of channel 32w + lane as kept.  Keys are shifted
-  // up by one so that the missing tokens of a short window (key 0) sort below every real one.
-  uint32_t kept[kWords];
-#pragma unroll
+  // 1. per channel: sort the window's keys, keep the kc largest (lower token on ties).
+  //    Bit 16w + t of `kept`: token t of channel 32w + lane is kept.
+  uint64_t kept = 0u;
+#pragma unroll 1
   for (int w = 0; w < kWords; ++w) {
-    uint32_t a[16];
+    uint32_t key[16], a[16];
+    uint16_t xs[16];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) a[t] = t < n ? (raw[t][w] & 0x7FFFu) + 1u : 0u;
+    for (int t = 0; t < 16; ++t) xs[t] = src(min(t, n - 1))[32 * w + lane];  // all 16 loads in flight at once
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      // keys are shifted up by one so that the missing tokens of a short window (0) sort last
+      key[t] = t < n ? (xs[t] & 0x7FFFu) + 1u : 0u;
+      a[t] = key[t];
+      if (win_dst != nullptr && t >= win_from && t < n) win_dst[kHeadDim * t + 32 * w + lane] = xs[t];
+    }
     sort16_desc(a);
     uint32_t T = a[0];  // the kc-th largest key
 #pragma unroll
@@ -257,9 +253,8 @@ __device__ __forceinline__ void warp_compress_window(Src src, int n, int F, uint
     uint32_t gt = 0u, eq = 0u;
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
-      const uint32_t key = (raw[t][w] & 0x7FFFu) + 1u;
-      gt |= (key > T ? 1u : 0u) << t;
-      eq |= (key == T ? 1u : 0u) << t;
+      gt |= (key[t] > T ? 1u : 0u) << t;
+      eq |= (key[t] == T ? 1u : 0u) << t;
     }
     gt &= valid;
     eq &= valid;
@@ -271,24 +266,45 @@ __device__ __forceinline__ void warp_compress_window(Src src, int n, int F, uint
       eq ^= low;
       --need;
     }
-    kept[w] = take;
+    kept |= static_cast<uint64_t>(take) << (16 * w);
   }
+  // 2. bitmap words by ballot, and where each (token, word) run starts: scratch[4t + w] holds the
+  //    word, scratch[64 + 4t + w] the run start within the window
+  uint32_t pre = 0u;
+#pragma unroll 1
+  for (int t = 0; t < n; ++t) {  // n is the same in every lane
+    uint32_t bm[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) bm[w] = __ballot_sync(0xffffffffu, (kept >> (16 * w + t)) & 1u);
+    if (lane < kWords) {
+      const uint32_t mine = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
+      const uint32_t before = lane == 0 ? 0u
+                              : lane == 1 ? __popc(bm[0])
+                              : lane == 2 ? __popc(bm[0]) + __popc(bm[1])
+                                          : __popc(bm[0]) + __popc(bm[1]) + __popc(bm[2]);
+      bm_dst[kWords * t + lane] = mine;
+      scratch[kWords * t + lane] = mine;
+      scratch[64 + kWords * t + lane] = pre + before;
+    }
+    pre += __popc(bm[0]) + __popc(bm[1]) + __popc(bm[2]) + __popc(bm[3]);
+  }
+  __syncwarp();
+  // 3. the kept values, one word (32 channels) of every token at a time
   const uint32_t below = (1u << lane) - 1u;
-  int pre = 0;
+#pragma unroll 1
+  for (int w = 0; w < kWords; ++w) {
+    uint16_t xs[16];
 #pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    if (t < n) {  // n is the same in every lane
-      uint32_t bm[kWords];
+    for (int t = 0; t < 16; ++t) xs[t] = src(min(t, n - 1))[32 * w + lane];  // all in flight at once
 #pragma unroll
-      for (int w = 0; w < kWords; ++w) bm[w] = __ballot_sync(0xffffffffu, (kept[w] >> t) & 1u);
-      if (lane < kWords) bm_dst[kWords * t + lane] = lane == 0 ? bm[0] : lane == 1 ? bm[1] : lane == 2 ? bm[2] : bm[3];
-#pragma unroll
-      for (int w = 0; w < kWords; ++w) {
-        if ((bm[w] >> lane) & 1u) val_dst[pre + __popc(bm[w] & below)] = static_cast<uint16_t>(raw[t][w]);
-        pre += __popc(bm[w]);
+    for (int t = 0; t < 16; ++t) {
+      if (t < n) {
+        const uint32_t word = scratch[kWords * t + w];
+        if ((word >> lane) & 1u) val_dst[scratch[64 + kWords * t + w] + __popc(word & below)] = xs[t];
       }
     }
   }
+  __syncwarp();  // the scratch may be reused by the caller's next window
 }
 
 }  // namespace mustafar

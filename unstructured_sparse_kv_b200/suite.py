@@ -190,7 +190,7 @@ def run(out_path: str, peak: float, which=("c1", "c3", "c4", "heads", "p24", "ch
                       workload=f"b{B} ctx{L} token-wise s0.7 (same inputs)"))
         for pattern in ("channel", "topk"):
             emit(dict(step_point(timer, peak, 32, 8, 8, 4096, 0.7, 1010, pattern=pattern),
-                      workload=f"fused decode step b8 ctx4096 s0.7 {pattern}"))
+                      workload=f"decode step call b8 ctx4096 s0.7 {pattern}"))
         emit(dict(compress_point(timer, peak, 8, 16384, 8, 0.7, 1004, pattern="channel"),
                   workload="compress b8 16k h8 channel-wise"))
     if "sweep" in which:

@@ -129,6 +129,8 @@ def test_append_rows_at_different_positions_and_out_of_range():
     (2, 8, 1, 1, 0.7, 0.7, 0, False),      # one token
     (2, 12, 4, 129, 0.0, 0.0, 2, True),    # sparsity 0: plain attention
     (1, 8, 8, 1000, 0.995, 0.995, 0, False),  # keep = 1
+    (2, 8, 2, 200, 0.25, 0.0, 0, True),    # keeps 96 and 128: runs staged token by token
+    (2, 8, 2, 150, 0.25, 0.7, 2, True),    # one cache staged token by token, one in a single copy
 ])
 def test_decode_small_cases(B, Hq, Hkv, L, sK, sV, splits, ragged):
     cap = ((L + 63) // 64) * 64

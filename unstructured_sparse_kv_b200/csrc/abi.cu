@@ -301,6 +301,10 @@ mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *w
   if (e != cudaSuccess) return cuda_fail(e, name);
   p.stage_bytes = plan.stage_bytes;
   p.warp_bytes = plan.warp_bytes;
+  p.lg_k = plan.lg_k;
+  p.lg_v = plan.lg_v;
+  p.skew_k = plan.skew_k;
+  p.skew_v = plan.skew_v;
   const size_t need = sparse_workspace_bytes(p.B, p.Hkv, p.G, plan.splits);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(MUSTAFAR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed (%d CTAs), got %zu", name, need,

@@ -176,7 +176,7 @@ __device__ __forceinline__ void load_q(const DecodeParams &P, int b, int g, int 
 // per-row half-word prefix table.  SCAN: token runs of varying length (a channel-wise cache), each
 // found by the kept counts of the tokens before it in the chunk; otherwise token T's run starts at
 // T*keep.
-template <bool HIROWS, bool PERHEAD, bool P24, bool SCAN>
+template <bool HIROWS, bool PERHEAD, bool P24, bool SCAN, bool SKEW>
 __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *stage, uint8_t *htab, uint32_t za,
                                               int t0, int L, int kKh, int kVh, int lane, const uint32_t (&qa)[8][4],
                                               Acc<HIROWS> &acc, const uint2 *lut24) {
@@ -232,8 +232,9 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
     if constexpr (P24) {
       // word qq's 16 values: 32 contiguous bytes of the token's 128-byte run, nibble j's two in value
       // pair j; placed into channel pairs (4j, 4j+1), (4j+2, 4j+3) by the nibble's two selectors
-      const uint4 va = *reinterpret_cast<const uint4 *>(stage + 512 + T * 128 + qq * 32);
-      const uint4 vb = *reinterpret_cast<const uint4 *>(stage + 512 + T * 128 + qq * 32 + 16);
+      const uint8_t *run = stage + 512 + T * 128 + (SKEW ? (T >> P.lg_k) << 4 : 0);
+      const uint4 va = *reinterpret_cast<const uint4 *>(run + qq * 32);
+      const uint4 vb = *reinterpret_cast<const uint4 *>(run + qq * 32 + 16);
       const uint32_t x[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -243,7 +244,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
       }
     } else {
       const uint32_t pre = *reinterpret_cast<const uint32_t *>(htab + T * 16 + qq * 4);  // halves 2q, 2q+1
-      const uint32_t rbase = SCAN ? kvals : kvals + 2 * T * kK;
+      const uint32_t rbase = SCAN ? kvals : kvals + 2 * T * kK + (SKEW ? (T >> P.lg_k) << 4 : 0);
       expand_word(word, rbase + 2 * (pre & 0xFFFFu), rbase + 2 * (pre >> 16), za, kb);
     }
 #pragma unroll
@@ -317,7 +318,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
 
   // ---- O^T += V~^T P^T : 8 m-tiles of 16 channels.  This lane's A fragments cover channels
   // 16g..16g+15 (half word g of the bitmap) of tokens 2q, 2q+1 and 2q+8, 2q+9.
-  const uint32_t vvals = smem_addr(stage + 512 + 32 * kK);
+  const uint32_t vvals = smem_addr(stage + 512 + 32 * kK + (SKEW ? P.skew_k : 0));
   uint32_t va[8][4];
   if constexpr (P24) {
     // half word gq of each token: 8 values, 16 contiguous bytes at 16*gq in the token's run
@@ -328,7 +329,8 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
       for (int e = 0; e < 2; ++e) {
         const int T = 2 * qq + 8 * pair + e;
         const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
-        const uint4 v = *reinterpret_cast<const uint4 *>(stage + 512 + 2048 + T * 128 + gq * 16);
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + 512 + 2048 + (SKEW ? P.skew_k : 0) + T * 128 +
+                                                         (SKEW ? (T >> P.lg_v) << 4 : 0) + gq * 16);
         const uint32_t x[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -352,7 +354,8 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
         const int T = 2 * qq + 8 * pair + e;
         const uint32_t bits = *reinterpret_cast<const uint16_t *>(stage + 256 + T * 16 + gq * 2);
         const uint32_t pre = *reinterpret_cast<const uint16_t *>(htab + (16 + T) * 16 + gq * 2);
-        expand_half(bits, vvals + 2 * ((SCAN ? 0 : T * kV) + pre), za, e ? x1 : x0);
+        expand_half(bits, vvals + (SCAN ? 0 : 2 * T * kV + (SKEW ? (T >> P.lg_v) << 4 : 0)) + 2 * pre, za,
+                    e ? x1 : x0);
       }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
@@ -564,7 +567,7 @@ __constant__ uint2 kLut24[16] = {
     {0x5454u, 0x5454u}, {0x5410u, 0x3254u}, {0x1054u, 0x3254u}, {0x5454u, 0x5454u},  // 8, 1001, 1010, 11
     {0x5454u, 0x3210u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}, {0x5454u, 0x5454u}};  // 1100, 13, 14, 15
 
-template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24, bool SCAN>
+template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24, bool SCAN, bool SKEW>
 __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
@@ -711,6 +714,40 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   }
   __syncwarp();
   auto produce = [&](int item) {
+    if constexpr (SKEW) {
+      // a cache whose keep is a multiple of 32 is staged in groups of 2^lg tokens (about 256 bytes),
+      // each group 16 bytes after the previous one ends: otherwise every token's run starts on the
+      // same bank and the lanes that read one word position of eight tokens collide.  Lanes 0-15
+      // copy K groups, 16-31 V groups; a cache without skew (lg = 4) arrives in one copy.
+      const int punit = sh_punit[warp];
+      if (punit >= u1) return;  // the same in every lane
+      Stream ps = sh_ps[warp];
+      while (punit >= ps.end()) next_stream(P, cap, ps);
+      const int slot = item % NSTAGE;
+      const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
+      const uint32_t bar = bars + 8 * slot;
+      const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
+      const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
+      const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
+      if (lane == 0) {
+        mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
+        bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+        bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      }
+      __syncwarp();
+      const bool kside = lane < 16;
+      const int g = lane & 15, keep = kside ? P.keep_k : P.keep_v, lg = kside ? P.lg_k : P.lg_v;
+      const uint32_t base = dst + 512 + (kside ? 0 : 32 * P.keep_k + P.skew_k);
+      const uint16_t *src = kside ? P.kval + tk * P.keep_k : P.vval + tv * P.keep_v;
+      if (g < (kChunk >> lg))  // group g: tokens g*2^lg .. (g+1)*2^lg - 1
+        bulk_g2s(base + ((2 * keep) << lg) * g + 16 * g, src + (keep << lg) * g, (2 * keep) << lg, bar);
+      __syncwarp();  // every lane has read the producer state before lane 0 moves it on
+      if (lane == 0) {
+        sh_ps[warp] = ps;
+        sh_punit[warp] = punit + kWarps;
+      }
+      return;
+    }
     if (lane != 0) return;
     int punit = sh_punit[warp];
     if (punit >= u1) return;
@@ -759,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       uint8_t *stage = wbase + slot * P.stage_bytes;
       if (!mbar_wait(bars + 8 * slot, (citem / NSTAGE) & 1, timed_out ? kWaitCyclesAfter : kWaitCycles))
         timed_out = true;
-      consume_chunk<HIROWS, PERHEAD, P24, SCAN>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
+      consume_chunk<HIROWS, PERHEAD, P24, SCAN, SKEW>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
                                           lut24);
       __syncwarp();
       produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
@@ -793,33 +830,35 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
 // ------------------------------------------------------------------------------------ host side
 using SparseFn = void (*)(const DecodeParams);
 
-template <int NSTAGE, bool PERHEAD, bool P24, bool SCAN>
+template <int NSTAGE, bool PERHEAD, bool P24, bool SCAN, bool SKEW>
 SparseFn pick_rows(bool hirows) {
-  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD, P24, SCAN>
-                : sparse_decode_kernel<NSTAGE, false, PERHEAD, P24, SCAN>;
+  return hirows ? sparse_decode_kernel<NSTAGE, true, PERHEAD, P24, SCAN, SKEW>
+                : sparse_decode_kernel<NSTAGE, false, PERHEAD, P24, SCAN, SKEW>;
 }
 
-template <bool PERHEAD, bool P24, bool SCAN>
+template <bool PERHEAD, bool P24, bool SCAN, bool SKEW>
 SparseFn pick_stages(int nstage, bool hirows) {
   switch (nstage) {
-    case 2: return pick_rows<2, PERHEAD, P24, SCAN>(hirows);
-    case 3: return pick_rows<3, PERHEAD, P24, SCAN>(hirows);
-    default: return pick_rows<4, PERHEAD, P24, SCAN>(hirows);
+    case 2: return pick_rows<2, PERHEAD, P24, SCAN, SKEW>(hirows);
+    case 3: return pick_rows<3, PERHEAD, P24, SCAN, SKEW>(hirows);
+    default: return pick_rows<4, PERHEAD, P24, SCAN, SKEW>(hirows);
   }
 }
 
 // variant: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4, 3 token runs found by
-// popcount prefixes (a channel-wise cache; either cache may also be token-wise or 2:4)
+// popcount prefixes (a channel-wise cache; either cache may also be token-wise or 2:4); 4 is 0 with
+// a cache staged in skewed token groups (keep a multiple of 32)
 SparseFn pick_sparse(int nstage, bool hirows, int variant) {
   switch (variant) {
-    case 1: return pick_stages<true, false, false>(nstage, hirows);
-    case 2: return pick_stages<false, true, false>(nstage, hirows);
-    case 3: return pick_stages<false, false, true>(nstage, hirows);
-    default: return pick_stages<false, false, false>(nstage, hirows);
+    case 1: return pick_stages<true, false, false, false>(nstage, hirows);
+    case 2: return pick_stages<false, true, false, false>(nstage, hirows);
+    case 3: return pick_stages<false, false, true, false>(nstage, hirows);
+    case 4: return pick_stages<false, false, false, true>(nstage, hirows);
+    default: return pick_stages<false, false, false, false>(nstage, hirows);
   }
 }
 
-// ensure_smem_limit / occupancy cache slots 12..35, one per kernel (compress and the dense kernel
+// ensure_smem_limit / occupancy cache slots 12..41, one per kernel (compress and the dense kernel
 // use 0..9)
 int sparse_slot(int nstage, bool hirows, int variant) { return 12 + 6 * variant + 2 * (nstage - 2) + (hirows ? 1 : 0); }
 
@@ -894,7 +933,22 @@ size_t sparse_workspace_bound(int B, int Hkv, int G, int max_len, int forced_spl
 cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep_v, int forced_splits, int variant,
                         DecodePlan *plan) {
   const bool hirows = G > 8;
-  const int stage_bytes = round_up(512 + 32 * (keep_k + keep_v), 128);
+  // a uniform or 2:4 cache whose keep is a multiple of 32 is staged token by token with a 16-byte
+  // skew (see the producer); its staged run then takes 2*keep + 16 bytes per token
+  // (not for 2:4: its 128-bit loads see at most 2-way conflicts, and the grouped staging cost more
+  // than it saved there, measured)
+  const bool can_skew = variant == 0;
+  // tokens per staged group, as log2 (4 = the chunk in one copy, no skew).  Only keeps of 96 and 128
+  // are staged token by token: there eight tokens' runs share 1-2 bank offsets; at keep 64 the
+  // grouped copies cost about what the conflicts did (measured: 0.94-1.08x), at 32 and below the
+  // runs are short
+  auto group_lg = [&](int keep) { return can_skew && keep % 32 == 0 && keep >= 96 ? 0 : 4; };
+  plan->lg_k = group_lg(keep_k);
+  plan->lg_v = group_lg(keep_v);
+  plan->skew_k = plan->lg_k < 4 ? 16 * (kChunk >> plan->lg_k) : 0;  // skew bytes added to the region
+  plan->skew_v = plan->lg_v < 4 ? 16 * (kChunk >> plan->lg_v) : 0;
+  if (plan->skew_k || plan->skew_v) variant = 4;
+  const int stage_bytes = round_up(512 + 32 * (keep_k + keep_v) + plan->skew_k + plan->skew_v, 128);
   const int merge_bytes = (2 * kWarps * 16 + kWarps * G * kHeadDim) * 4;
   auto warp_bytes_of = [&](int ns) { return round_up(ns * stage_bytes + 512 + 8 * ns, 128); };
   int nstage = 2;

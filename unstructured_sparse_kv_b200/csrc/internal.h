@@ -82,6 +82,8 @@ struct DecodeParams {
   float scale_log2;
   int num_splits, chunks_per_split;
   int stage_bytes, warp_bytes;
+  int lg_k, lg_v;      // sparse kernel: a cache is staged in groups of 2^lg tokens, 16 B apart (4: one copy)
+  int skew_k, skew_v;  // sparse kernel: bytes those gaps add to the cache's staged region
   uint16_t *out;
   float *lse;
   float *ws_part;     // sparse kernel: [2 * ctas][32 + G*128] partial (m, l, o) slots
@@ -104,6 +106,7 @@ struct DecodePlan {
   int stage_bytes;
   int warp_bytes;
   int smem_bytes;
+  int lg_k, lg_v, skew_k, skew_v;  // sparse kernel: staging groups of a keep that is a multiple of 32
   int variant;  // sparse kernel: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4,
                 // 3 token runs located by popcount prefixes (a channel-wise cache)
 };

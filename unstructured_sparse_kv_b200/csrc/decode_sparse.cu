@@ -862,7 +862,7 @@ SparseFn pick_sparse(int nstage, bool hirows, int variant) {
 // use 0..9)
 int sparse_slot(int nstage, bool hirows, int variant) { return 12 + 6 * variant + 2 * (nstage - 2) + (hirows ? 1 : 0); }
 
-constexpr int kMinUnitsPerCta = 2 * kWarps;  // at least two chunks per warp
+constexpr int kMinUnitsPerCta = kWarps;  // at least one chunk per warp
 constexpr int kMaxCtasPerSm = 4;
 constexpr int kCtaSmemBudget = 56000;        // four CTAs per SM fit in 228 KB with this much each
 
@@ -913,7 +913,12 @@ int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_s
     const long long wave = static_cast<long long>(sms_of_current_device()) * per_sm;
     const long long per_stream = wave / streams;
     ctas = per_stream >= 1 && per_stream * streams * 20 >= wave * 19 ? per_stream * streams : wave;
-    const long long by_len = units / kMinUnitsPerCta;
+    // short rows: about two chunks per warp, but never fewer CTAs than streams (up to a wave): the
+    // four warps of a CTA step through its stream pieces together, so a CTA holding many one-chunk
+    // pieces would run them one after another
+    long long by_len = units / kMinUnitsPerCta;
+    const long long spread = streams < wave ? streams : wave;
+    by_len = by_len > spread ? by_len : spread;
     ctas = by_len < ctas ? by_len : ctas;
   }
   ctas = ctas > units ? units : ctas;

@@ -244,6 +244,30 @@ def test_decode_step_same_bits_as_append_then_attend():
         assert torch.equal(a.bitmap, b.bitmap) and torch.equal(a.values, b.values)
 
 
+def test_prepared_decode_step_matches_direct_calls():
+    # the prepared call runs the same C entry point on buffers whose contents change between steps
+    B, Hq, Hkv, L0, cap = 2, 8, 2, 70, 128
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L0, cap, 0.7, 0.5, 91)
+    kc2, vc2 = M.CompressedCache(B, Hkv, cap, 0.7), M.CompressedCache(B, Hkv, cap, 0.5)
+    for a, b in ((kc, kc2), (vc, vc2)):
+        b.bitmap.copy_(a.bitmap)
+        b.values.copy_(a.values)
+        b.tile_offset.copy_(a.tile_offset)
+    qb, knb, vnb = torch.empty_like(q), torch.empty(B, Hkv, D, dtype=torch.float16, device=DEV), \
+        torch.empty(B, Hkv, D, dtype=torch.float16, device=DEV)
+    posb = torch.empty(B, dtype=torch.int32, device=DEV)
+    call, out_p, lse_p = M.prepare_decode_step(qb, knb, vnb, posb, kc2, vc2, cap, 0.5)
+    for st in range(5):
+        kn, vn = synth.step_tokens(B, Hkv, D, 91, st, DEV)
+        qs = synth.queries(B, Hq, D, 91, DEV, step=st)
+        pos = torch.full((B,), L0 + st, dtype=torch.int32, device=DEV)
+        o1, l1 = M.mustafar_decode_step(qs, kn, vn, pos, kc, vc, cap, 0.5)
+        qb.copy_(qs), knb.copy_(kn), vnb.copy_(vn), posb.copy_(pos)
+        call()
+        assert torch.equal(o1, out_p) and torch.equal(l1, lse_p), f"step {st}"
+    assert torch.equal(kc.values, kc2.values) and torch.equal(vc.bitmap, vc2.bitmap)
+
+
 def test_decode_step_out_of_range_positions():
     B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 23)

@@ -336,12 +336,19 @@ def mustafar_decode_attn_noalloc(q: torch.Tensor, k: CompressedCache, v: Compres
     return out, lse
 
 
-def mustafar_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
-                         k: CompressedCache, v: CompressedCache, max_len: int, scale: float, out=None, lse=None,
-                         workspace=None, num_splits: int = 0, err=None, stream=None, want_lse: bool = True):
-    """One decode step in one launch: compress ``k_new``/``v_new`` ([B, Hkv, d] fp16) into slot
-    ``pos[b]`` of the caches, then attend over the ``pos[b] + 1`` tokens ``[0, pos[b]]``.
-    Returns (out [B,Hq,d] fp16, lse [B,Hq] fp32); ``max_len`` bounds ``pos[b] + 1``."""
+class PreparedCall:
+    """One library call whose arguments were checked and marshalled once.  Calling it runs the C
+    entry point again with the same buffers, shapes and stream (the buffers' contents may change
+    between calls); a serving loop that reuses its buffers saves the per-call Python marshalling."""
+
+    def __init__(self, fn, args, keep_alive):
+        self._fn, self._args, self._keep = fn, args, keep_alive
+
+    def __call__(self) -> None:
+        _check(self._fn(*self._args))
+
+
+def _step_args(q, k_new, v_new, pos, k, v, max_len, scale, out, lse, workspace, num_splits, err, stream, want_lse):
     _cuda_f16(q, "q")
     if not q.is_contiguous() or q.dim() != 3:
         raise ValueError("q must be a contiguous [B, Hq, d] tensor")
@@ -355,8 +362,29 @@ def mustafar_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tens
     if workspace is None:
         workspace = torch.zeros(mustafar_decode_workspace_bytes(q.shape[0], q.shape[1], k.num_kv_heads, max_len,
                                                                 num_splits), dtype=torch.uint8, device=q.device)
-    _check(load().mustafar_decode_step(_ptr(q), q.shape[1], _ptr(k_new), k_new.stride(0), k_new.stride(1),
-                                       _ptr(v_new), v_new.stride(0), v_new.stride(1), _ptr(pos), C.byref(k.struct),
-                                       C.byref(v.struct), max_len, scale, _ptr(out), _ptr(lse), _ptr(workspace),
-                                       workspace.numel(), num_splits, _ptr(err), _stream(stream)))
+    args = (_ptr(q), q.shape[1], _ptr(k_new), k_new.stride(0), k_new.stride(1), _ptr(v_new), v_new.stride(0),
+            v_new.stride(1), _ptr(pos), C.byref(k.struct), C.byref(v.struct), max_len, scale, _ptr(out), _ptr(lse),
+            _ptr(workspace), workspace.numel(), num_splits, _ptr(err), _stream(stream))
+    return args, out, lse, (q, k_new, v_new, pos, k, v, out, lse, workspace, err)
+
+
+def prepare_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
+                        k: CompressedCache, v: CompressedCache, max_len: int, scale: float, out=None, lse=None,
+                        workspace=None, num_splits: int = 0, err=None, stream=None, want_lse: bool = True):
+    """``mustafar_decode_step`` with its arguments marshalled once: returns (call, out, lse), where
+    ``call()`` runs the step again on the same buffers (fill q, k_new, v_new and pos in place)."""
+    args, out, lse, keep = _step_args(q, k_new, v_new, pos, k, v, max_len, scale, out, lse, workspace, num_splits,
+                                      err, stream, want_lse)
+    return PreparedCall(load().mustafar_decode_step, args, keep), out, lse
+
+
+def mustafar_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
+                         k: CompressedCache, v: CompressedCache, max_len: int, scale: float, out=None, lse=None,
+                         workspace=None, num_splits: int = 0, err=None, stream=None, want_lse: bool = True):
+    """One decode step in one launch: compress ``k_new``/``v_new`` ([B, Hkv, d] fp16) into slot
+    ``pos[b]`` of the caches, then attend over the ``pos[b] + 1`` tokens ``[0, pos[b]]``.
+    Returns (out [B,Hq,d] fp16, lse [B,Hq] fp32); ``max_len`` bounds ``pos[b] + 1``."""
+    args, out, lse, _ = _step_args(q, k_new, v_new, pos, k, v, max_len, scale, out, lse, workspace, num_splits, err,
+                                   stream, want_lse)
+    _check(load().mustafar_decode_step(*args))
     return out, lse

@@ -57,6 +57,19 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
   __syncthreads();
 
   if (tid < ntok) {
+    uint32_t T = 0;
+    if constexpr (!P24) {
+      // the threshold's high bits from the row's high bytes, before the full keys take registers
+      uint32_t hb[32];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(in_stage + stage_off(tid, j));
+        hb[2 * j] = __byte_perm(v.x, v.y, 0x7531u) & 0x7F7F7F7Fu;
+        hb[2 * j + 1] = __byte_perm(v.z, v.w, 0x7531u) & 0x7F7F7F7Fu;
+      }
+      T = high_threshold(hb, k);
+      asm volatile("" ::: "memory");  // the full row is loaded only now, after the high bytes are dead
+    }
     uint32_t raw[64];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -70,7 +83,7 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
     if constexpr (P24) {
       bitmap_24(raw, bm);
     } else {
-      topk_bitmap(raw, k, bm);
+      topk_bitmap(raw, k, T, bm);
     }
     reinterpret_cast<uint4 *>(bitmap)[stream * cap + t0 + tid] = make_uint4(bm[0], bm[1], bm[2], bm[3]);
     // pack the kept values in ascending channel order

@@ -7,9 +7,9 @@
 // and on equal keys the lower channel index is kept.
 //
 // Method: a 15-step binary search for the k-th largest key T (the largest T with
-// #{key >= T} >= k).  Each count is SIMD-within-a-register: two 15-bit keys share a
-// 32-bit word, and key + (0x8000 - T) sets bit 15 of its half exactly when key >= T
-// (no carry leaves a half).  Keys are paired as (channel i, channel i+16) of a 32-channel
+// #{key >= T} >= k).  Each count is SIMD-within-a-register: for the top 7 bits four key high
+// bytes share a word, for the low 8 two 15-bit keys do, and key + (0x8000 - T) sets bit 15 of
+// its half exactly when key >= T (no carry leaves a half).  Keys are paired as (channel i, channel i+16) of a 32-channel
 // group so that shifting the sum right by 15-i drops both indicator bits onto bits i and
 // 16+i: OR-ing the 16 pairs of a group yields that group's bitmap word directly.
 #pragma once
@@ -42,8 +42,11 @@ __device__ __forceinline__ void ge_bitmap(const uint32_t (&p)[64], uint32_t T, u
     uint32_t acc = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint32_t t = p[16 * w + i] + c;
-      acc |= (t >> (15 - i)) & ((1u << i) | (1u << (16 + i)));
+      // bits 15 and 31 of t -> bits i and 16+i: t >> (15-i) as a multiply-high, so that the integer
+      // multiply-add unit takes the shift and the accumulation off the logic pipe (the positions
+      // never overlap, so adding is OR-ing)
+      const uint32_t t = (p[16 * w + i] + c) & 0x80008000u;
+      acc += i == 15 ? t : __umulhi(t, 1u << (17 + i));
     }
     g[w] = acc;
   }
@@ -53,14 +56,33 @@ __device__ __forceinline__ int popc4(const uint32_t (&g)[kWords]) {
   return __popc(g[0]) + __popc(g[1]) + __popc(g[2]) + __popc(g[3]);
 }
 
-// Kept-channel bitmap of the k largest keys, ties toward the lower channel index.
-__device__ __forceinline__ void topk_bitmap(const uint32_t (&raw)[64], int k, uint32_t (&bm)[kWords]) {
+// Bits 14..8 of the top-k threshold (the largest T with #{key >= T} >= k), from the keys' high
+// bytes packed four to a word (any channel order: only counts are needed).  For a candidate with a
+// zero low byte, key >= cand exactly when (key >> 8) >= (cand >> 8), and byte + (0x80 - h) sets
+// the byte's bit 7 exactly when byte >= h (no carry leaves a byte).
+__device__ __forceinline__ uint32_t high_threshold(const uint32_t (&hb)[32], int k) {
+  uint32_t T = 0;
+#pragma unroll 1
+  for (int bit = 6; bit >= 0; --bit) {
+    const uint32_t h = (T >> 8) | (1u << bit);
+    const uint32_t c = (0x80u - h) * 0x01010101u;
+    uint32_t acc = 0;  // four per-byte counts (each at most 32)
+#pragma unroll
+    for (int r = 0; r < 32; ++r) acc += __umulhi((hb[r] + c) & 0x80808080u, 1u << 25);
+    if (static_cast<int>((acc * 0x01010101u) >> 24) >= k) T = h << 8;
+  }
+  return T;
+}
+
+// Kept-channel bitmap of the k largest keys, ties toward the lower channel index, given bits
+// 14..8 of the threshold (high_threshold).
+__device__ __forceinline__ void topk_bitmap(const uint32_t (&raw)[64], int k, uint32_t T, uint32_t (&bm)[kWords]) {
   uint32_t p[64];
   make_keys(raw, p);
-  uint32_t T = 0;
+  // bits 7..0 on the full keys, two per register
   uint32_t g[kWords];
 #pragma unroll 1
-  for (int bit = 14; bit >= 0; --bit) {
+  for (int bit = 7; bit >= 0; --bit) {
     const uint32_t cand = T | (1u << bit);
     ge_bitmap(p, cand, g);
     if (popc4(g) >= k) T = cand;

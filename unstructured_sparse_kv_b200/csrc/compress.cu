@@ -168,12 +168,15 @@ append_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, const int3
 }
 
 // Channel-wise compress: warp w of CTA x takes window 4x + w of stream (b = z, h = y), and the
-// warp of an incomplete last window also keeps its tokens in the stream's dense window copy.
+// warp of an incomplete last window also keeps its tokens in the stream's dense window copy.  The
+// CTA first stages its 64 dense rows in shared memory with coalesced 16-byte copies, so that the
+// selection reads its keys with plain shared loads.
 __global__ void __launch_bounds__(128)
 compress_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t st, int L, int H, int keep,
                         int F, int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
                         uint32_t *__restrict__ tile_offset, uint16_t *__restrict__ window) {
   __shared__ uint32_t scratch[4][128];
+  __shared__ __align__(16) uint16_t rows[4 * kWindowTokens][kHeadDim];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.y, b = blockIdx.z;
   const int64_t stream = static_cast<int64_t>(b) * H + h;
@@ -181,14 +184,24 @@ compress_channel_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, 
   const int ntiles = cap / kTileTokens;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ntiles; i += gridDim.x * blockDim.x)
     tile_offset[stream * ntiles + i] = static_cast<uint32_t>(i) * kTileTokens * static_cast<uint32_t>(keep);
-  const int t0 = (blockIdx.x * 4 + warp) * kWindowTokens;
+  const int tb = blockIdx.x * 4 * kWindowTokens;
+  const int ntok = min(4 * kWindowTokens, L - tb);
+  if (ntok <= 0) return;
+  const uint16_t *xs = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh;
+  for (int idx = threadIdx.x; idx < ntok * 16; idx += blockDim.x) {
+    const int tok = idx >> 4, j = idx & 15;
+    cp_async16(smem_addr(&rows[tok][8 * j]), xs + static_cast<int64_t>(tb + tok) * st + 8 * j);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  const int t0 = tb + warp * kWindowTokens;
   if (t0 >= L) return;
   const int n = min(kWindowTokens, L - t0);
-  const uint16_t *xs = x + static_cast<int64_t>(b) * sb + static_cast<int64_t>(h) * sh + static_cast<int64_t>(t0) * st;
+  const uint16_t *ws = &rows[warp * kWindowTokens][0];
   uint16_t *win = n < kWindowTokens ? window + stream * kWindowTokens * kHeadDim : nullptr;
-  warp_compress_window([=](int t) { return xs + static_cast<int64_t>(t) * st; }, n, F,
-                       bitmap + (stream * cap + t0) * kWords, values + (stream * cap + t0) * keep, win, 0,
-                       scratch[warp], lane);
+  warp_compress_window<false>([=](int t) { return ws + t * kHeadDim; }, n, F, bitmap + (stream * cap + t0) * kWords,
+                       values + (stream * cap + t0) * keep, win, 0, scratch[warp], lane);
 }
 
 // Channel-wise append: one warp per (cache, b, kv head), for one or two caches (a decode step's K
@@ -214,7 +227,7 @@ append_channel_kernel(const ChannelAppend c0, const ChannelAppend c1, const int3
   const int64_t stream = static_cast<int64_t>(b) * H + h;
   const uint16_t *xn = c.x + static_cast<int64_t>(b) * c.sb + static_cast<int64_t>(h) * c.sh;
   uint16_t *win = c.window + stream * kWindowTokens * kHeadDim;
-  warp_compress_window([=](int t) -> const uint16_t * { return t < r ? win + t * kHeadDim : xn; }, r + 1, c.F,
+  warp_compress_window<true>([=](int t) -> const uint16_t * { return t < r ? win + t * kHeadDim : xn; }, r + 1, c.F,
                        c.bitmap + (stream * c.cap + t0) * kWords, c.values + (stream * c.cap + t0) * c.keep, win, r,
                        scratch[threadIdx.x >> 5], lane);
 }

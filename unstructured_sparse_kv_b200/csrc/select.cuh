@@ -234,7 +234,7 @@ __device__ __forceinline__ void sort16_desc(uint32_t (&a)[16]) {
 }
 
 // One warp prunes and compresses one window of n (1..16) tokens of a stream, channel-wise.
-// src(t) points at token t's 128 fp16 channels (device memory).  Writes the n tokens' bitmap rows
+// src(t) points at token t's 128 fp16 channels (device memory when GLOBAL_SRC, else shared).  Writes the n tokens' bitmap rows
 // from bm_dst (4 words a token) and the window's packed values from val_dst, token after token,
 // each token's kept channels in ascending order.  When win_dst is not null, tokens win_from .. n-1
 // are also copied, dense, to win_dst + 128 t.  `scratch` is 128 words of this warp's shared
@@ -242,13 +242,13 @@ __device__ __forceinline__ void sort16_desc(uint32_t (&a)[16]) {
 // is one bitmap word.  All 32 lanes must call it.
 // The loops over words and tokens stay rolled: the routine often runs once per warp (an append),
 // where a long unrolled body would be fetched from a cold instruction cache.
-template <class Src>
+template <bool GLOBAL_SRC, class Src>
 __device__ __forceinline__ void warp_compress_window(Src src, int n, int F, uint32_t *bm_dst, uint16_t *val_dst,
                                                      uint16_t *win_dst, int win_from, uint32_t *scratch, int lane) {
   const int kc = window_keep(n, F);
   const uint32_t valid = n >= 16 ? 0xFFFFu : (1u << n) - 1u;
-  // the window's rows (two 128-byte lines each) are requested up front
-  if (lane < 2 * n) {
+  // rows in device memory (two 128-byte lines each) are requested up front
+  if (GLOBAL_SRC && lane < 2 * n) {
     const uint16_t *line = src(lane >> 1) + 64 * (lane & 1);
     asm volatile("prefetch.global.L1 [%0];\n" ::"l"(line));
   }

@@ -222,3 +222,15 @@ def test_channel_keep_count_sizes_and_checks(lib):
     with pytest.raises(ValueError):
         M.CompressedCache(1, 2, 64, [0.5, 0.7], pattern="channel", device="cpu")
 
+
+def test_channel_cache_cannot_pair_with_per_head(lib):
+    # rejected in host validation, before any plan or launch
+    kc = _cache(keep=40)
+    kc.pattern, kc.window = 2, 0x4000
+    keeps = (C.c_int32 * 2)(39, 64)
+    vc = _cache(keep=64)
+    vc.head_keep = C.cast(keeps, C.c_void_p).value
+    st, err = _status(lib, "mustafar_decode_attn", 0x7000, 8, C.byref(kc), C.byref(vc), 0x6000, 64, 1.0, 0x8000,
+                      None, 0x9000, 1 << 20, 0, None, None)
+    assert st == 2 and "per-head" in err, (st, err)
+

@@ -943,13 +943,18 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
   // (not for 2:4: its 128-bit loads see at most 2-way conflicts, and the grouped staging cost more
   // than it saved there, measured)
   const bool can_skew = variant == 0;
-  // tokens per staged group, as log2 (4 = the chunk in one copy, no skew).  Only keeps of 96 and 128
-  // are staged token by token: there eight tokens' runs share 1-2 bank offsets; at keep 64 the
-  // grouped copies cost about what the conflicts did (measured: 0.94-1.08x), at 32 and below the
-  // runs are short
-  auto group_lg = [&](int keep) { return can_skew && keep % 32 == 0 && keep >= 96 ? 0 : 4; };
-  plan->lg_k = group_lg(keep_k);
-  plan->lg_v = group_lg(keep_v);
+  // tokens per staged group, as log2 (4 = the chunk in one copy, no skew).  Keeps of 96 and 128 are
+  // staged token by token: there eight tokens' runs share one or two bank offsets (s = 0: 1.2-1.8x).
+  // Keep 64 goes in 4-token groups when the other cache's keep is also a multiple of 32 (s = 0.5:
+  // 1.05-1.10x); paired with an unskewed cache the grouped copies measured 4 % slower.  Smaller keeps
+  // have short runs and stay in one copy.
+  auto group_lg = [&](int keep, int other) {
+    if (!can_skew || keep % 32 != 0) return 4;
+    if (keep >= 96) return 0;
+    return keep == 64 && other % 32 == 0 ? 2 : 4;
+  };
+  plan->lg_k = group_lg(keep_k, keep_v);
+  plan->lg_v = group_lg(keep_v, keep_k);
   plan->skew_k = plan->lg_k < 4 ? 16 * (kChunk >> plan->lg_k) : 0;  // skew bytes added to the region
   plan->skew_v = plan->lg_v < 4 ? 16 * (kChunk >> plan->lg_v) : 0;
   if (plan->skew_k || plan->skew_v) variant = 4;

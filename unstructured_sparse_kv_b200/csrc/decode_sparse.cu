@@ -862,7 +862,7 @@ SparseFn pick_sparse(int nstage, bool hirows, int variant) {
 // use 0..9)
 int sparse_slot(int nstage, bool hirows, int variant) { return 12 + 6 * variant + 2 * (nstage - 2) + (hirows ? 1 : 0); }
 
-constexpr int kMinUnitsPerCta = kWarps;  // at least one chunk per warp
+constexpr int kMinUnitsPerCta = 2 * kWarps;  // at least two chunks per warp (more CTAs per stream cost more merging)
 constexpr int kMaxCtasPerSm = 4;
 constexpr int kCtaSmemBudget = 56000;        // four CTAs per SM fit in 228 KB with this much each
 

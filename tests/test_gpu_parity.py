@@ -131,6 +131,7 @@ def test_append_rows_at_different_positions_and_out_of_range():
     (1, 8, 8, 1000, 0.995, 0.995, 0, False),  # keep = 1
     (2, 8, 2, 200, 0.25, 0.0, 0, True),    # keeps 96 and 128: runs staged token by token
     (2, 8, 2, 150, 0.25, 0.7, 2, True),    # one cache staged token by token, one in a single copy
+    (2, 8, 2, 213, 0.5, 0.5, 3, True),     # keep 64 in both caches: staged in 4-token groups
 ])
 def test_decode_small_cases(B, Hq, Hkv, L, sK, sV, splits, ragged):
     cap = ((L + 63) // 64) * 64

@@ -132,6 +132,7 @@ def test_append_rows_at_different_positions_and_out_of_range():
     (2, 8, 2, 200, 0.25, 0.0, 0, True),    # keeps 96 and 128: runs staged token by token
     (2, 8, 2, 150, 0.25, 0.7, 2, True),    # one cache staged token by token, one in a single copy
     (2, 8, 2, 213, 0.5, 0.5, 3, True),     # keep 64 in both caches: staged in 4-token groups
+    (1, 32, 2, 170, 0.0, 0.25, 0, False),  # G = 16 with both caches staged token by token
 ])
 def test_decode_small_cases(B, Hq, Hkv, L, sK, sV, splits, ragged):
     cap = ((L + 63) // 64) * 64
@@ -606,6 +607,24 @@ def test_channel_decode_step_ragged_rows(v_pat):
     _channel_matches(kc, U.bits(K), lens)
     if v_pat == "channel":
         _channel_matches(vc, U.bits(V), lens)
+
+
+def test_channel_decode_gqa16():
+    # G = 16 (two row tiles of q heads) over channel-wise K and V caches, ragged rows
+    B, Hq, Hkv, L, cap = 2, 32, 2, 181, 192
+    K = synth.keys(B, Hkv, L, D, 87, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L, D, 87, DEV, capacity=cap)
+    kc = M.CompressedCache(B, Hkv, cap, 0.7, pattern="channel")
+    vc = M.CompressedCache(B, Hkv, cap, 0.5, pattern="channel")
+    M.mustafar_compress(K, L, 0.7, kc)
+    M.mustafar_compress(V, L, 0.5, vc)
+    q = synth.queries(B, Hq, D, 87, DEV)
+    seq = torch.tensor([L, 100], dtype=torch.int32)
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), L, 0.088)
+    Kb, Vb = U.bits(K)[:, :, :L], U.bits(V)[:, :, :L]
+    o_ref, l_ref = oracle.attention(U.bits(q), oracle.prune_channel(Kb, 0.7), oracle.prune_channel(Vb, 0.5),
+                                    seq.numpy(), 0.088)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag="channel G=16")
 
 
 def test_channel_decode_step_same_bits_as_append_then_attend():

@@ -413,6 +413,9 @@ def main(argv=None):
     ap.add_argument("--profile-shape", default=None,
                     help="ncu case: 'B,L,sK,sV' -- GQA 32/8 decode over two rotating compressed-cache copies "
                          "of that shape (larger than L2 for B*L >= 64k), six mustafar_decode_attn launches, no timing")
+    ap.add_argument("--profile-compress", default=None,
+                    help="ncu case: 'PATTERN,s' (topk or channel) -- prefill compress of one [8, 16384, 8, 128] "
+                         "fp16 tensor ([B, L, H, d] storage), three launches, no timing")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
@@ -421,6 +424,21 @@ def main(argv=None):
         from unstructured_sparse_kv_b200 import suite
         M.load()
         suite.run(args.suite, measured_peak()[0], tuple(args.suite_parts.split(",")))
+        return 0
+    if args.profile_compress:
+        import torch
+        import unstructured_sparse_kv_b200 as M
+        M.load()
+        pattern, sp = args.profile_compress.split(",")
+        B, L, H, d = 8, 16384, 8, 128
+        g = torch.Generator(device="cuda")
+        g.manual_seed(5)
+        x = torch.randn(B, L, H, d, generator=g, device="cuda").to(torch.float16)
+        c = M.CompressedCache(B, H, L, float(sp), pattern=pattern)
+        for _ in range(3):
+            M.mustafar_compress(x.permute(0, 2, 1, 3), L, float(sp), c)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": "compress", "pattern": pattern, "sparsity": float(sp), "launches": 3}))
         return 0
     if args.profile_shape:
         import torch

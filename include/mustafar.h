@@ -230,7 +230,8 @@ MUSTAFAR_API mustafar_status mustafar_decode_attn(const void *q, int32_t num_q_h
  * run time: Mustafar abstract).  The CTA that will read the new token's 16-token chunk
  * compresses it first, so no separate append launch is needed; a channel-wise cache is the
  * exception: its append (which prunes the token's whole window again) runs as a launch of its
- * own on the same stream just before the attention.
+ * own on the same stream just before the attention (if the attention launch then fails, with
+ * MUSTAFAR_ERR_CUDA, that cache already holds the new token).
  *   k_new, v_new : fp16 [batch][num_kv_heads][head_dim], element (b, h, c) at
  *                  k_new[b*k_stride_b + h*k_stride_h + c]; 16-byte aligned, strides multiples of 8.
  *   d_pos        : int32 [batch]; a slot outside [0, capacity) skips the append, sets

@@ -233,6 +233,25 @@ __device__ __forceinline__ void sort16_desc(uint32_t (&a)[16]) {
   }
 }
 
+// The same network on two 16-bit keys per word (independent sorts of the two halves).
+__device__ __forceinline__ void sort16_desc_x2(uint32_t (&a)[16]) {
+#pragma unroll
+  for (int k = 2; k <= 16; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const uint32_t hi = __vmaxu2(a[i], a[l]), lo = __vminu2(a[i], a[l]);
+          a[i] = (i & k) == 0 ? hi : lo;
+          a[l] = (i & k) == 0 ? lo : hi;
+        }
+      }
+    }
+  }
+}
+
 // One warp prunes and compresses one window of n (1..16) tokens of a stream, channel-wise.
 // src(t) points at token t's 128 fp16 channels (device memory when GLOBAL_SRC, else shared).  Writes the n tokens' bitmap rows
 // from bm_dst (4 words a token) and the window's packed values from val_dst, token after token,
@@ -252,43 +271,55 @@ __device__ __forceinline__ void warp_compress_window(Src src, int n, int F, uint
     const uint16_t *line = src(lane >> 1) + 64 * (lane & 1);
     asm volatile("prefetch.global.L1 [%0];\n" ::"l"(line));
   }
-  // 1. per channel: sort the window's keys, keep the kc largest (lower token on ties).
-  //    Bit 16w + t of `kept`: token t of channel 32w + lane is kept.
+  // 1. per channel: sort the window's keys, keep the kc largest (lower token on ties).  Two channels
+  //    (words 2p and 2p+1) are sorted together, their keys (at most 0x8000) packed in the two halves of
+  //    a word and compared with SIMD 16-bit min/max.  Bit 16w + t of `kept`: token t of channel
+  //    32w + lane is kept.
   uint64_t kept = 0u;
 #pragma unroll 1
-  for (int w = 0; w < kWords; ++w) {
+  for (int pw = 0; pw < kWords / 2; ++pw) {
     uint32_t key[16], a[16];
-    uint16_t xs[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) xs[t] = src(min(t, n - 1))[32 * w + lane];  // all 16 loads in flight at once
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
+      const uint16_t *row = src(min(t, n - 1));
+      key[t] = row[64 * pw + lane] | (static_cast<uint32_t>(row[64 * pw + 32 + lane]) << 16);  // all in flight
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      if (win_dst != nullptr && t >= win_from && t < n) {
+        win_dst[kHeadDim * t + 64 * pw + lane] = static_cast<uint16_t>(key[t]);
+        win_dst[kHeadDim * t + 64 * pw + 32 + lane] = static_cast<uint16_t>(key[t] >> 16);
+      }
       // keys are shifted up by one so that the missing tokens of a short window (0) sort last
-      key[t] = t < n ? (xs[t] & 0x7FFFu) + 1u : 0u;
+      key[t] = t < n ? (key[t] & 0x7FFF7FFFu) + 0x00010001u : 0u;
       a[t] = key[t];
-      if (win_dst != nullptr && t >= win_from && t < n) win_dst[kHeadDim * t + 32 * w + lane] = xs[t];
     }
-    sort16_desc(a);
-    uint32_t T = a[0];  // the kc-th largest key
+    sort16_desc_x2(a);
+    uint32_t T2 = a[0];  // the kc-th largest key of each half
 #pragma unroll
-    for (int i = 1; i < 16; ++i) T = i == kc - 1 ? a[i] : T;
-    uint32_t gt = 0u, eq = 0u;
+    for (int i = 1; i < 16; ++i) T2 = i == kc - 1 ? a[i] : T2;
 #pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      gt |= (key[t] > T ? 1u : 0u) << t;
-      eq |= (key[t] == T ? 1u : 0u) << t;
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t T = (T2 >> (16 * h)) & 0xFFFFu;
+      uint32_t gt = 0u, eq = 0u;
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const uint32_t kk = (key[t] >> (16 * h)) & 0xFFFFu;
+        gt |= (kk > T ? 1u : 0u) << t;
+        eq |= (kk == T ? 1u : 0u) << t;
+      }
+      gt &= valid;
+      eq &= valid;
+      int need = kc - __popc(gt);  // keys equal to T that survive, lowest tokens first
+      uint32_t take = gt;
+      while (eq != 0u && need > 0) {
+        const uint32_t low = eq & (0u - eq);
+        take |= low;
+        eq ^= low;
+        --need;
+      }
+      kept |= static_cast<uint64_t>(take) << (16 * (2 * pw + h));
     }
-    gt &= valid;
-    eq &= valid;
-    int need = kc - __popc(gt);  // keys equal to T that survive, lowest tokens first
-    uint32_t take = gt;
-    while (eq != 0u && need > 0) {
-      const uint32_t low = eq & (0u - eq);
-      take |= low;
-      eq ^= low;
-      --need;
-    }
-    kept |= static_cast<uint64_t>(take) << (16 * w);
   }
   // 2. bitmap words by ballot, and where each (token, word) run starts: scratch[4t + w] holds the
   //    word, scratch[64 + 4t + w] the run start within the window

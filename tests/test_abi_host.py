@@ -234,3 +234,12 @@ def test_channel_cache_cannot_pair_with_per_head(lib):
                       None, 0x9000, 1 << 20, 0, None, None)
     assert st == 2 and "per-head" in err, (st, err)
 
+
+def test_24_cache_cannot_have_head_keep(lib):
+    keeps = (C.c_int32 * 2)(64, 64)
+    c = _cache(keep=64)
+    c.pattern = 1
+    c.head_keep = C.cast(keeps, C.c_void_p).value
+    st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(c), None, None)
+    assert st == 1 and "2:4" in err, (st, err)
+

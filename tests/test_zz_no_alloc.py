@@ -54,6 +54,30 @@ def test_noalloc_matches_workspace_entry_point_twice(B, Hq, Hkv, L, num_splits):
         _close(out, ref_out, lse, ref_lse)
 
 
+@pytest.mark.parametrize("pattern_k,pattern_v", [("channel", "channel"), ("channel", "2:4"), ("2:4", "2:4")])
+def test_noalloc_variants_match_workspace_entry_point(pattern_k, pattern_v):
+    # the other cache formats go through the same allocation-free entry point
+    lib = M.load()
+    B, Hq, Hkv, L, cap = 4, 32, 8, 1000, 1024
+    K = synth.keys(B, Hkv, L, 128, 37, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L, 128, 37, DEV, capacity=cap)
+    sk = 0.5 if pattern_k == "2:4" else 0.7
+    sv = 0.5 if pattern_v == "2:4" else 0.7
+    kc = M.CompressedCache(B, Hkv, cap, sk, pattern=pattern_k)
+    vc = M.CompressedCache(B, Hkv, cap, sv, pattern=pattern_v)
+    M.mustafar_compress(K, L, sk, kc)
+    M.mustafar_compress(V, L, sv, vc)
+    seq = synth.seq_lens(B, L, True, 5).to(DEV)
+    q = synth.queries(B, Hq, 128, 37, DEV)
+    ref_out, ref_lse = M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=DEV)
+    st = _noalloc(lib, q, kc, vc, seq, L, out, lse)
+    assert st == 0, lib.mustafar_last_error().decode()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)  # the same kernel and plan
+
+
 def test_noalloc_rejects_a_plan_beyond_its_scratch():
     lib = M.load()
     B, Hq, Hkv, L = 8, 32, 8, 4096

@@ -270,6 +270,34 @@ def test_prepared_decode_step_matches_direct_calls():
     assert torch.equal(kc.values, kc2.values) and torch.equal(vc.bitmap, vc2.bitmap)
 
 
+def test_captured_decode_loop_matches_eager_steps():
+    # a graph of 6 fused steps (one launch each) replayed gives the eager calls' bits
+    B, Hq, Hkv, L0, cap, steps = 2, 8, 2, 90, 128, 6
+    K = synth.keys(B, Hkv, L0, D, 93, DEV, capacity=cap)
+    V = synth.values(B, Hkv, L0, D, 93, DEV, capacity=cap)
+    caches = []
+    for _ in range(2):
+        kc, vc = M.CompressedCache(B, Hkv, cap, 0.7), M.CompressedCache(B, Hkv, cap, 0.7)
+        M.mustafar_compress(K, L0, 0.7, kc)
+        M.mustafar_compress(V, L0, 0.7, vc)
+        caches.append((kc, vc))
+    q = torch.stack([synth.queries(B, Hq, D, 93, DEV, step=i) for i in range(steps)])
+    toks = [synth.step_tokens(B, Hkv, D, 93, i, DEV) for i in range(steps)]
+    kn = torch.stack([t[0] for t in toks])
+    vn = torch.stack([t[1] for t in toks])
+    pos = torch.stack([torch.full((B,), L0 + i, dtype=torch.int32, device=DEV) for i in range(steps)])
+    out = torch.empty(steps, B, Hq, D, dtype=torch.float16, device=DEV)
+    lse = torch.empty(steps, B, Hq, dtype=torch.float32, device=DEV)
+    g = M.capture_decode_steps(q, kn, vn, pos, caches[0][0], caches[0][1], cap, 0.5, out, lse)
+    g.replay()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        o, l = M.mustafar_decode_step(q[i], kn[i], vn[i], pos[i], caches[1][0], caches[1][1], cap, 0.5)
+        assert torch.equal(o, out[i]) and torch.equal(l, lse[i]), f"step {i}"
+    for a, b in zip(caches[0], caches[1]):
+        assert torch.equal(a.bitmap, b.bitmap) and torch.equal(a.values, b.values)
+
+
 def test_decode_step_out_of_range_positions():
     B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 23)

@@ -388,3 +388,34 @@ def mustafar_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tens
                                    stream, want_lse)
     _check(load().mustafar_decode_step(*args))
     return out, lse
+
+
+def capture_decode_steps(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
+                         k: CompressedCache, v: CompressedCache, max_len: int, scale: float, out: torch.Tensor,
+                         lse: torch.Tensor, workspace: torch.Tensor = None, num_splits: int = 0):
+    """A multi-step decode loop as one CUDA graph: step i runs ``mustafar_decode_step`` on
+    ``q[i]``, ``k_new[i]``, ``v_new[i]``, ``pos[i]`` (leading step axis) and writes ``out[i]``,
+    ``lse[i]``.  Returns the captured ``torch.cuda.CUDAGraph``; each ``replay()`` runs every step
+    again, in order, on whatever the input tensors then hold (the graph keeps their addresses).
+    One warm-up step runs eagerly first (plans and kernel attributes are set outside capture), so
+    the caches already hold step 0's token when the function returns."""
+    steps = q.shape[0]
+    if not all(t.shape[0] == steps for t in (k_new, v_new, pos, out, lse)):
+        raise ValueError("q, k_new, v_new, pos, out and lse need the same number of steps")
+    if workspace is None:
+        workspace = torch.zeros(mustafar_decode_workspace_bytes(q.shape[1], q.shape[2], k.num_kv_heads, max_len,
+                                                                num_splits), dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.Stream(device=q.device)
+    stream.wait_stream(torch.cuda.current_stream(q.device))
+    with torch.cuda.stream(stream):
+        mustafar_decode_step(q[0], k_new[0], v_new[0], pos[0], k, v, max_len, scale, out=out[0], lse=lse[0],
+                             workspace=workspace, num_splits=num_splits, stream=stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(steps):
+                mustafar_decode_step(q[i], k_new[i], v_new[i], pos[i], k, v, max_len, scale, out=out[i], lse=lse[i],
+                                     workspace=workspace, num_splits=num_splits, stream=stream)
+    torch.cuda.current_stream(q.device).wait_stream(stream)
+    graph._mustafar_keep = (q, k_new, v_new, pos, k, v, out, lse, workspace)
+    return graph
+

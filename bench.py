@@ -89,10 +89,15 @@ def decode_algorithmic_bytes(B, Hq, Hkv, d, lens, kK, kV):
 
 
 def kernel_source_hash() -> str:
+    """Hash of the decode kernel's code (comments and blank space removed, so that editing a comment
+    does not invalidate the recorded DRAM traffic)."""
+    import re
     h = hashlib.sha256()
     for f in ("common.cuh", "select.cuh", "decode_sparse.cu"):
-        with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f)) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("\n".join(line.strip() for line in text.splitlines() if line.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -27,6 +27,12 @@
 //   reading a shared zero.  The contraction index is permuted so that a lane's channels are one
 //   bitmap word (K) or half word (V); q's fragments use the same permutation and the output
 //   channels are put back in order at the merge.  Online softmax per head in the log2 domain.
+//
+// Template variants (chosen on the host per call): PERHEAD reads a keep count and value base per
+// kv head; P24 expands 2:4 caches with byte permutes instead of the per-channel walk; SCAN finds
+// each token's run from popcount prefix sums (channel-wise caches, whose tokens keep varying
+// counts); SKEW stages a cache whose keep is a multiple of 32 in 16-byte-skewed token groups so
+// that the runs do not all start on one shared-memory bank.
 #include <cfloat>
 
 #include "common.cuh"

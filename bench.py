@@ -9,10 +9,15 @@ The workload is 4096 prefill tokens plus 64 decode steps at K and V sparsity 0.7
 steps cycle through the 64 decode positions.  Inputs are synthetic (seeded; see
 ``unstructured_sparse_kv_b200/synth.py``).
 
-Timing: CUDA graphs of 64 steps are replayed; every step reads one of 8 rotating copies
-of the compressed caches (8 x 49.5 MB, over twice the 126 MB L2), so no step finds the
-previous step's cache in L2.  The timed region is bracketed by a barrier and
-``torch.cuda.synchronize()``; the time is the max over ranks.
+Timing: the timed region replays CUDA graphs that hold exactly ``--steps`` decode steps (graphs
+of 64 steps plus one graph of the remaining ``steps % 64``); warm-up replays exactly
+``--warmup`` steps the same way.  Every step reads one of 8 rotating copies of the compressed
+caches (8 x 49.5 MB, over twice the 126 MB L2), so no step finds the previous step's cache in
+L2.  The timed region is bracketed by a barrier and ``torch.cuda.synchronize()``; the time is
+the max over ranks.  SM clocks and throttle reasons are polled through NVML while the GPU runs.
+The comparison legs (the same step as three launches, the attention launch alone, dense fp16
+attention, and attention at sparsity 0 / 0.3 / 0.5 / 0.7 / 0.9) are all timed the same way:
+replays of 64-step graphs over the same rotation.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
 """
@@ -37,6 +42,7 @@ WORKLOAD = dict(batch=8, q_heads=32, kv_heads=8, head_dim=128, context=4096, dec
                 sparsity_k=0.7, sparsity_v=0.7)
 ROTATE = 8
 GRAPH_STEPS = 64
+SPARSITY_AXIS = (0.0, 0.3, 0.5, 0.7, 0.9)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -71,6 +77,11 @@ def barrier():
         dist.barrier()
 
 
+def graph_counts(n: int):
+    """How exactly n steps are replayed: (replays of the 64-step graph, steps of the one remainder graph)."""
+    return divmod(int(n), GRAPH_STEPS)
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -89,15 +100,13 @@ def decode_algorithmic_bytes(B, Hq, Hkv, d, lens, kK, kV):
 
 
 def kernel_source_hash() -> str:
-    """Hash of the decode kernel's code (comments and blank space removed, so that editing a comment
-    does not invalidate the recorded DRAM traffic)."""
-    import re
+    """Hash of the raw text of every source the decode launch is built from (kernel, device helpers,
+    the parameter block and the host-side plan / launch code); any edit invalidates the recorded
+    DRAM traffic."""
     h = hashlib.sha256()
-    for f in ("common.cuh", "select.cuh", "decode_sparse.cu"):
-        with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f)) as fh:
-            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
-        text = re.sub(r"//[^\n]*", "", text)
-        h.update("\n".join(line.strip() for line in text.splitlines() if line.strip()).encode())
+    for f in ("common.cuh", "select.cuh", "internal.h", "decode_sparse.cu", "abi.cu"):
+        with open(os.path.join(ROOT, "unstructured_sparse_kv_b200", "csrc", f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -115,53 +124,85 @@ def recorded_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event (throttle) reasons of one GPU, polled through NVML about every
+    2 ms in a background thread while the GPU works, so that even a timed region of a millisecond gets
+    samples.  ``mark()`` records the host time at which the timed region starts and ends."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, device_index: int):
-        self.dev = device_index
-        self.proc = None
-        self.path = None
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []  # (t, sm_mhz, reasons_bitmask, power_w)
+        self.marks = []
+        self.err = None
+        self._stop = None
+        self._thread = None
+
+    def _handle(self, nv):
+        import torch
+        try:
+            pr = torch.cuda.get_device_properties(self.dev)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
 
     def __enter__(self):
-        import tempfile
-        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.dev), "-lms", "200"], stdout=open(self.path, "w"),
-                                         stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: the record says so
+            self.err = f"nvml unavailable: {e}"
+            return self
+        self._stop = threading.Event()
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((time.perf_counter(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         int(nv.nvmlDeviceGetCurrentClocksEventReasons(h)),
+                                         nv.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception as e:
+                    self.err = str(e)
+                    return
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=poll, daemon=True)
+        self._thread.start()
         return self
 
+    def mark(self):
+        self.marks.append(time.perf_counter())
+
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
             try:
-                self.proc.wait(timeout=5)
+                import pynvml as nv
+                nv.nvmlShutdown()
             except Exception:
-                self.proc.kill()
+                pass
 
     def summary(self):
-        if self.path is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
-        mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"], "samples": 0}
+        window = self.samples
+        source = "whole run"
+        if len(self.marks) >= 2:
+            inside = [x for x in self.samples if self.marks[0] <= x[0] <= self.marks[1]]
+            if inside:
+                window, source = inside, "timed region"
+        sm = sorted(x[1] for x in window)
+        bits = 0
+        for x in window:
+            bits |= x[2]
+        return {"sm_mhz": sm[len(sm) // 2], "sm_min_mhz": sm[0], "sm_max_mhz": self.max_mhz,
+                "reasons": [n for n, b in self.REASONS if bits & b], "samples": len(window),
+                "power_w_max": max(x[3] for x in window), "source": f"NVML every ~2 ms, {source}"}
 
 
 # ------------------------------------------------------------------------------------------ workload
@@ -200,6 +241,7 @@ class Workload:
         self.ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, cap), dtype=torch.uint8, device=device)
         self.splits = M.mustafar_decode_plan_splits(B, Hkv, cap, self.kc[0].keep, self.vc[0].keep)
         self.compressed_bytes = self.kc[0].nbytes() + self.vc[0].nbytes()
+        self.dense_cache_bytes = 2 * self.K.numel() * self.K.element_size()
 
     def step(self, i: int, mode: str = "fused"):
         """One decode step: "fused" (one launch), "separate" (append K, append V, attend) or
@@ -215,16 +257,33 @@ class Workload:
         M.mustafar_decode_attn(self.q[j], self.kc[r], self.vc[r], self.seq[j], self.cap, 1.0, out=self.out,
                                lse=self.lse, workspace=self.ws)
 
-    def graph(self, mode="fused", dense=None):
+    def capture(self, n: int, run=None, mode: str = "fused"):
+        """A CUDA graph of n consecutive steps 0 .. n-1 of ``run(i)`` (default: ``self.step(i, mode)``);
+        the steps run once eagerly first (plans, kernel attributes) and are then captured."""
         torch = self.torch
-        g = torch.cuda.CUDAGraph()
-        for i in range(GRAPH_STEPS):  # warm once eagerly (plans, attributes) before capture
-            (dense.step(i) if dense else self.step(i, mode))
+        run = run or (lambda i: self.step(i, mode))
+        for i in range(n):
+            run(i)
         torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for i in range(GRAPH_STEPS):
-                (dense.step(i) if dense else self.step(i, mode))
+            for i in range(n):
+                run(i)
         return g
+
+    def exact(self, n: int, run=None, mode: str = "fused"):
+        """Graphs that replay exactly n steps: n // 64 replays of a 64-step graph, then one graph of the
+        remaining n % 64 steps.  Returns (replay function, graphs)."""
+        full, rest = graph_counts(n)
+        g64 = self.capture(GRAPH_STEPS, run, mode) if full else None
+        gr = self.capture(rest, run, mode) if rest else None
+
+        def replay():
+            for _ in range(full):
+                g64.replay()
+            if gr is not None:
+                gr.replay()
+        return replay, [g for g in (g64, gr) if g is not None]
 
 
 class DenseBaseline:
@@ -242,6 +301,33 @@ class DenseBaseline:
         wl, r, j = self.wl, i % 3, i % self.wl.steps
         self.M.mustafar_dense_decode_attn(wl.q[j], self.copies[r], self.vcopies[r], wl.seq[j], wl.cap, 1.0,
                                           out=wl.out, lse=wl.lse, workspace=self.ws)
+
+    def release(self):
+        self.copies, self.vcopies = self.copies[:1], self.vcopies[:1]
+
+
+class SparsityPoint:
+    """The bench workload's caches compressed at one sparsity (K and V alike), ROTATE copies, and the
+    attention launch alone over them (same queries, lengths and rotation as the decode step)."""
+
+    def __init__(self, wl: Workload, sparsity: float):
+        M = wl.M
+        self.wl, self.M = wl, M
+        self.kc, self.vc = [], []
+        for _ in range(ROTATE):
+            kc = M.CompressedCache(wl.B, wl.Hkv, wl.cap, sparsity, device=wl.dev)
+            vc = M.CompressedCache(wl.B, wl.Hkv, wl.cap, sparsity, device=wl.dev)
+            M.mustafar_compress(wl.K, wl.cap, sparsity, kc)
+            M.mustafar_compress(wl.V, wl.cap, sparsity, vc)
+            self.kc.append(kc)
+            self.vc.append(vc)
+        self.keep = self.kc[0].keep
+        self.nbytes = self.kc[0].nbytes() + self.vc[0].nbytes()
+
+    def step(self, i: int):
+        wl, r, j = self.wl, i % ROTATE, i % self.wl.steps
+        self.M.mustafar_decode_attn(wl.q[j], self.kc[r], self.vc[r], wl.seq[j], wl.cap, 1.0, out=wl.out,
+                                    lse=wl.lse, workspace=wl.ws)
 
 
 def time_graph(g, replays: int, stream) -> float:
@@ -399,15 +485,15 @@ def config_dict():
                         "attention",
             "batch": w["batch"], "context": w["context"], "decode_steps": w["decode_steps"],
             "sparsity_k": w["sparsity_k"], "sparsity_v": w["sparsity_v"],
-            "l2": f"{ROTATE} rotating compressed-cache copies (> 2x the 126 MB L2)", "timing": "CUDA graphs of 64 steps"}
+            "l2": f"{ROTATE} rotating compressed-cache copies (> 2x the 126 MB L2)", "timing": "exactly --steps fused steps replayed from CUDA graphs (64-step graphs + one graph of the remainder), CUDA events on the launching stream"}
 
 
 # ------------------------------------------------------------------------------------------ main
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64 * 2000)
-    ap.add_argument("--warmup", type=int, default=64 * 20)
+    ap.add_argument("--steps", type=int, default=64 * 300)
+    ap.add_argument("--warmup", type=int, default=64 * 4)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--suite", default=None, help="write the workload-shape suite (JSONL) to this path and exit")
@@ -426,7 +512,7 @@ def main(argv=None):
         return run_reference(args)
     if args.suite:
         import unstructured_sparse_kv_b200 as M
-        from unstructured_sparse_kv_b200 import suite
+        import suite
         M.load()
         suite.run(args.suite, measured_peak()[0], tuple(args.suite_parts.split(",")))
         return 0
@@ -499,28 +585,32 @@ def main(argv=None):
     wl = Workload(rank_seed(rank), dev)
     stream = torch.cuda.current_stream()
 
-    # ---- the timed region: K steps (graphs of 64 steps; a tail of K % 64 eager steps)
-    g_step = wl.graph()
-    reps_w = max(1, math.ceil(args.warmup / GRAPH_STEPS))
-    for _ in range(reps_w):
-        g_step.replay()
-    torch.cuda.synchronize()
-    reps, tail = divmod(args.steps, GRAPH_STEPS)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
+    # ---- the timed region: exactly K fused steps, replayed from CUDA graphs (one launch per step)
+    timed, timed_graphs = wl.exact(args.steps)
+    warm, warm_graphs = wl.exact(args.warmup) if args.warmup > 0 else (lambda: None, [])
+    leg64 = wl.capture(GRAPH_STEPS)  # 64-step graph of the same fused step for the clock soak
+    with ClockSampler(dev) as clocks:
+        # keep the GPU under load for about a second before the timed region, so that its clocks are
+        # the loaded ones and the sampler has a record around the timed region
+        soak_reps = max(1, int(0.8e6 / (GRAPH_STEPS * 40.0)))
+        for _ in range(soak_reps):
+            leg64.replay()
+        warm()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        clocks.mark()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(reps):
-            g_step.replay()
-        for i in range(tail):
-            wl.step(i)
+        timed()
         e1.record(stream)
         torch.cuda.synchronize()
-    barrier()
+        clocks.mark()
+        barrier()
     elapsed_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     us_per_step = aggregate_us_per_step(elapsed_ms, args.steps, world)
     clk = clocks.summary()
+    del timed_graphs, warm_graphs
 
     # ---- the dominant (and only) kernel of the step is the fused decode kernel: one launch per
     # step, so its average launch duration is the timed region's time per step
@@ -530,26 +620,44 @@ def main(argv=None):
     peak, peak_kind = measured_peak()
     achieved = avg_bytes / (us_per_step * world * 1e-6) / 1e9  # per launch on one GPU
 
-    # ---- the same step as three launches, and the attention launch alone (same inputs and rotation)
-    extra_us = {}
-    for mode in ("separate", "attend"):
-        g = wl.graph(mode)
+    # ---- comparison legs, all timed alike: replays of 64-step graphs over the same rotation
+    leg_steps = GRAPH_STEPS * max(8, min(100, args.steps // GRAPH_STEPS))
+
+    def time_leg(g):
         for _ in range(3):
             g.replay()
         torch.cuda.synchronize()
-        n = max(20, min(400, reps))
-        extra_us[mode] = time_graph(g, n, stream) * 1000.0 / (n * GRAPH_STEPS)
-        del g
-    att_us = extra_us["attend"]
+        return time_graph(g, leg_steps // GRAPH_STEPS, stream) * 1000.0 / leg_steps
 
-    # ---- dense fp16 baseline on the same context
+    legs = {"fused": time_leg(leg64)}
+    del leg64
+    for mode in ("separate", "attend"):
+        g = wl.capture(GRAPH_STEPS, mode=mode)
+        legs[mode] = time_leg(g)
+        del g
     dense = DenseBaseline(wl)
-    g_dense = wl.graph(dense=dense)
-    for _ in range(3):
-        g_dense.replay()
-    torch.cuda.synchronize()
-    dense_reps = max(10, min(200, reps))
-    dense_us = time_graph(g_dense, dense_reps, stream) * 1000.0 / (dense_reps * GRAPH_STEPS)
+    g = wl.capture(GRAPH_STEPS, run=dense.step)
+    legs["dense"] = time_leg(g)
+    del g
+    att_us, dense_us = legs["attend"], legs["dense"]
+    dense_bytes = sum(4 * wl.B * wl.Hkv * L * wl.d for L in lens) / len(lens) + 4 * wl.B * wl.Hq * wl.d
+
+    # ---- the sparsity axis: attention alone over caches compressed at each sparsity (K and V alike),
+    # the same inputs, rotation and timing; dense fp16 on the same inputs is the leg above
+    by_sparsity = []
+    for sp in SPARSITY_AXIS:
+        pt = SparsityPoint(wl, sp)
+        g = wl.capture(GRAPH_STEPS, run=pt.step)
+        us = time_leg(g)
+        del g
+        b = sum(decode_algorithmic_bytes(wl.B, wl.Hq, wl.Hkv, wl.d, [L] * wl.B, pt.keep, pt.keep)
+                for L in lens) / len(lens)
+        by_sparsity.append({"sparsity": sp, "keep": pt.keep, "attend_us": us, "gbs": b / (us * 1e-6) / 1e9,
+                            "frac": b / (us * 1e-6) / 1e9 / peak, "algorithmic_bytes_per_launch": b,
+                            "dense_us": dense_us, "speedup_vs_dense": dense_us / us,
+                            "compressed_over_dense_bytes": pt.nbytes / wl.dense_cache_bytes})
+        del pt
+    dense.release()
 
     # ---- end to end through the public API with host buffers (eager calls)
     e2e = None
@@ -617,20 +725,22 @@ def main(argv=None):
                       "on side streams into two buffer sets, so they overlap the neighbouring steps"}
 
     line = {"metric": METRIC, "value": us_per_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": reps_w * GRAPH_STEPS, "ms_per_step": us_per_step / 1000.0, "higher_is_better": False,
+            "warmup": args.warmup, "ms_per_step": us_per_step / 1000.0, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config_dict(),
             "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "traffic": recorded_traffic(),
                          "kernel": "sparse_decode_kernel (fused append)", "algorithmic_bytes_per_launch": avg_bytes,
                          "us_per_launch": us_per_step * world, "splits": wl.splits},
-            "separate_launches": {"us_per_step": extra_us["separate"], "attend_us_per_launch": att_us,
-                                  "attend_frac": avg_bytes / (att_us * 1e-6) / 1e9 / peak,
-                                  "how": "append K + append V + decode_attn, 3 launches per step"},
-            "dense_baseline": {"us_per_launch": dense_us, "sparse_speedup": dense_us / att_us,
-                               "fused_step_speedup": dense_us / (us_per_step * world),
-                               "bytes_per_launch": sum(4 * wl.B * wl.Hkv * L * wl.d for L in lens) / len(lens)
-                               + 4 * wl.B * wl.Hq * wl.d},
+            "legs": {"how": f"replays of 64-step CUDA graphs, {leg_steps} steps each, same rotation",
+                     "fused_us": legs["fused"], "separate_us": legs["separate"], "attend_us": att_us,
+                     "dense_us": dense_us, "attend_frac": avg_bytes / (att_us * 1e-6) / 1e9 / peak,
+                     "dense_frac": dense_bytes / (dense_us * 1e-6) / 1e9 / peak,
+                     "sparse_speedup": dense_us / att_us, "fused_step_speedup": dense_us / legs["fused"],
+                     "fused_over_separate": legs["separate"] / legs["fused"],
+                     "separate": "append K + append V + decode_attn, 3 launches per step",
+                     "dense_bytes_per_launch": dense_bytes},
+            "by_sparsity": by_sparsity,
             "compressed_kv_bytes": wl.compressed_bytes,
             "clocks": clk, "e2e": e2e}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -638,7 +748,6 @@ def main(argv=None):
         line["cpu_baseline"]["all_cores"] = oracle_decode_all_cores()
     if rank == 0:
         print(json.dumps(line))
-    del g_step, g_dense
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -263,7 +263,7 @@ MUSTAFAR_API mustafar_status mustafar_dense_decode_attn(const void *q, int32_t n
 
 /* Bytes of device memory the library reserves (on every GPU that loads it, until the
  * process exits) for mustafar_decode_attn_noalloc's split-K scratch. */
-#define MUSTAFAR_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define MUSTAFAR_NOALLOC_SCRATCH_BYTES (16u << 20)
 
 /* Sparse decode attention that allocates nothing and takes no workspace.
  * The paper has no counterpart to this call: it exists for callers that cannot hand the
@@ -274,11 +274,13 @@ MUSTAFAR_API mustafar_status mustafar_dense_decode_attn(const void *q, int32_t n
  * the split-K partial states and ticket counters kept in a fixed array of
  * MUSTAFAR_NOALLOC_SCRATCH_BYTES inside the library instead.
  *   - A call whose split plan needs more scratch than that (a very large batch x heads x
- *     num_splits) is rejected with MUSTAFAR_ERR_WORKSPACE and a message.  On a 148-SM B200
- *     the automatic plan (num_splits = 0) always fits: it needs at most about 4.9 MB, reached
- *     with 16 q heads per kv head.
- *   - The first call on each device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *     num_splits) is rejected with MUSTAFAR_ERR_WORKSPACE and a message.  The automatic plan
+ *     (num_splits = 0) needs at most one wave of CTAs (SMs x 4) x 2 partial slots x
+ *     (32 + 128 G) x 4 bytes, plus 4 bytes per (batch row, kv head) for the ticket counters:
+ *     9.9 MB on a 148-SM B200 at G = 16 q heads per kv head, so it always fits there.
+ *   - Every call looks up the array's device address in the current device's context (a host
+ *     query; the first one on a device also loads the library's device code there), so make
+ *     the first call on each device before any stream capture.
  *   - Every call shares the one array, on every stream: calls that overlap on the GPU race
  *     and corrupt each other's results.  Each call first clears the ticket counters it uses.
  *   - No cudaMalloc, cudaFree or allocating library routine is called.

@@ -13,8 +13,8 @@ import time
 
 import torch
 
-from . import _lib as M
-from . import synth
+import unstructured_sparse_kv_b200 as M
+from unstructured_sparse_kv_b200 import synth
 
 D = 128
 FLUSH_BYTES = 256 << 20

@@ -86,6 +86,56 @@ def test_noalloc_rejects_a_plan_beyond_its_scratch():
     seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
     out = torch.empty_like(q)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=DEV)
-    st = _noalloc(lib, q, kc, vc, seq, L, out, lse, num_splits=128)  # 8*32*128 partial states > 8 MiB
+    st = _noalloc(lib, q, kc, vc, seq, L, out, lse, num_splits=128)  # 64 streams x 128 splits: 36 MB > 16 MiB
     assert st == 5  # MUSTAFAR_ERR_WORKSPACE
     assert "scratch" in lib.mustafar_last_error().decode()
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_noalloc_automatic_plan_fits_its_scratch(G):
+    # the automatic plan at a batch whose streams fill a whole wave of CTAs, for every supported group size:
+    # its split-K scratch must fit the fixed array, so the call is accepted and matches the workspace call
+    lib = M.load()
+    Hkv, L = 8, 2048
+    B = 32
+    Hq = G * Hkv
+    cap = L
+    K = synth.keys(B, Hkv, L, 128, 41, DEV)
+    V = synth.values(B, Hkv, L, 128, 41, DEV)
+    kc, vc = M.CompressedCache(B, Hkv, cap, 0.7), M.CompressedCache(B, Hkv, cap, 0.7)
+    M.mustafar_compress(K, L, 0.7, kc)
+    M.mustafar_compress(V, L, 0.7, vc)
+    seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    q = synth.queries(B, Hq, 128, 41, DEV)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=DEV)
+    st = _noalloc(lib, q, kc, vc, seq, L, out, lse)
+    assert st == 0, lib.mustafar_last_error().decode()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0)
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+
+
+def test_noalloc_call_allocates_no_device_memory():
+    # the property the entry point exists for: a warm call leaves the device's free memory unchanged
+    # (torch's caching allocator is not involved: the call only gets raw pointers)
+    lib = M.load()
+    B, Hq, Hkv, L = 8, 32, 8, 4096
+    K = synth.keys(B, Hkv, L, 128, 43, DEV)
+    V = synth.values(B, Hkv, L, 128, 43, DEV)
+    kc, vc = M.CompressedCache(B, Hkv, L, 0.7), M.CompressedCache(B, Hkv, L, 0.7)
+    M.mustafar_compress(K, L, 0.7, kc)
+    M.mustafar_compress(V, L, 0.7, vc)
+    del K, V
+    seq = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    q = synth.queries(B, Hq, 128, 43, DEV)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=DEV)
+    assert _noalloc(lib, q, kc, vc, seq, L, out, lse) == 0  # first call: loads the device code if needed
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _noalloc(lib, q, kc, vc, seq, L, out, lse) == 0
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before

@@ -17,25 +17,17 @@ namespace {
 
 // Split-K scratch for mustafar_decode_attn_noalloc.  Every GPU that loads the library holds
 // these bytes until the process exits.  Host code must not pass this symbol to a kernel: on the
-// host it is only a stand-in, so its device address is looked up once per device below.
+// host it is only a stand-in, so its device address is looked up below.
 static __device__ __align__(256) uint8_t g_decode_scratch[MUSTAFAR_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices];
-
-// Device address of g_decode_scratch on the current device (looked up on first use).
+// Device address of g_decode_scratch in the current device's context.  Looked up on every call
+// (a cheap host query once the module is loaded) rather than cached, so that a context created
+// again after cudaDeviceReset is never handed an address from the one before it.
 cudaError_t scratch_address(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

@@ -815,7 +815,17 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     } while (more && cs.n == 0);
     if (!more) break;
   }
-  if (timed_out && lane == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_TIMEOUT);
+  if (timed_out) {
+    // a copy that did not land in time may still be in flight into this warp's buffers: before the CTA
+    // can exit (and its shared memory be reused), wait once more, again bounded, for the latest copy
+    // issued into each buffer of the ring
+    if (lane == 0 && P.err != nullptr) atomicOr(P.err, MUSTAFAR_DEVERR_TIMEOUT);
+#pragma unroll 1
+    for (int s = 0; s < NSTAGE && s < citem; ++s) {
+      const int last = s + NSTAGE * ((citem - 1 - s) / NSTAGE);  // the latest item that used buffer s
+      mbar_wait(bars + 8 * s, (last / NSTAGE) & 1, kWaitCyclesAfter);
+    }
+  }
 
   // ---- tickets for the pieces shared with other CTAs; the last CTA of a stream merges it
   const int np = sh_npend;  // the partial stores are ordered before this by flush_piece's barrier

@@ -66,12 +66,48 @@ __device__ __forceinline__ uint32_t high_threshold(const uint32_t (&hb)[32], int
   for (int bit = 6; bit >= 0; --bit) {
     const uint32_t h = (T >> 8) | (1u << bit);
     const uint32_t c = (0x80u - h) * 0x01010101u;
-    uint32_t acc = 0;  // four per-byte counts (each at most 32)
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};  // four per-byte counts each (at most 8): four independent chains
 #pragma unroll
-    for (int r = 0; r < 32; ++r) acc += __umulhi((hb[r] + c) & 0x80808080u, 1u << 25);
-    if (static_cast<int>((acc * 0x01010101u) >> 24) >= k) T = h << 8;
+    for (int r = 0; r < 32; ++r) acc[r & 3] += __umulhi((hb[r] + c) & 0x80808080u, 1u << 25);
+    const uint32_t sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);  // each byte at most 32
+    if (static_cast<int>((sum * 0x01010101u) >> 24) >= k) T = h << 8;
   }
   return T;
+}
+
+// #{key >= T} over the 128 keys packed two per register, by fp16x2 compares: valid when T is a finite
+// fp16 pattern (T < 0x7C00) and only for keys that are not NaN.  set.ge gives 1.0 or 0.0 per half; the
+// sums (at most 16 per half in each of four accumulators) are exact in fp16.
+__device__ __forceinline__ uint32_t count_f16_ge(const uint32_t (&p)[64], uint32_t T) {
+  const uint32_t t2 = T | (T << 16);
+  uint32_t acc[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    uint32_t s;
+    asm("set.ge.f16x2.f16x2 %0, %1, %2;" : "=r"(s) : "r"(p[i]), "r"(t2));
+    asm("add.rn.f16x2 %0, %0, %1;" : "+r"(acc[i & 3]) : "r"(s));
+  }
+  uint32_t a01, a23, a;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(a01) : "r"(acc[0]), "r"(acc[1]));
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(a23) : "r"(acc[2]), "r"(acc[3]));
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(a) : "r"(a01), "r"(a23));
+  const __half2 h = *reinterpret_cast<const __half2 *>(&a);
+  return static_cast<uint32_t>(__half2float(__low2half(h)) + __half2float(__high2half(h)));
+}
+
+// #{key that is a NaN pattern (key > 0x7C00)} over the 128 packed keys (an unordered self-compare).
+__device__ __forceinline__ uint32_t count_f16_nan(const uint32_t (&p)[64]) {
+  uint32_t acc[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    uint32_t s;
+    asm("set.nan.f16x2.f16x2 %0, %1, %1;" : "=r"(s) : "r"(p[i]));
+    asm("add.rn.f16x2 %0, %0, %1;" : "+r"(acc[i & 1]) : "r"(s));
+  }
+  uint32_t a;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(a) : "r"(acc[0]), "r"(acc[1]));
+  const __half2 h = *reinterpret_cast<const __half2 *>(&a);
+  return static_cast<uint32_t>(__half2float(__low2half(h)) + __half2float(__high2half(h)));
 }
 
 // Kept-channel bitmap of the k largest keys, ties toward the lower channel index, given bits
@@ -81,11 +117,24 @@ __device__ __forceinline__ void topk_bitmap(const uint32_t (&raw)[64], int k, ui
   make_keys(raw, p);
   // bits 7..0 on the full keys, two per register
   uint32_t g[kWords];
+  if (T < 0x7C00u) {
+    // a finite threshold: a key is a non-negative fp16 bit pattern, and for two such patterns that are
+    // not NaN the integer order is the fp16 order, so the counts can use fp16x2 compares (one logic-pipe
+    // op per two keys instead of two); NaN keys rank above every finite candidate but compare false,
+    // so they are counted once and added
+    const uint32_t nan = count_f16_nan(p);
 #pragma unroll 1
-  for (int bit = 7; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    ge_bitmap(p, cand, g);
-    if (popc4(g) >= k) T = cand;
+    for (int bit = 7; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      if (count_f16_ge(p, cand) + nan >= static_cast<uint32_t>(k)) T = cand;
+    }
+  } else {
+#pragma unroll 1
+    for (int bit = 7; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      ge_bitmap(p, cand, g);
+      if (popc4(g) >= k) T = cand;
+    }
   }
   ge_bitmap(p, T, g);  // #{key >= T} >= k, and #{key > T} < k
   if (popc4(g) == k) {

@@ -154,6 +154,33 @@ def test_split_count_invariance():
         assert float((o.float() - outs[0][0].float()).abs().max()) <= 2e-3
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,L,ragged", [(8, 32, 8, 3000, True), (8, 32, 8, 2300, False), (37, 64, 4, 640, True)])
+def test_one_cluster_per_stream_plans(B, Hq, Hkv, L, ragged):
+    """Shapes whose automatic plan gives every stream the same number of CTAs (9 per stream at 8 x 8 kv
+    heads, 3 per stream at 37 x 4 with 16 q heads per kv head): those CTAs form one cluster per stream and
+    merge in distributed shared memory.  Ragged rows (one of them empty) and a fused decode step too."""
+    cap = ((L + 1 + 63) // 64) * 64
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.7, 0.5, 61)
+    seq = synth.seq_lens(B, L, ragged, 61)
+    if ragged:
+        seq[B // 2] = 0
+    rows = (seq > 0).nonzero().flatten()  # the oracle defines no output for an empty row
+    o_ref, l_ref = U.oracle_attention(q[rows], U.bits(K)[rows], U.bits(V)[rows], kc.keep, vc.keep,
+                                      seq[rows].numpy(), 1.0)
+    for splits, tag in ((0, f"cluster plan B{B} G{Hq // Hkv} ragged={ragged}"), (31, "ticket plan")):
+        out, lse = _attend(q, kc, vc, seq, L, splits=splits)
+        U.assert_attn_close(out[rows.to(DEV)], o_ref, lse[rows.to(DEV)], l_ref, tag=tag)
+        if ragged:
+            assert float(out[B // 2].abs().max()) == 0.0 and torch.isinf(lse[B // 2]).all() and (lse[B // 2] < 0).all()
+    # one fused step: the new token at position L of every row (rows of any length attend over L + 1)
+    kn, vn = synth.step_tokens(B, Hkv, D, 61, 0, DEV)
+    pos = torch.full((B,), L, dtype=torch.int32, device=DEV)
+    out, lse = M.mustafar_decode_step(q, kn, vn, pos, kc, vc, L + 1, 1.0)
+    K[:, :, L], V[:, :, L] = kn, vn
+    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, [L + 1] * B, 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag="cluster plan fused step")
+
+
 def test_seq_len_zero_and_beyond_capacity():
     B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 21)

@@ -305,6 +305,7 @@ mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *w
   p.lg_v = plan.lg_v;
   p.skew_k = plan.skew_k;
   p.skew_v = plan.skew_v;
+  p.clu = plan.clu;
   const size_t need = sparse_workspace_bytes(p.B, p.Hkv, p.G, plan.splits);
   if (workspace == nullptr || workspace_bytes < need)
     return fail(MUSTAFAR_ERR_WORKSPACE, "%s: workspace of %zu bytes needed (%d CTAs), got %zu", name, need,

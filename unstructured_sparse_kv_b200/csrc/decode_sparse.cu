@@ -34,6 +34,7 @@
 // counts); SKEW stages a cache whose keep is a multiple of 32 in 16-byte-skewed token groups so
 // that the runs do not all start on one shared-memory bank.
 #include <cfloat>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -74,6 +75,14 @@ __device__ __forceinline__ int row_len(const DecodeParams &P, int b, int cap) {
   return row_len(P, b, cap, ignored);
 }
 
+// Lengths of the batch rows below kRowCache, read once per CTA at the start (one round of
+// independent loads by warp 0) and kept in shared memory: the later look-ups of a row's length
+// (the plan, the rows a CTA reports, every stream step) then cost no global round trip.
+constexpr int kRowCache = 128;
+__device__ __forceinline__ int len_of(const DecodeParams &P, const int *sh_len, int b, int cap) {
+  return b < kRowCache ? sh_len[b] : row_len(P, b, cap);
+}
+
 // The chunk units of one stream in the end-to-end sequence: [start, start + n).
 struct Stream {
   int b, g;   // batch row, kv head
@@ -83,12 +92,12 @@ struct Stream {
 };
 
 // Step to the next stream in (b, g) order; false past the last one.
-__device__ __forceinline__ bool next_stream(const DecodeParams &P, int cap, Stream &s) {
+__device__ __forceinline__ bool next_stream(const DecodeParams &P, const int *sh_len, int cap, Stream &s) {
   s.start += s.n;
   if (++s.g == P.Hkv) {
     s.g = 0;
     if (++s.b >= P.B) return false;
-    s.n = n_chunks(row_len(P, s.b, cap));
+    s.n = n_chunks(len_of(P, sh_len, s.b, cap));
   }
   return true;
 }
@@ -380,7 +389,7 @@ __device__ __forceinline__ void consume_chunk(const DecodeParams &P, uint8_t *st
 
 // Write the merged row r (out, lse) of q head hq from its (m, l, o[c]) sums.
 __device__ __forceinline__ void write_row(const DecodeParams &P, int64_t hq, int c, float M, float lsum, float acc) {
-  P.out[hq * kHeadDim + c] = __half_as_ushort(__float2half_rn(lsum > 0.f ? acc / lsum : 0.f));
+  P.out[hq * kHeadDim + c] = __half_as_ushort(__float2half_rn(lsum > 0.f ? __fdividef(acc, lsum) : 0.f));
   if (c == 0 && P.lse != nullptr) P.lse[hq] = lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : kNegInf;
 }
 
@@ -392,8 +401,28 @@ struct Pending {
   int first_slot;  // workspace slot of CTA ca's partial (CTA ca + j > ca uses slot 2 (ca + j))
 };
 
+// ---- thread-block clusters: barrier over all threads of the cluster (release / acquire), and loads
+// from another CTA's shared memory
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t cta_rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(local_addr), "r"(cta_rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// Per-warp output rows in the merge area: channel c of (warp, head) row i at i * kMerStride +
+// mer_pos(c), 16-channel groups 18 floats apart.  A lane's accumulator pair (channels 16g + 2m,
+// +1 of one head) goes in with one 8-byte store, and the 16 lanes of a half warp (groups g, heads
+// 2q) then hit 16 different bank pairs; unpadded rows put them on two bank pairs (8-way conflicts).
+constexpr int kMerStride = 148;
+__device__ __forceinline__ int mer_pos(int c) { return c + 2 * (c >> 4); }
+
 // End of one piece [seg_a, ...) of stream st: the four warps merge their (m, l, o) in shared
-// memory (`mer`: m[4][16], l[4][16], o[4][G][128] fp32).  A stream held by this CTA alone is
+// memory (`mer`: m[4][16], l[4][16], o[4][G][kMerStride] fp32).  A stream held by this CTA alone is
 // written out; otherwise the CTA's partial goes to its workspace slot and the piece is queued in
 // `pend`.  Called by every thread of the CTA.
 template <bool HIROWS>
@@ -419,31 +448,77 @@ __device__ void flush_piece(const DecodeParams &P, Acc<HIROWS> &acc, float *mer,
   }
   {
     const int h0 = 2 * qq, h1 = 2 * qq + 1;
+    auto row = [&](int h) { return reinterpret_cast<float2 *>(sm_o + (warp * G + h) * kMerStride + 18 * gq); };
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      const int ch0 = 16 * gq + 2 * mt, ch1 = ch0 + 1;  // channels of accumulator rows g and g+8
-      if (h0 < G) {
-        sm_o[(warp * G + h0) * kHeadDim + ch0] = acc.ot[mt][0];
-        sm_o[(warp * G + h0) * kHeadDim + ch1] = acc.ot[mt][2];
-      }
-      if (h1 < G) {
-        sm_o[(warp * G + h1) * kHeadDim + ch0] = acc.ot[mt][1];
-        sm_o[(warp * G + h1) * kHeadDim + ch1] = acc.ot[mt][3];
-      }
+      // accumulator rows g and g+8 are channels 16g + 2mt and 16g + 2mt + 1: mer_pos = 18g + 2mt, +1
+      if (h0 < G) row(h0)[mt] = make_float2(acc.ot[mt][0], acc.ot[mt][2]);
+      if (h1 < G) row(h1)[mt] = make_float2(acc.ot[mt][1], acc.ot[mt][3]);
       if constexpr (HIROWS) {
-        if (h0 + 8 < G) {
-          sm_o[(warp * G + h0 + 8) * kHeadDim + ch0] = acc.oh[mt][0];
-          sm_o[(warp * G + h0 + 8) * kHeadDim + ch1] = acc.oh[mt][2];
-        }
-        if (h1 + 8 < G) {
-          sm_o[(warp * G + h1 + 8) * kHeadDim + ch0] = acc.oh[mt][1];
-          sm_o[(warp * G + h1 + 8) * kHeadDim + ch1] = acc.oh[mt][3];
-        }
+        if (h0 + 8 < G) row(h0 + 8)[mt] = make_float2(acc.oh[mt][0], acc.oh[mt][2]);
+        if (h1 + 8 < G) row(h1 + 8)[mt] = make_float2(acc.oh[mt][1], acc.oh[mt][3]);
       }
     }
   }
   __syncthreads();
 
+  if (P.clu > 0) {
+    // one cluster per stream: this CTA's merged (m, l, o) replaces the per-warp states in `mer`, then,
+    // after a cluster barrier, CTA rank j merges rows j, j + C, ... of the cluster's C partials through
+    // distributed shared memory and writes them out; a second barrier keeps every CTA's partial alive
+    // until all reads are done.  Every thread of every CTA of the cluster reaches both barriers.
+    static_assert(kThreads == kHeadDim, "one thread per output channel");
+    const int c = threadIdx.x;
+    float pm[16], pl[16], po[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      pm[r] = kNegInf;
+      pl[r] = po[r] = 0.f;
+      if (r < G) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) pm[r] = fmaxf(pm[r], sm_m[w * 16 + r]);
+        if (pm[r] != kNegInf) {
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const float wt = fast_exp2(sm_m[w * 16 + r] - pm[r]);
+            pl[r] += sm_l[w * 16 + r] * wt;
+            po[r] += sm_o[(w * G + r) * kMerStride + mer_pos(c)] * wt;
+          }
+        }
+      }
+    }
+    __syncthreads();  // every thread has read the per-warp states
+    float *cpart = mer;  // m[16], l[16], o[G][128]
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if (r < G) {
+        cpart[32 + r * kHeadDim + c] = po[r];
+        if (c == 0) {
+          cpart[r] = pm[r];
+          cpart[16 + r] = pl[r];
+        }
+      }
+    }
+    cluster_sync_all();
+    const int C = P.clu, rank = cta % C;
+    const uint32_t cbase = smem_addr(cpart);
+    const int64_t hq0 = static_cast<int64_t>(st.b) * P.Hq + static_cast<int64_t>(st.g) * G;
+    for (int r = rank; r < G; r += C) {
+      float M = kNegInf;
+      for (int j = 0; j < C; ++j) M = fmaxf(M, ld_cluster_f32(cbase + 4 * r, j));
+      float lsum = 0.f, o = 0.f;
+      if (M != kNegInf) {
+        for (int j = 0; j < C; ++j) {
+          const float wt = fast_exp2(ld_cluster_f32(cbase + 4 * r, j) - M);
+          lsum += ld_cluster_f32(cbase + 4 * (16 + r), j) * wt;
+          o += ld_cluster_f32(cbase + 4 * (32 + r * kHeadDim + c), j) * wt;
+        }
+      }
+      write_row(P, hq0 + r, c, M, lsum, o);
+    }
+    cluster_sync_all();
+    return;
+  }
   // the CTAs holding part of this stream: ca .. cb (an empty range that starts exactly where
   // the stream starts belongs to no stream)
   const int ca = cta_of(st.start, U, nctas), cb = cta_of(st.end() - 1, U, nctas);
@@ -452,26 +527,44 @@ __device__ void flush_piece(const DecodeParams &P, Acc<HIROWS> &acc, float *mer,
     const int c = threadIdx.x;  // output channel
     const int64_t hq0 = static_cast<int64_t>(st.b) * P.Hq + static_cast<int64_t>(st.g) * G;
     float *part = P.ws_part + static_cast<int64_t>(2 * cta + (seg_a == u0 ? 0 : 1)) * slot_floats;
-    for (int r = 0; r < G; ++r) {
-      float M = kNegInf;
+    const int pc = mer_pos(c);
+    // four rows at a time, all their shared loads issued before any result is used
+    for (int r0 = 0; r0 < G; r0 += 4) {
+      float M[4], lsum[4], o[4];
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w * 16 + r]);
-      float lsum = 0.f, o = 0.f;
-      if (M != kNegInf) {
+      for (int j = 0; j < 4; ++j) {
+        const int r = r0 + j;
+        M[j] = kNegInf;
+        lsum[j] = o[j] = 0.f;
+        if (r < G) {
+          float mw[kWarps];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float wt = fast_exp2(sm_m[w * 16 + r] - M);
-          lsum += sm_l[w * 16 + r] * wt;
-          o += sm_o[(w * G + r) * kHeadDim + c] * wt;
+          for (int w = 0; w < kWarps; ++w) {
+            mw[w] = sm_m[w * 16 + r];
+            M[j] = fmaxf(M[j], mw[w]);
+          }
+          if (M[j] != kNegInf) {
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+              const float wt = fast_exp2(mw[w] - M[j]);
+              lsum[j] += sm_l[w * 16 + r] * wt;
+              o[j] += sm_o[(w * G + r) * kMerStride + pc] * wt;
+            }
+          }
         }
       }
-      if (ca == cb) {
-        write_row(P, hq0 + r, c, M, lsum, o);
-      } else {
-        part[32 + r * kHeadDim + c] = o;
-        if (c == 0) {
-          part[r] = M;
-          part[16 + r] = lsum;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = r0 + j;
+        if (r >= G) continue;
+        if (ca == cb) {
+          write_row(P, hq0 + r, c, M[j], lsum[j], o[j]);
+        } else {
+          part[32 + r * kHeadDim + c] = o[j];
+          if (c == 0) {
+            part[r] = M[j];
+            part[16 + r] = lsum[j];
+          }
         }
       }
     }
@@ -578,6 +671,9 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
   __shared__ int sh_info[3];  // U, batch row of this CTA's first unit (-1: none), that row's first unit
+  __shared__ int sh_len[kRowCache];
+  __shared__ int sh_pos[kRowCache];  // fused step: the new token's position in each row
+  __shared__ uint32_t sh_bits;       // device error flags of the cached rows this CTA reports
   __shared__ Pending sh_pend[2];
   __shared__ int sh_npend, sh_last[2];
   __shared__ uint2 lut24[16];
@@ -585,50 +681,73 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   const int cta = blockIdx.x, nctas = gridDim.x;
   const int cap = min(P.cap_k, P.cap_v);
 
-  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts (rows up
-  // to 128 are read once, in one round of independent loads, and kept in registers)
+  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts.  Warp 0
+  // reads the lengths of rows below kRowCache in one round of independent loads into sh_len (and
+  // the error flags of the rows this CTA reports); longer batches read the rest from global memory.
+  // With one cluster per stream, the cluster's C CTAs split that stream's chunks evenly and nothing
+  // else.
   if (warp == 0) {
-    int nrow[4];
+    int nrow[kRowCache / 32];
     int tot = 0;
+    uint32_t bits = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kRowCache / 32; ++i) {
       const int b = lane + 32 * i;
-      nrow[i] = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
+      int L = 0;
+      if (b < P.B) {
+        uint32_t rb = 0;
+        L = row_len(P, b, cap, rb);
+        sh_len[b] = L;
+        if (P.pos != nullptr) sh_pos[b] = P.pos[b];
+        if (b % nctas == cta) bits |= rb;
+      }
+      nrow[i] = P.Hkv * n_chunks(L);
       tot += nrow[i];
     }
-    for (int b = 128 + lane; b < P.B; b += 32) tot += P.Hkv * n_chunks(row_len(P, b, cap));
+    bits = __reduce_or_sync(0xffffffffu, bits);
+    if (lane == 0) sh_bits = bits;
+    if (P.clu > 0) {
+      if (lane == 0) {
+        const int s = cta / P.clu;
+        sh_info[0] = 0;
+        sh_info[1] = s / P.Hkv;
+        sh_info[2] = s % P.Hkv;
+      }
+    } else {
+      for (int b = kRowCache + lane; b < P.B; b += 32) tot += P.Hkv * n_chunks(row_len(P, b, cap));
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    const int u0 = range_start(cta, tot, nctas);
-    int row = -1, row_start = 0, before = 0;
-    for (int b0 = 0; b0 < P.B && u0 < tot; b0 += 32) {
-      const int b = b0 + lane;
-      int n;
-      if (b0 < 128) {
-        const int i = b0 >> 5;
-        n = i == 0 ? nrow[0] : i == 1 ? nrow[1] : i == 2 ? nrow[2] : nrow[3];
-      } else {
-        n = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
-      }
-      int incl = n;
+      for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      const int u0 = range_start(cta, tot, nctas);
+      int row = -1, row_start = 0, before = 0;
+      for (int b0 = 0; b0 < P.B && u0 < tot; b0 += 32) {
+        const int b = b0 + lane;
+        int n;
+        if (b0 < kRowCache) {
+          const int i = b0 >> 5;
+          n = i == 0 ? nrow[0] : i == 1 ? nrow[1] : i == 2 ? nrow[2] : nrow[3];
+        } else {
+          n = b < P.B ? P.Hkv * n_chunks(row_len(P, b, cap)) : 0;
+        }
+        int incl = n;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, before + incl > u0);
+        if (hit != 0u) {
+          const int f = __ffs(hit) - 1;
+          row = b0 + f;
+          row_start = before + __shfl_sync(0xffffffffu, incl - n, f);
+          break;
+        }
+        before += __shfl_sync(0xffffffffu, incl, 31);
       }
-      const unsigned hit = __ballot_sync(0xffffffffu, before + incl > u0);
-      if (hit != 0u) {
-        const int f = __ffs(hit) - 1;
-        row = b0 + f;
-        row_start = before + __shfl_sync(0xffffffffu, incl - n, f);
-        break;
+      if (lane == 0) {
+        sh_info[0] = tot;
+        sh_info[1] = row;
+        sh_info[2] = row_start;
       }
-      before += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) {
-      sh_info[0] = tot;
-      sh_info[1] = row;
-      sh_info[2] = row_start;
     }
   }
   if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
@@ -645,13 +764,17 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   }
   __syncthreads();
   const int U = sh_info[0];
-  const int u0 = range_start(cta, U, nctas), u1 = range_start(cta + 1, U, nctas);
+  int u0 = range_start(cta, U, nctas), u1 = range_start(cta + 1, U, nctas);
+  if (P.clu > 0) {  // units are counted from the stream's first chunk
+    const int n = n_chunks(len_of(P, sh_len, sh_info[1], cap)), r = cta % P.clu;
+    u0 = static_cast<int>(static_cast<long long>(r) * n / P.clu);
+    u1 = static_cast<int>(static_cast<long long>(r + 1) * n / P.clu);
+  }
 
   // ---- rows this CTA reports on: device error flags, and the output of rows with no tokens
+  uint32_t bits = sh_bits;
   for (int b = cta; b < P.B; b += nctas) {
-    uint32_t bits = 0;
-    const int L = row_len(P, b, cap, bits);
-    if (threadIdx.x == 0 && bits != 0u && P.err != nullptr) atomicOr(P.err, bits);
+    const int L = b < kRowCache ? sh_len[b] : row_len(P, b, cap, bits);
     if (L == 0) {
       uint16_t *o = P.out + static_cast<int64_t>(b) * P.Hq * kHeadDim;
       for (int i = threadIdx.x; i < P.Hq * kHeadDim; i += kThreads) o[i] = 0;
@@ -659,13 +782,19 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
         for (int i = threadIdx.x; i < P.Hq; i += kThreads) P.lse[static_cast<int64_t>(b) * P.Hq + i] = kNegInf;
     }
   }
-  if (sh_info[1] < 0) return;  // an empty range at the end of the sequence
+  if (threadIdx.x == 0 && bits != 0u && P.err != nullptr) atomicOr(P.err, bits);
+  if (sh_info[1] < 0) return;  // an empty range at the end of the sequence (never with clusters)
 
   Stream first;
   first.b = sh_info[1];
-  first.n = n_chunks(row_len(P, first.b, cap));
-  first.g = (u0 - sh_info[2]) / first.n;
-  first.start = sh_info[2] + first.g * first.n;
+  first.n = n_chunks(len_of(P, sh_len, first.b, cap));
+  if (P.clu > 0) {
+    first.g = sh_info[2];
+    first.start = 0;
+  } else {
+    first.g = (u0 - sh_info[2]) / first.n;
+    first.start = sh_info[2] + first.g * first.n;
+  }
 
   // ---- fused decode step: compress the new token of every stream whose new-token chunk lies in
   // this range (warp 0: K, warp 1: V) before any chunk is copied in
@@ -673,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     Stream st = first;
     bool any = false;
     while (st.start < u1) {
-      const int p = P.pos[st.b];
+      const int p = st.b < kRowCache ? sh_pos[st.b] : P.pos[st.b];
       if (st.n > 0 && p >= 0 && p < cap) {
         const int unit = st.start + p / kChunk;
         if (unit >= u0 && unit < u1) {
@@ -700,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
           }
         }
       }
-      if (!next_stream(P, cap, st)) break;
+      if (!next_stream(P, sh_len, cap, st)) break;
     }
     if (any) {
       fence_proxy_async_global();  // these stores before the bulk copies that read them
@@ -719,7 +848,11 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     sh_punit[warp] = u0 + warp;
   }
   __syncwarp();
-  auto produce = [&](int item) {
+  // ALL4 (the first fill of the ring, when nothing else runs yet): lanes 0-3 issue a chunk's four
+  // copies together; in the chunk loop lane 0 issues them (four more lanes' addresses there would
+  // spill registers)
+  auto produce = [&](int item, auto all4) {
+    constexpr bool ALL4 = decltype(all4)::value;
     if constexpr (SKEW) {
       // a cache whose keep is a multiple of 32 is staged in groups of 2^lg tokens (about 256 bytes),
       // each group 16 bytes after the previous one ends: otherwise every token's run starts on the
@@ -728,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       const int punit = sh_punit[warp];
       if (punit >= u1) return;  // the same in every lane
       Stream ps = sh_ps[warp];
-      while (punit >= ps.end()) next_stream(P, cap, ps);
+      while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
       const int slot = item % NSTAGE;
       const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
       const uint32_t bar = bars + 8 * slot;
@@ -754,36 +887,58 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       }
       return;
     }
-    if (lane != 0) return;
-    int punit = sh_punit[warp];
-    if (punit >= u1) return;
+    if (lane >= (ALL4 ? 4 : 1)) return;
+    const int punit = sh_punit[warp];
+    if (punit >= u1) return;  // the same in lanes 0-3
     Stream ps = sh_ps[warp];
-    while (punit >= ps.end()) next_stream(P, cap, ps);
+    while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
     const int slot = item % NSTAGE;
     const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
     const uint32_t bar = bars + 8 * slot;
     const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
     const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
     const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
-    if constexpr (PERHEAD) {
-      const int kK = P.hk_k.k[ps.g], kV = P.hk_v.k[ps.g];
+    // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
+    const int kK = PERHEAD ? P.hk_k.k[ps.g] : P.keep_k, kV = PERHEAD ? P.hk_v.k[ps.g] : P.keep_v;
+    if (!ALL4) {
       mbar_expect_tx(bar, 512 + 32 * (kK + kV));
       bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
       bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-      bulk_g2s(dst + 512, P.kval + P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK, 32 * kK, bar);
-      bulk_g2s(dst + 512 + 32 * kK, P.vval + P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV, 32 * kV, bar);
-    } else {  // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
-      mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
-      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
-      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
-      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
+      bulk_g2s(dst + 512, P.kval + (PERHEAD ? P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK : tk * kK),
+               32 * kK, bar);
+      bulk_g2s(dst + 512 + 32 * kK,
+               P.vval + (PERHEAD ? P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV : tv * kV), 32 * kV, bar);
+      sh_ps[warp] = ps;
+      sh_punit[warp] = punit + kWarps;
+      return;
     }
-    sh_ps[warp] = ps;
-    sh_punit[warp] = punit + kWarps;
+    // lanes 0-3: K bitmaps, V bitmaps, K values, V values, after lane 0 has announced their bytes
+    if (lane == 0) mbar_expect_tx(bar, 512 + 32 * (kK + kV));
+    __syncwarp(0xFu);
+    const void *src;
+    uint32_t off, bytes;
+    if (lane < 2) {
+      src = lane == 0 ? static_cast<const void *>(P.kbm + tk * kWords) : static_cast<const void *>(P.vbm + tv * kWords);
+      off = 256 * lane;
+      bytes = 256;
+    } else if (lane == 2) {
+      src = P.kval + (PERHEAD ? P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK : tk * kK);
+      off = 512;
+      bytes = 32 * kK;
+    } else {
+      src = P.vval + (PERHEAD ? P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV : tv * kV);
+      off = 512 + 32 * kK;
+      bytes = 32 * kV;
+    }
+    bulk_g2s(dst + off, src, bytes, bar);
+    __syncwarp(0xFu);  // lanes 0-3 have read the producer state before lane 0 moves it on
+    if (lane == 0) {
+      sh_ps[warp] = ps;
+      sh_punit[warp] = punit + kWarps;
+    }
   };
 #pragma unroll 1
-  for (int i = 0; i < NSTAGE; ++i) produce(i);
+  for (int i = 0; i < NSTAGE; ++i) produce(i, std::true_type{});
 
   Stream cs = first;
   int cunit = u0 + warp, citem = 0;
@@ -792,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   uint32_t qa[8][4];
   for (;;) {
     const int seg_a = max(cs.start, u0), seg_e = min(cs.end(), u1);
-    const int L = row_len(P, cs.b, cap);
+    const int L = len_of(P, sh_len, cs.b, cap);
     const int kK = keep_of<PERHEAD>(P.hk_k, P.keep_k, cs.g), kV = keep_of<PERHEAD>(P.hk_v, P.keep_v, cs.g);
     load_q<HIROWS>(P, cs.b, cs.g, lane, qa);
     acc.reset();
@@ -805,13 +960,13 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       consume_chunk<HIROWS, PERHEAD, P24, SCAN, SKEW>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
                                           lut24);
       __syncwarp();
-      produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
+      produce(citem + NSTAGE, std::false_type{});  // the unit NSTAGE items ahead goes into the buffer just read
     }
     flush_piece<HIROWS>(P, acc, mer, warp, lane, cs, seg_a, u0, U, cta, nctas, sh_pend, &sh_npend);
     if (seg_e >= u1) break;
     bool more;
     do {
-      more = next_stream(P, cap, cs);
+      more = next_stream(P, sh_len, cap, cs);
     } while (more && cs.n == 0);
     if (!more) break;
   }
@@ -915,6 +1070,47 @@ cudaError_t resident_ctas(SparseFn fn, int slot, int smem, int *per_sm) {
   return e;
 }
 
+// Whether `clusters` clusters of C CTAs of this kernel (one per stream) are resident on the device at
+// once, cached per (device, kernel, C) with the shared memory it was asked for, so that planning stays
+// capture-safe once warm.  Sizes above 8 need the kernel's non-portable cluster attribute, set here.
+bool clusters_fit(SparseFn fn, int slot, int smem, int C, int clusters) {
+  constexpr int kDevs = 16, kMaxC = 16;
+  static int cache_smem[kDevs][kKernelSlots][kMaxC + 1];
+  static int cache_val[kDevs][kKernelSlots][kMaxC + 1];
+  int dev = 0;
+  if (C < 2 || C > kMaxC || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs || slot < 0 ||
+      slot >= kKernelSlots)
+    return false;
+  if (cache_smem[dev][slot][C] != smem) {
+    int n = 0;
+    if (C > 8 && cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                      1) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = -1;
+    }
+    if (n == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(C));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = static_cast<unsigned>(C);
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = -1;
+      }
+    }
+    cache_smem[dev][slot][C] = smem;
+    cache_val[dev][slot][C] = n;
+  }
+  return cache_val[dev][slot][C] >= clusters;
+}
+
 }  // namespace
 
 int sparse_decode_ctas(int B, int Hkv, int max_len, int forced_splits, int per_sm) {
@@ -975,7 +1171,7 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
   plan->skew_v = plan->lg_v < 4 ? 16 * (kChunk >> plan->lg_v) : 0;
   if (plan->skew_k || plan->skew_v) variant = 4;
   const int stage_bytes = round_up(512 + 32 * (keep_k + keep_v) + plan->skew_k + plan->skew_v, 128);
-  const int merge_bytes = (2 * kWarps * 16 + kWarps * G * kHeadDim) * 4;
+  const int merge_bytes = (2 * kWarps * 16 + kWarps * G * kMerStride) * 4;
   auto warp_bytes_of = [&](int ns) { return round_up(ns * stage_bytes + 512 + 8 * ns, 128); };
   int nstage = 2;
   for (int ns = 4; ns > 2; --ns)
@@ -995,6 +1191,15 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
   per_sm = per_sm < 1 ? 1 : (per_sm > kMaxCtasPerSm ? kMaxCtasPerSm : per_sm);
   plan->splits = sparse_decode_ctas(B, Hkv, max_len, forced_splits, per_sm);
   plan->chunks_per_split = 0;
+  // the automatic plan gives every stream the same whole number C of CTAs when that fills the wave;
+  // then each stream's CTAs form one thread-block cluster that merges its partials in distributed
+  // shared memory (no global partials, no tickets), provided all the clusters are resident at once
+  plan->clu = 0;
+  const long long streams = static_cast<long long>(B) * Hkv;
+  if (forced_splits <= 0 && plan->splits % streams == 0) {
+    const int C = static_cast<int>(plan->splits / streams);
+    if (C >= 2 && C <= 16 && clusters_fit(fn, slot, smem, C, static_cast<int>(streams))) plan->clu = C;
+  }
   plan->nstage = nstage;
   plan->stage_bytes = stage_bytes;
   plan->warp_bytes = warp_bytes;
@@ -1005,6 +1210,21 @@ cudaError_t plan_sparse(int B, int Hkv, int G, int max_len, int keep_k, int keep
 
 cudaError_t launch_sparse(const DecodeParams &p, const DecodePlan &plan, cudaStream_t stream) {
   SparseFn fn = pick_sparse(plan.nstage, p.G > 8, plan.variant);
+  if (plan.clu > 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.splits));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem_bytes);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = static_cast<unsigned>(plan.clu);
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, p);
+  }
   fn<<<plan.splits, kThreads, plan.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }

@@ -86,6 +86,8 @@ struct DecodeParams {
   int skew_k, skew_v;  // sparse kernel: bytes those gaps add to the cache's staged region
   uint16_t *out;
   float *lse;
+  int clu;            // sparse kernel: 0, or the CTAs of one thread-block cluster per stream (each takes an
+                      // equal share of its stream's chunks; partials merge in distributed shared memory)
   float *ws_part;     // sparse kernel: [2 * ctas][32 + G*128] partial (m, l, o) slots
   float *ws_o;        // [B*Hq][splits][128]
   float *ws_ml;       // [B*Hq][splits][2]
@@ -109,6 +111,7 @@ struct DecodePlan {
   int lg_k, lg_v, skew_k, skew_v;  // sparse kernel: staging groups of a keep that is a multiple of 32
   int variant;  // sparse kernel: 0 uniform caches, 1 a keep count per kv head, 2 both caches 2:4,
                 // 3 token runs located by popcount prefixes (a channel-wise cache)
+  int clu;      // sparse kernel: CTAs per thread-block cluster, one cluster per stream (0: no clusters)
 };
 
 // Dense fp16 baseline: plan (split count, pipeline depth, shared memory) and launch.

@@ -34,7 +34,6 @@
 // counts); SKEW stages a cache whose keep is a multiple of 32 in 16-byte-skewed token groups so
 // that the runs do not all start on one shared-memory bank.
 #include <cfloat>
-#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -102,12 +101,20 @@ __device__ __forceinline__ bool next_stream(const DecodeParams &P, const int *sh
   return true;
 }
 
+// floor(p / d) for 0 <= p, 0 < d: a 32-bit division whenever p fits (every shape up to about 2^31
+// chunk-CTA products), which is several times shorter than the 64-bit routine on this latency path
+__device__ __forceinline__ long long div_floor(long long p, long long d) {
+  if (p <= 0xFFFFFFFFLL && d <= 0xFFFFFFFFLL)
+    return static_cast<long long>(static_cast<uint32_t>(p) / static_cast<uint32_t>(d));
+  return p / d;
+}
+
 // The CTA whose range holds unit u: ranges are [floor(c U / n), floor((c+1) U / n)).
 __device__ __forceinline__ int cta_of(long long u, long long U, long long n) {
-  return static_cast<int>(((u + 1) * n - 1) / U);
+  return static_cast<int>(div_floor((u + 1) * n - 1, U));
 }
 __device__ __forceinline__ int range_start(long long c, long long U, long long n) {
-  return static_cast<int>(c * U / n);
+  return static_cast<int>(div_floor(c * U, n));
 }
 
 // x = (bits & MASK) ? the fp16 at shared address ra : 0 (read from the CTA's zero slot `za`);
@@ -670,7 +677,7 @@ template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24, bool SCAN, bool SKEW>
 __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
-  __shared__ int sh_info[3];  // U, batch row of this CTA's first unit (-1: none), that row's first unit
+  __shared__ int sh_info[5];  // U, batch row of the CTA's first unit (-1: none), that row's first unit, u0, u1
   __shared__ int sh_len[kRowCache];
   __shared__ int sh_pos[kRowCache];  // fused step: the new token's position in each row
   __shared__ uint32_t sh_bits;       // device error flags of the cached rows this CTA reports
@@ -707,11 +714,15 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     bits = __reduce_or_sync(0xffffffffu, bits);
     if (lane == 0) sh_bits = bits;
     if (P.clu > 0) {
+      // units are counted from the stream's first chunk
       if (lane == 0) {
-        const int s = cta / P.clu;
+        const int s = cta / P.clu, r = cta % P.clu, b = s / P.Hkv;
+        const int n = n_chunks(len_of(P, sh_len, b, cap));
         sh_info[0] = 0;
-        sh_info[1] = s / P.Hkv;
+        sh_info[1] = b;
         sh_info[2] = s % P.Hkv;
+        sh_info[3] = r * n / P.clu;
+        sh_info[4] = (r + 1) * n / P.clu;
       }
     } else {
       for (int b = kRowCache + lane; b < P.B; b += 32) tot += P.Hkv * n_chunks(row_len(P, b, cap));
@@ -747,6 +758,8 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
         sh_info[0] = tot;
         sh_info[1] = row;
         sh_info[2] = row_start;
+        sh_info[3] = u0;
+        sh_info[4] = range_start(cta + 1, tot, nctas);
       }
     }
   }
@@ -763,13 +776,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     mbar_init_fence();
   }
   __syncthreads();
-  const int U = sh_info[0];
-  int u0 = range_start(cta, U, nctas), u1 = range_start(cta + 1, U, nctas);
-  if (P.clu > 0) {  // units are counted from the stream's first chunk
-    const int n = n_chunks(len_of(P, sh_len, sh_info[1], cap)), r = cta % P.clu;
-    u0 = static_cast<int>(static_cast<long long>(r) * n / P.clu);
-    u1 = static_cast<int>(static_cast<long long>(r + 1) * n / P.clu);
-  }
+  const int U = sh_info[0], u0 = sh_info[3], u1 = sh_info[4];
 
   // ---- rows this CTA reports on: device error flags, and the output of rows with no tokens
   uint32_t bits = sh_bits;
@@ -848,11 +855,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     sh_punit[warp] = u0 + warp;
   }
   __syncwarp();
-  // ALL4 (the first fill of the ring, when nothing else runs yet): lanes 0-3 issue a chunk's four
-  // copies together; in the chunk loop lane 0 issues them (four more lanes' addresses there would
-  // spill registers)
-  auto produce = [&](int item, auto all4) {
-    constexpr bool ALL4 = decltype(all4)::value;
+  auto produce = [&](int item) {
     if constexpr (SKEW) {
       // a cache whose keep is a multiple of 32 is staged in groups of 2^lg tokens (about 256 bytes),
       // each group 16 bytes after the previous one ends: otherwise every token's run starts on the
@@ -887,9 +890,9 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       }
       return;
     }
-    if (lane >= (ALL4 ? 4 : 1)) return;
-    const int punit = sh_punit[warp];
-    if (punit >= u1) return;  // the same in lanes 0-3
+    if (lane != 0) return;
+    int punit = sh_punit[warp];
+    if (punit >= u1) return;
     Stream ps = sh_ps[warp];
     while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
     const int slot = item % NSTAGE;
@@ -898,47 +901,25 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
     const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
     const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
-    // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
-    const int kK = PERHEAD ? P.hk_k.k[ps.g] : P.keep_k, kV = PERHEAD ? P.hk_v.k[ps.g] : P.keep_v;
-    if (!ALL4) {
+    if constexpr (PERHEAD) {
+      const int kK = P.hk_k.k[ps.g], kV = P.hk_v.k[ps.g];
       mbar_expect_tx(bar, 512 + 32 * (kK + kV));
       bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
       bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-      bulk_g2s(dst + 512, P.kval + (PERHEAD ? P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK : tk * kK),
-               32 * kK, bar);
-      bulk_g2s(dst + 512 + 32 * kK,
-               P.vval + (PERHEAD ? P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV : tv * kV), 32 * kV, bar);
-      sh_ps[warp] = ps;
-      sh_punit[warp] = punit + kWarps;
-      return;
+      bulk_g2s(dst + 512, P.kval + P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK, 32 * kK, bar);
+      bulk_g2s(dst + 512 + 32 * kK, P.vval + P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV, 32 * kV, bar);
+    } else {  // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
+      mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
+      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
+      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
     }
-    // lanes 0-3: K bitmaps, V bitmaps, K values, V values, after lane 0 has announced their bytes
-    if (lane == 0) mbar_expect_tx(bar, 512 + 32 * (kK + kV));
-    __syncwarp(0xFu);
-    const void *src;
-    uint32_t off, bytes;
-    if (lane < 2) {
-      src = lane == 0 ? static_cast<const void *>(P.kbm + tk * kWords) : static_cast<const void *>(P.vbm + tv * kWords);
-      off = 256 * lane;
-      bytes = 256;
-    } else if (lane == 2) {
-      src = P.kval + (PERHEAD ? P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK : tk * kK);
-      off = 512;
-      bytes = 32 * kK;
-    } else {
-      src = P.vval + (PERHEAD ? P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV : tv * kV);
-      off = 512 + 32 * kK;
-      bytes = 32 * kV;
-    }
-    bulk_g2s(dst + off, src, bytes, bar);
-    __syncwarp(0xFu);  // lanes 0-3 have read the producer state before lane 0 moves it on
-    if (lane == 0) {
-      sh_ps[warp] = ps;
-      sh_punit[warp] = punit + kWarps;
-    }
+    sh_ps[warp] = ps;
+    sh_punit[warp] = punit + kWarps;
   };
 #pragma unroll 1
-  for (int i = 0; i < NSTAGE; ++i) produce(i, std::true_type{});
+  for (int i = 0; i < NSTAGE; ++i) produce(i);
 
   Stream cs = first;
   int cunit = u0 + warp, citem = 0;
@@ -960,7 +941,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       consume_chunk<HIROWS, PERHEAD, P24, SCAN, SKEW>(P, stage, htab, za, (cunit - cs.start) * kChunk, L, kK, kV, lane, qa, acc,
                                           lut24);
       __syncwarp();
-      produce(citem + NSTAGE, std::false_type{});  // the unit NSTAGE items ahead goes into the buffer just read
+      produce(citem + NSTAGE);  // the unit NSTAGE items ahead goes into the buffer just read
     }
     flush_piece<HIROWS>(P, acc, mer, warp, lane, cs, seg_a, u0, U, cta, nctas, sh_pend, &sh_npend);
     if (seg_e >= u1) break;

@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MUSTAFAR_ABI_VERSION 4
+#define MUSTAFAR_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define MUSTAFAR_API __attribute__((visibility("default")))
@@ -297,6 +297,18 @@ MUSTAFAR_API mustafar_status mustafar_decode_attn_noalloc(const void *q, int32_t
  * benchmarks and tests).  Returns a value >= 1, or -1 on invalid shapes. */
 MUSTAFAR_API int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t head_dim,
                                     int32_t max_len, int32_t keep_k, int32_t keep_v, int32_t dense);
+
+/* How the automatic plan of mustafar_decode_attn merges the split-K partials of a pair of
+ * uniform token-wise caches (host query, for benchmarks and tests; num_splits = 0).  When the
+ * plan gives every (batch row, kv head) stream the same number C of CTAs and all B * Hkv
+ * clusters of C CTAs fit on the device at once, each stream's CTAs run as one thread-block
+ * cluster and merge in distributed shared memory: the call returns C (2..16).  It returns 0 when
+ * the partials go through the workspace and a per-stream ticket instead (one CTA per stream, or
+ * CTAs per stream not whole, above 16 or not all resident), and -1 on invalid shapes.  Both
+ * merges compute the same log-sum-exp combination of the same partials. */
+MUSTAFAR_API int32_t mustafar_decode_plan_cluster(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                                  int32_t head_dim, int32_t max_len, int32_t keep_k,
+                                                  int32_t keep_v);
 
 MUSTAFAR_API const char *mustafar_status_string(mustafar_status s);
 MUSTAFAR_API const char *mustafar_last_error(void);

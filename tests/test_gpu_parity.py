@@ -154,13 +154,16 @@ def test_split_count_invariance():
         assert float((o.float() - outs[0][0].float()).abs().max()) <= 2e-3
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,L,ragged", [(8, 32, 8, 3000, True), (8, 32, 8, 2300, False), (37, 64, 4, 640, True)])
+@pytest.mark.parametrize("B,Hq,Hkv,L,ragged", [(8, 32, 8, 1024, True), (8, 32, 8, 256, False), (8, 128, 8, 256, True)])
 def test_one_cluster_per_stream_plans(B, Hq, Hkv, L, ragged):
-    """Shapes whose automatic plan gives every stream the same number of CTAs (9 per stream at 8 x 8 kv
-    heads, 3 per stream at 37 x 4 with 16 q heads per kv head): those CTAs form one cluster per stream and
-    merge in distributed shared memory.  Ragged rows (one of them empty) and a fused decode step too."""
-    cap = ((L + 1 + 63) // 64) * 64
-    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.7, 0.5, 61)
+    """Shapes whose automatic plan gives every stream the same whole number C of CTAs with all B x Hkv
+    clusters resident (B200: C = 8 at 8 x 8 kv heads x 1024 tokens, 2 at 256 tokens with 4 or 16 q heads
+    per kv head): those CTAs form one thread-block cluster per stream and merge in
+    distributed shared memory.  Ragged rows (one of them empty) and a fused decode step too; the
+    ticket plan (a forced split count) on the same caches must agree with the oracle as well."""
+    keep = oracle.keep_count(D, 0.7)
+    assert M.mustafar_decode_plan_cluster(B, Hq, Hkv, L, keep, oracle.keep_count(D, 0.5)) >= 2
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, L, 0.7, 0.5, 61)
     seq = synth.seq_lens(B, L, ragged, 61)
     if ragged:
         seq[B // 2] = 0
@@ -172,12 +175,13 @@ def test_one_cluster_per_stream_plans(B, Hq, Hkv, L, ragged):
         U.assert_attn_close(out[rows.to(DEV)], o_ref, lse[rows.to(DEV)], l_ref, tag=tag)
         if ragged:
             assert float(out[B // 2].abs().max()) == 0.0 and torch.isinf(lse[B // 2]).all() and (lse[B // 2] < 0).all()
-    # one fused step: the new token at position L of every row (rows of any length attend over L + 1)
+    # one fused step that rewrites the last token of every row (position L - 1), so that the step
+    # attends over L tokens under the same cluster plan
     kn, vn = synth.step_tokens(B, Hkv, D, 61, 0, DEV)
-    pos = torch.full((B,), L, dtype=torch.int32, device=DEV)
-    out, lse = M.mustafar_decode_step(q, kn, vn, pos, kc, vc, L + 1, 1.0)
-    K[:, :, L], V[:, :, L] = kn, vn
-    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, [L + 1] * B, 1.0)
+    pos = torch.full((B,), L - 1, dtype=torch.int32, device=DEV)
+    out, lse = M.mustafar_decode_step(q, kn, vn, pos, kc, vc, L, 1.0)
+    K[:, :, L - 1], V[:, :, L - 1] = kn, vn
+    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, [L] * B, 1.0)
     U.assert_attn_close(out, o_ref, lse, l_ref, tag="cluster plan fused step")
 
 

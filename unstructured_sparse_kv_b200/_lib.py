@@ -29,7 +29,8 @@ WINDOW_TOKENS = 16
 ABI_SYMBOLS = (
     "mustafar_keep_count", "mustafar_cache_sizes", "mustafar_compress", "mustafar_append",
     "mustafar_decode_workspace_bytes", "mustafar_decode_attn", "mustafar_dense_decode_attn",
-    "mustafar_decode_plan_splits", "mustafar_status_string", "mustafar_last_error", "mustafar_abi_version",
+    "mustafar_decode_plan_splits", "mustafar_decode_plan_cluster", "mustafar_status_string", "mustafar_last_error",
+    "mustafar_abi_version",
     "mustafar_decode_attn_noalloc", "mustafar_decode_step", "mustafar_cache_sizes_per_head",
     "mustafar_keep_count_channel", "mustafar_cache_sizes_channel",
 )
@@ -75,6 +76,7 @@ def load() -> C.CDLL:
         "mustafar_dense_decode_attn": (i32, [vp, i32, vp, vp, i32, i32, i32, i32, vp, i32, f32, vp, vp, vp, sz,
                                              i32, vp, vp]),
         "mustafar_decode_plan_splits": (i32, [i32, i32, i32, i32, i32, i32, i32]),
+        "mustafar_decode_plan_cluster": (i32, [i32, i32, i32, i32, i32, i32, i32]),
         "mustafar_status_string": (C.c_char_p, [i32]),
         "mustafar_last_error": (C.c_char_p, []),
         "mustafar_abi_version": (i32, []),
@@ -153,6 +155,14 @@ def mustafar_decode_plan_splits(batch, num_kv_heads, max_len, keep_k, keep_v, de
     if s < 1:
         raise MustafarError(1, "invalid shapes for the split plan")
     return s
+
+
+def mustafar_decode_plan_cluster(batch, num_q_heads, num_kv_heads, max_len, keep_k, keep_v, head_dim=HEAD_DIM):
+    """CTAs per thread-block cluster of the automatic plan (0: ticket merge through the workspace)."""
+    c = load().mustafar_decode_plan_cluster(batch, num_q_heads, num_kv_heads, head_dim, max_len, keep_k, keep_v)
+    if c < 0:
+        raise MustafarError(1, "invalid shapes for the decode plan")
+    return c
 
 
 # ------------------------------------------------------------------------------------------- caches

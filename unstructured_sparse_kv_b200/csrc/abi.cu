@@ -288,6 +288,18 @@ int32_t mustafar_decode_plan_splits(int32_t batch, int32_t num_kv_heads, int32_t
   return (plan.splits + streams - 1) / streams;
 }
 
+int32_t mustafar_decode_plan_cluster(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t max_len, int32_t keep_k, int32_t keep_v) {
+  if (batch <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      head_dim != kHeadDim || max_len <= 0 || keep_k < 1 || keep_k > kHeadDim || keep_v < 1 || keep_v > kHeadDim)
+    return -1;
+  const int G = num_q_heads / num_kv_heads;
+  if (G > 16 || (G & (G - 1)) != 0) return -1;
+  DecodePlan plan;
+  if (plan_sparse(batch, num_kv_heads, G, max_len, keep_k, keep_v, 0, 0, &plan) != cudaSuccess) return -1;
+  return plan.clu;
+}
+
 namespace {
 
 mustafar_status run_sparse(DecodeParams &p, int max_len, int num_splits, void *workspace, size_t workspace_bytes,

@@ -185,6 +185,34 @@ def test_one_cluster_per_stream_plans(B, Hq, Hkv, L, ragged):
     U.assert_attn_close(out, o_ref, lse, l_ref, tag="cluster plan fused step")
 
 
+def test_cluster_plan_replays_from_a_cuda_graph():
+    """A cluster launch recorded in a CUDA graph (after one eager call of the shape, as for every
+    plan) replays bit-identically to the eager call."""
+    B, Hq, Hkv, L = 8, 32, 8, 1024
+    keep = oracle.keep_count(D, 0.7)
+    assert M.mustafar_decode_plan_cluster(B, Hq, Hkv, L, keep, keep) >= 2
+    K, V, q, kc, vc, seq = _setup(B, Hq, Hkv, L, L, 0.7, 0.7, 67)
+    seq = seq.to(DEV)
+    ref_out, ref_lse = M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=DEV)
+    ws = torch.zeros(M.mustafar_decode_workspace_bytes(B, Hq, Hkv, L), dtype=torch.uint8, device=DEV)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0, out=out, lse=lse, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        M.mustafar_decode_attn(q, kc, vc, seq, L, 1.0, out=out, lse=lse, workspace=ws)
+    out.zero_()
+    lse.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    del g
+
+
 def test_seq_len_zero_and_beyond_capacity():
     B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 21)

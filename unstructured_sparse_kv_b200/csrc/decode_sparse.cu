@@ -855,6 +855,28 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     sh_punit[warp] = u0 + warp;
   }
   __syncwarp();
+  // the four copies of unit punit of stream ps into ring buffer `slot` (lane 0; not the SKEW staging)
+  auto issue = [&](const Stream &ps, int punit, int slot) {
+    const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
+    const uint32_t bar = bars + 8 * slot;
+    const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
+    const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
+    const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
+    if constexpr (PERHEAD) {
+      const int kK = P.hk_k.k[ps.g], kV = P.hk_v.k[ps.g];
+      mbar_expect_tx(bar, 512 + 32 * (kK + kV));
+      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      bulk_g2s(dst + 512, P.kval + P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK, 32 * kK, bar);
+      bulk_g2s(dst + 512 + 32 * kK, P.vval + P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV, 32 * kV, bar);
+    } else {  // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
+      mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
+      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
+      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
+      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
+      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
+    }
+  };
   auto produce = [&](int item) {
     if constexpr (SKEW) {
       // a cache whose keep is a multiple of 32 is staged in groups of 2^lg tokens (about 256 bytes),
@@ -895,31 +917,29 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     if (punit >= u1) return;
     Stream ps = sh_ps[warp];
     while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
-    const int slot = item % NSTAGE;
-    const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
-    const uint32_t bar = bars + 8 * slot;
-    const int64_t sid = static_cast<int64_t>(ps.b) * P.Hkv + ps.g;
-    const int64_t t0 = static_cast<int64_t>(punit - ps.start) * kChunk;
-    const int64_t tk = sid * P.cap_k + t0, tv = sid * P.cap_v + t0;
-    if constexpr (PERHEAD) {
-      const int kK = P.hk_k.k[ps.g], kV = P.hk_v.k[ps.g];
-      mbar_expect_tx(bar, 512 + 32 * (kK + kV));
-      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
-      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-      bulk_g2s(dst + 512, P.kval + P.hk_k.value_base(ps.b, ps.g, P.Hkv, P.cap_k) + t0 * kK, 32 * kK, bar);
-      bulk_g2s(dst + 512 + 32 * kK, P.vval + P.hk_v.value_base(ps.b, ps.g, P.Hkv, P.cap_v) + t0 * kV, 32 * kV, bar);
-    } else {  // stream (b, h) of a uniform cache starts at (b*H + h) * cap * keep
-      mbar_expect_tx(bar, 512 + 32 * (P.keep_k + P.keep_v));
-      bulk_g2s(dst, P.kbm + tk * kWords, 256, bar);
-      bulk_g2s(dst + 256, P.vbm + tv * kWords, 256, bar);
-      bulk_g2s(dst + 512, P.kval + tk * P.keep_k, 32 * P.keep_k, bar);
-      bulk_g2s(dst + 512 + 32 * P.keep_k, P.vval + tv * P.keep_v, 32 * P.keep_v, bar);
-    }
+    issue(ps, punit, item % NSTAGE);
     sh_ps[warp] = ps;
     sh_punit[warp] = punit + kWarps;
   };
+  if constexpr (SKEW) {
 #pragma unroll 1
-  for (int i = 0; i < NSTAGE; ++i) produce(i);
+    for (int i = 0; i < NSTAGE; ++i) produce(i);
+  } else {
+    // the first fill of the ring: lane 0 walks the streams in registers and issues every item in one
+    // pass (the chunk loop's producer keeps its state in shared memory to spare registers)
+    if (lane == 0) {
+      Stream ps = first;
+      int punit = u0 + warp;
+#pragma unroll 1
+      for (int i = 0; i < NSTAGE && punit < u1; ++i, punit += kWarps) {
+        while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
+        issue(ps, punit, i);
+      }
+      sh_ps[warp] = ps;
+      sh_punit[warp] = punit;
+    }
+    __syncwarp();
+  }
 
   Stream cs = first;
   int cunit = u0 + warp, citem = 0;

@@ -677,8 +677,7 @@ template <int NSTAGE, bool HIROWS, bool PERHEAD, bool P24, bool SCAN, bool SKEW>
 __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel(const DecodeParams P) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(16) uint32_t zero_slot[4];
-  __shared__ int sh_info[5];  // U, batch row of the CTA's first unit (-1: none), that row's first unit, u0, u1
-  __shared__ int sh_len[kRowCache];
+  __shared__ int sh_len[kWarps][kRowCache];  // each warp's copy of the row-length cache
   __shared__ int sh_pos[kRowCache];  // fused step: the new token's position in each row
   __shared__ uint32_t sh_bits;       // device error flags of the cached rows this CTA reports
   __shared__ Pending sh_pend[2];
@@ -688,12 +687,25 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   const int cta = blockIdx.x, nctas = gridDim.x;
   const int cap = min(P.cap_k, P.cap_v);
 
-  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts.  Warp 0
-  // reads the lengths of rows below kRowCache in one round of independent loads into sh_len (and
-  // the error flags of the rows this CTA reports); longer batches read the rest from global memory.
-  // With one cluster per stream, the cluster's C CTAs split that stream's chunks evenly and nothing
-  // else.
-  if (warp == 0) {
+  uint8_t *wbase = smem + warp * P.warp_bytes;
+  uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // [32 rows][8 half words] u16 prefixes
+  const uint32_t bars = smem_addr(htab + 512);     // NSTAGE mbarriers of this warp
+  float *mer = reinterpret_cast<float *>(smem + kWarps * P.warp_bytes);
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < NSTAGE; ++i) mbar_init(bars + 8 * i, 1);
+    mbar_init_fence();
+  }
+
+  // ---- the end-to-end chunk sequence: its length U and where this CTA's range starts.  Every warp
+  // computes them itself (the same values), so that it can fill its copy ring without waiting for the
+  // others: it reads the lengths of rows below kRowCache in one round of independent loads into its
+  // own copy of the row cache (warp 0 also collects the error flags of the rows this CTA reports);
+  // longer batches read the rest from global memory.  With one cluster per stream, the cluster's C
+  // CTAs split that stream's chunks evenly and nothing else.
+  int *const my_len = sh_len[warp];
+  int U, u0, u1, row, row_start;  // row: batch row of the CTA's first unit (-1: none); row_start: its first unit
+  {
     int nrow[kRowCache / 32];
     int tot = 0;
     uint32_t bits = 0;
@@ -704,32 +716,39 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       if (b < P.B) {
         uint32_t rb = 0;
         L = row_len(P, b, cap, rb);
-        sh_len[b] = L;
-        if (P.pos != nullptr) sh_pos[b] = P.pos[b];
-        if (b % nctas == cta) bits |= rb;
+        my_len[b] = L;
+        if (warp == 0) {
+          if (P.pos != nullptr) sh_pos[b] = P.pos[b];
+          if (b % nctas == cta) bits |= rb;
+        }
       }
       nrow[i] = P.Hkv * n_chunks(L);
       tot += nrow[i];
     }
-    bits = __reduce_or_sync(0xffffffffu, bits);
-    if (lane == 0) sh_bits = bits;
+    if (warp == 0) {
+      bits = __reduce_or_sync(0xffffffffu, bits);
+      if (lane == 0) sh_bits = bits;
+    }
+    __syncwarp();  // this warp's row cache is complete
     if (P.clu > 0) {
-      // units are counted from the stream's first chunk
-      if (lane == 0) {
-        const int s = cta / P.clu, r = cta % P.clu, b = s / P.Hkv;
-        const int n = n_chunks(len_of(P, sh_len, b, cap));
-        sh_info[0] = 0;
-        sh_info[1] = b;
-        sh_info[2] = s % P.Hkv;
-        sh_info[3] = r * n / P.clu;
-        sh_info[4] = (r + 1) * n / P.clu;
-      }
+      // units are counted from the stream's first chunk; row_start holds the stream's kv head
+      const int s = cta / P.clu, r = cta % P.clu;
+      row = s / P.Hkv;
+      row_start = s % P.Hkv;
+      const int n = n_chunks(len_of(P, my_len, row, cap));
+      U = 0;
+      u0 = r * n / P.clu;
+      u1 = (r + 1) * n / P.clu;
     } else {
       for (int b = kRowCache + lane; b < P.B; b += 32) tot += P.Hkv * n_chunks(row_len(P, b, cap));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-      const int u0 = range_start(cta, tot, nctas);
-      int row = -1, row_start = 0, before = 0;
+      U = tot;
+      u0 = range_start(cta, tot, nctas);
+      u1 = range_start(cta + 1, tot, nctas);
+      row = -1;
+      row_start = 0;
+      int before = 0;
       for (int b0 = 0; b0 < P.B && u0 < tot; b0 += 32) {
         const int b = b0 + lane;
         int n;
@@ -754,94 +773,18 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
         }
         before += __shfl_sync(0xffffffffu, incl, 31);
       }
-      if (lane == 0) {
-        sh_info[0] = tot;
-        sh_info[1] = row;
-        sh_info[2] = row_start;
-        sh_info[3] = u0;
-        sh_info[4] = range_start(cta + 1, tot, nctas);
-      }
     }
   }
-  if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
-  if (threadIdx.x == 0) sh_npend = 0;
-  if (P24 && threadIdx.x < 16) lut24[threadIdx.x] = kLut24[threadIdx.x];
-  uint8_t *wbase = smem + warp * P.warp_bytes;
-  uint8_t *htab = wbase + NSTAGE * P.stage_bytes;  // [32 rows][8 half words] u16 prefixes
-  const uint32_t bars = smem_addr(htab + 512);     // NSTAGE mbarriers of this warp
-  float *mer = reinterpret_cast<float *>(smem + kWarps * P.warp_bytes);
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < NSTAGE; ++i) mbar_init(bars + 8 * i, 1);
-    mbar_init_fence();
-  }
-  __syncthreads();
-  const int U = sh_info[0], u0 = sh_info[3], u1 = sh_info[4];
-
-  // ---- rows this CTA reports on: device error flags, and the output of rows with no tokens
-  uint32_t bits = sh_bits;
-  for (int b = cta; b < P.B; b += nctas) {
-    const int L = b < kRowCache ? sh_len[b] : row_len(P, b, cap, bits);
-    if (L == 0) {
-      uint16_t *o = P.out + static_cast<int64_t>(b) * P.Hq * kHeadDim;
-      for (int i = threadIdx.x; i < P.Hq * kHeadDim; i += kThreads) o[i] = 0;
-      if (P.lse != nullptr)
-        for (int i = threadIdx.x; i < P.Hq; i += kThreads) P.lse[static_cast<int64_t>(b) * P.Hq + i] = kNegInf;
-    }
-  }
-  if (threadIdx.x == 0 && bits != 0u && P.err != nullptr) atomicOr(P.err, bits);
-  if (sh_info[1] < 0) return;  // an empty range at the end of the sequence (never with clusters)
 
   Stream first;
-  first.b = sh_info[1];
-  first.n = n_chunks(len_of(P, sh_len, first.b, cap));
+  first.b = row;
+  first.n = row >= 0 ? n_chunks(len_of(P, my_len, row, cap)) : 0;
   if (P.clu > 0) {
-    first.g = sh_info[2];
+    first.g = row_start;
     first.start = 0;
   } else {
-    first.g = (u0 - sh_info[2]) / first.n;
-    first.start = sh_info[2] + first.g * first.n;
-  }
-
-  // ---- fused decode step: compress the new token of every stream whose new-token chunk lies in
-  // this range (warp 0: K, warp 1: V) before any chunk is copied in
-  if (P.pos != nullptr) {
-    Stream st = first;
-    bool any = false;
-    while (st.start < u1) {
-      const int p = st.b < kRowCache ? sh_pos[st.b] : P.pos[st.b];
-      if (st.n > 0 && p >= 0 && p < cap) {
-        const int unit = st.start + p / kChunk;
-        if (unit >= u0 && unit < u1) {
-          any = true;
-          if (warp < 2) {
-            const bool kside = warp == 0;
-            const uint16_t *src =
-                kside ? P.kn + st.b * P.kn_sb + st.g * P.kn_sh : P.vn + st.b * P.vn_sb + st.g * P.vn_sh;
-            const int capx = kside ? P.cap_k : P.cap_v;
-            const int keep = kside ? keep_of<PERHEAD>(P.hk_k, P.keep_k, st.g) : keep_of<PERHEAD>(P.hk_v, P.keep_v, st.g);
-            const int64_t base = kside ? base_of<PERHEAD>(P.hk_k, P.keep_k, st.b, st.g, P.Hkv, capx)
-                                       : base_of<PERHEAD>(P.hk_v, P.keep_v, st.b, st.g, P.Hkv, capx);
-            // a channel-wise cache got its new token from a separate launch before this one (its whole
-            // window is pruned again, which would weigh on this kernel's registers)
-            if (!SCAN || (kside ? P.kwin : P.vwin) == nullptr) {
-              const int64_t sid = static_cast<int64_t>(st.b) * P.Hkv + st.g;
-              uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + (sid * capx + p) * kWords;
-              uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
-              if (kside ? P.p24_k : P.p24_v)
-                warp_compress_vector_24(src, bm, vals, lane);
-              else
-                warp_compress_vector(src, keep, bm, vals, lane);
-            }
-          }
-        }
-      }
-      if (!next_stream(P, sh_len, cap, st)) break;
-    }
-    if (any) {
-      fence_proxy_async_global();  // these stores before the bulk copies that read them
-      __syncthreads();
-    }
+    first.g = row >= 0 ? (u0 - row_start) / first.n : 0;
+    first.start = row_start + first.g * first.n;
   }
 
   // ---- the warp's chunks: units u0 + warp + 4j of the range, through a ring of NSTAGE buffers
@@ -886,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
       const int punit = sh_punit[warp];
       if (punit >= u1) return;  // the same in every lane
       Stream ps = sh_ps[warp];
-      while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
+      while (punit >= ps.end()) next_stream(P, my_len, cap, ps);
       const int slot = item % NSTAGE;
       const uint32_t dst = smem_addr(wbase + slot * P.stage_bytes);
       const uint32_t bar = bars + 8 * slot;
@@ -916,30 +859,98 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     int punit = sh_punit[warp];
     if (punit >= u1) return;
     Stream ps = sh_ps[warp];
-    while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
+    while (punit >= ps.end()) next_stream(P, my_len, cap, ps);
     issue(ps, punit, item % NSTAGE);
     sh_ps[warp] = ps;
     sh_punit[warp] = punit + kWarps;
   };
-  if constexpr (SKEW) {
+  // fill the copy ring with the warp's first NSTAGE units
+  auto fill = [&]() {
+    if constexpr (SKEW) {
 #pragma unroll 1
-    for (int i = 0; i < NSTAGE; ++i) produce(i);
-  } else {
-    // the first fill of the ring: lane 0 walks the streams in registers and issues every item in one
-    // pass (the chunk loop's producer keeps its state in shared memory to spare registers)
-    if (lane == 0) {
-      Stream ps = first;
-      int punit = u0 + warp;
+      for (int i = 0; i < NSTAGE; ++i) produce(i);
+    } else {
+      // lane 0 walks the streams in registers and issues every item in one pass (the chunk loop's
+      // producer keeps its state in shared memory to spare registers)
+      if (lane == 0) {
+        Stream ps = first;
+        int punit = u0 + warp;
 #pragma unroll 1
-      for (int i = 0; i < NSTAGE && punit < u1; ++i, punit += kWarps) {
-        while (punit >= ps.end()) next_stream(P, sh_len, cap, ps);
-        issue(ps, punit, i);
+        for (int i = 0; i < NSTAGE && punit < u1; ++i, punit += kWarps) {
+          while (punit >= ps.end()) next_stream(P, my_len, cap, ps);
+          issue(ps, punit, i);
+        }
+        sh_ps[warp] = ps;
+        sh_punit[warp] = punit;
       }
-      sh_ps[warp] = ps;
-      sh_punit[warp] = punit;
+      __syncwarp();
     }
-    __syncwarp();
+  };
+  // attention alone: fill the ring before waiting for the other warps (a fused step fills it after
+  // the new tokens are in the caches, below)
+  if (P.pos == nullptr && row >= 0) fill();
+
+  if (threadIdx.x < 4) zero_slot[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) sh_npend = 0;
+  if (P24 && threadIdx.x < 16) lut24[threadIdx.x] = kLut24[threadIdx.x];
+  __syncthreads();
+
+  // ---- rows this CTA reports on: device error flags, and the output of rows with no tokens
+  uint32_t bits = sh_bits;
+  for (int b = cta; b < P.B; b += nctas) {
+    const int L = b < kRowCache ? my_len[b] : row_len(P, b, cap, bits);
+    if (L == 0) {
+      uint16_t *o = P.out + static_cast<int64_t>(b) * P.Hq * kHeadDim;
+      for (int i = threadIdx.x; i < P.Hq * kHeadDim; i += kThreads) o[i] = 0;
+      if (P.lse != nullptr)
+        for (int i = threadIdx.x; i < P.Hq; i += kThreads) P.lse[static_cast<int64_t>(b) * P.Hq + i] = kNegInf;
+    }
   }
+  if (threadIdx.x == 0 && bits != 0u && P.err != nullptr) atomicOr(P.err, bits);
+  if (row < 0) return;  // an empty range at the end of the sequence (never with clusters)
+
+  // ---- fused decode step: compress the new token of every stream whose new-token chunk lies in
+  // this range (warp 0: K, warp 1: V) before any chunk is copied in
+  if (P.pos != nullptr) {
+    Stream st = first;
+    bool any = false;
+    while (st.start < u1) {
+      const int p = st.b < kRowCache ? sh_pos[st.b] : P.pos[st.b];
+      if (st.n > 0 && p >= 0 && p < cap) {
+        const int unit = st.start + p / kChunk;
+        if (unit >= u0 && unit < u1) {
+          any = true;
+          if (warp < 2) {
+            const bool kside = warp == 0;
+            const uint16_t *src =
+                kside ? P.kn + st.b * P.kn_sb + st.g * P.kn_sh : P.vn + st.b * P.vn_sb + st.g * P.vn_sh;
+            const int capx = kside ? P.cap_k : P.cap_v;
+            const int keep = kside ? keep_of<PERHEAD>(P.hk_k, P.keep_k, st.g) : keep_of<PERHEAD>(P.hk_v, P.keep_v, st.g);
+            const int64_t base = kside ? base_of<PERHEAD>(P.hk_k, P.keep_k, st.b, st.g, P.Hkv, capx)
+                                       : base_of<PERHEAD>(P.hk_v, P.keep_v, st.b, st.g, P.Hkv, capx);
+            // a channel-wise cache got its new token from a separate launch before this one (its whole
+            // window is pruned again, which would weigh on this kernel's registers)
+            if (!SCAN || (kside ? P.kwin : P.vwin) == nullptr) {
+              const int64_t sid = static_cast<int64_t>(st.b) * P.Hkv + st.g;
+              uint32_t *bm = const_cast<uint32_t *>(kside ? P.kbm : P.vbm) + (sid * capx + p) * kWords;
+              uint16_t *vals = const_cast<uint16_t *>(kside ? P.kval : P.vval) + base + static_cast<int64_t>(p) * keep;
+              if (kside ? P.p24_k : P.p24_v)
+                warp_compress_vector_24(src, bm, vals, lane);
+              else
+                warp_compress_vector(src, keep, bm, vals, lane);
+            }
+          }
+        }
+      }
+      if (!next_stream(P, my_len, cap, st)) break;
+    }
+    if (any) {
+      fence_proxy_async_global();  // these stores before the bulk copies that read them
+      __syncthreads();
+    }
+    fill();
+  }
+
 
   Stream cs = first;
   int cunit = u0 + warp, citem = 0;
@@ -948,7 +959,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
   uint32_t qa[8][4];
   for (;;) {
     const int seg_a = max(cs.start, u0), seg_e = min(cs.end(), u1);
-    const int L = len_of(P, sh_len, cs.b, cap);
+    const int L = len_of(P, my_len, cs.b, cap);
     const int kK = keep_of<PERHEAD>(P.hk_k, P.keep_k, cs.g), kV = keep_of<PERHEAD>(P.hk_v, P.keep_v, cs.g);
     load_q<HIROWS>(P, cs.b, cs.g, lane, qa);
     acc.reset();
@@ -967,7 +978,7 @@ __global__ void __launch_bounds__(kThreads, HIROWS ? 3 : 4) sparse_decode_kernel
     if (seg_e >= u1) break;
     bool more;
     do {
-      more = next_stream(P, sh_len, cap, cs);
+      more = next_stream(P, my_len, cap, cs);
     } while (more && cs.n == 0);
     if (!more) break;
   }

@@ -213,6 +213,49 @@ def test_cluster_plan_replays_from_a_cuda_graph():
     del g
 
 
+@pytest.mark.parametrize("kind", ["per-head", "2:4", "channel", "keep-64 skewed staging"])
+def test_cache_variants_under_a_cluster_plan(kind):
+    """The other cache formats at a shape whose plan is one 8-CTA cluster per stream for uniform caches
+    (batch 8 x 8 kv heads x 1024 tokens): the variants share the plan, the range split and the cluster
+    merge.  Ragged rows, one of them empty."""
+    B, Hq, Hkv, L = 8, 32, 8, 1024
+    K = synth.keys(B, Hkv, L, D, 91, DEV)
+    V = synth.values(B, Hkv, L, D, 91, DEV)
+    Kb, Vb = U.bits(K), U.bits(V)
+    if kind == "per-head":
+        sK, sV = [0.5, 0.6, 0.7, 0.8, 0.9, 0.7, 0.6, 0.8], [0.8, 0.6, 0.7, 0.9, 0.8, 0.7, 0.6, 0.5]
+        kc, vc = M.CompressedCache(B, Hkv, L, sK), M.CompressedCache(B, Hkv, L, sV)
+        M.mustafar_compress(K, L, 0.0, kc)
+        M.mustafar_compress(V, L, 0.0, vc)
+        kp, vp = oracle.prune_heads(Kb, kc.head_keep), oracle.prune_heads(Vb, vc.head_keep)
+    elif kind == "2:4":
+        kc, vc = M.CompressedCache(B, Hkv, L, 0.5, pattern="2:4"), M.CompressedCache(B, Hkv, L, 0.5, pattern="2:4")
+        M.mustafar_compress(K, L, 0.5, kc)
+        M.mustafar_compress(V, L, 0.5, vc)
+        kp, vp = oracle.prune_24(Kb), oracle.prune_24(Vb)
+    elif kind == "channel":
+        kc, vc = M.CompressedCache(B, Hkv, L, 0.7, pattern="channel"), M.CompressedCache(B, Hkv, L, 0.7)
+        M.mustafar_compress(K, L, 0.7, kc)
+        M.mustafar_compress(V, L, 0.7, vc)
+        kp, vp = oracle.prune_channel(Kb, 0.7), oracle.prune(Vb, oracle.keep_count(D, 0.7))
+    else:
+        keep = oracle.keep_count(D, 0.5)
+        assert keep == 64 and M.mustafar_decode_plan_cluster(B, Hq, Hkv, L, keep, keep) >= 2
+        kc, vc = M.CompressedCache(B, Hkv, L, 0.5), M.CompressedCache(B, Hkv, L, 0.5)
+        M.mustafar_compress(K, L, 0.5, kc)
+        M.mustafar_compress(V, L, 0.5, vc)
+        kp, vp = oracle.prune(Kb, keep), oracle.prune(Vb, keep)
+    q = synth.queries(B, Hq, D, 91, DEV)
+    seq = synth.seq_lens(B, L, True, 91)
+    seq[0] = L
+    seq[3] = 0
+    out, lse = M.mustafar_decode_attn(q, kc, vc, seq.to(DEV), L, 0.088)
+    rows = (seq > 0).nonzero().flatten()
+    o_ref, l_ref = oracle.attention(U.bits(q[rows]), kp[rows.numpy()], vp[rows.numpy()], seq[rows].numpy(), 0.088)
+    U.assert_attn_close(out[rows.to(DEV)], o_ref, lse[rows.to(DEV)], l_ref, tag=f"{kind} caches, cluster plan")
+    assert float(out[3].abs().max()) == 0.0 and torch.isinf(lse[3]).all()
+
+
 def test_seq_len_zero_and_beyond_capacity():
     B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 21)

@@ -7,8 +7,8 @@
 // compress: one CTA = 128 consecutive tokens of one (b, kv head) stream, one thread per
 //   token.  The CTA stages its 32 KB of dense rows in shared memory with coalesced
 //   16-byte cp.async (16 threads per 256-byte row), each thread runs the top-k on its
-//   own row and writes its 16-byte bitmap; then the CTA packs the kept values into a shared
-//   staging run (one thread per 8-channel slice of a row) and writes the 128*k packed values
+//   own row, writes its 16-byte bitmap and packs its kept values into a shared staging run
+//   (one predicated 16-bit store per channel); then the CTA writes the 128*k packed values
 //   with coalesced 16-byte stores.
 // append: one warp per (b, kv head) vector of the new token.
 // channel-wise caches: one warp per 16-token window (compress) or per stream's newest window
@@ -19,11 +19,24 @@
 namespace mustafar {
 
 constexpr int kCompressThreads = 128;
-constexpr int kThreadPackMaxKeep = 48;  // up to this keep a thread packs its own row (measured crossover)
 constexpr int kRowBytesDense = kHeadDim * 2;  // 256
 
 // byte offset of 16-byte chunk j of staged row `tok` (XOR swizzle: conflict-free row reads)
 __device__ __forceinline__ int stage_off(int tok, int j) { return tok * kRowBytesDense + ((j ^ (tok & 15)) << 4); }
+
+// Channels I and I+1 of a chunk (the halves of x): each whose bit is set in `bits` is stored at the
+// shared address dst, which then steps by one value.
+template <int I>
+__device__ __forceinline__ void pack_pair(uint32_t &dst, uint32_t bits, uint32_t x) {
+  asm volatile(
+      "{\n .reg .pred p, q;\n .reg .b32 t, h;\n"
+      " and.b32 t, %1, %3;\n setp.ne.u32 p, t, 0;\n @p st.shared.u16 [%0], %2;\n @p add.u32 %0, %0, 2;\n"
+      " and.b32 t, %1, %4;\n setp.ne.u32 q, t, 0;\n shr.u32 h, %2, 16;\n @q st.shared.u16 [%0], h;\n"
+      " @q add.u32 %0, %0, 2;\n}\n"
+      : "+r"(dst)
+      : "r"(bits), "r"(x), "n"(1u << I), "n"(2u << I)
+      : "memory");
+}
 
 template <bool P24>
 __global__ void __launch_bounds__(kCompressThreads)
@@ -31,7 +44,6 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
                 int cap, uint32_t *__restrict__ bitmap, uint16_t *__restrict__ values,
                 uint32_t *__restrict__ tile_offset) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint4 bm_sh[kCompressThreads];  // the CTA's bitmap rows, for the packing pass
   uint8_t *in_stage = smem;
   uint16_t *out_stage = reinterpret_cast<uint16_t *>(smem + kCompressThreads * kRowBytesDense);
 
@@ -90,39 +102,21 @@ compress_kernel(const uint16_t *__restrict__ x, int64_t sb, int64_t sh, int64_t 
     }
     const uint4 row = make_uint4(bm[0], bm[1], bm[2], bm[3]);
     reinterpret_cast<uint4 *>(bitmap)[stream * cap + t0 + tid] = row;
-    bm_sh[tid] = row;
-    if (k <= kThreadPackMaxKeep) {
-      // few kept values: the thread packs its own row, walking the set bits
-      uint16_t *dst = out_stage + tid * k;
-      int jj = 0;
+    if (popc4(bm) == k) {  // (the bitmap holds k bits by construction; the check keeps the run in bounds)
+      // the thread packs its own row: one predicated 16-bit store per channel (bit set: store and step
+      // the run pointer), reading the staged row 16 bytes at a time, so the cost does not grow with k
+      // (a walk over the set bits costs about 25 instructions per kept value, and a CTA-wide pass with
+      // one thread per 8-channel slice of a row measured slower than this at every keep)
+      uint32_t dst = smem_addr(out_stage + tid * k);
 #pragma unroll
-      for (int w = 0; w < kWords; ++w) {
-        uint32_t m = bm[w];
-        while (m && jj < k) {
-          const int ch = 32 * w + __ffs(m) - 1;
-          m &= m - 1;
-          dst[jj++] = *reinterpret_cast<const uint16_t *>(in_stage + stage_off(tid, ch >> 3) + ((ch & 7) << 1));
-        }
+      for (int j = 0; j < 16; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(in_stage + stage_off(tid, j));
+        const uint32_t bits = bm[j >> 2] >> (8 * (j & 3));  // channels 8j .. 8j+7
+        pack_pair<0>(dst, bits, v.x);
+        pack_pair<2>(dst, bits, v.y);
+        pack_pair<4>(dst, bits, v.z);
+        pack_pair<6>(dst, bits, v.w);
       }
-    }
-  }
-  __syncthreads();
-
-  // many kept values: one thread per (token, 8-channel slice) packs the slice's kept values, so the
-  // cost does not grow with the keep count; token t's run starts at t*k of the staging run
-  for (int item = tid; k > kThreadPackMaxKeep && item < ntok * 16; item += kCompressThreads) {
-    const int tok = item >> 4, j = item & 15, wi = j >> 2, sh = 8 * (j & 3);
-    const uint4 row = bm_sh[tok];
-    const uint32_t word = wi == 0 ? row.x : wi == 1 ? row.y : wi == 2 ? row.z : row.w;
-    const uint32_t mb = (word >> sh) & 0xFFu;
-    if (mb == 0u) continue;
-    int pos = tok * k + __popc(word & ((1u << sh) - 1u)) + (wi > 0 ? __popc(row.x) : 0) + (wi > 1 ? __popc(row.y) : 0) +
-              (wi > 2 ? __popc(row.z) : 0);
-    const uint4 v = *reinterpret_cast<const uint4 *>(in_stage + stage_off(tok, j));
-    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if ((mb >> i) & 1u) out_stage[pos++] = static_cast<uint16_t>(vv[i >> 1] >> (16 * (i & 1)));
     }
   }
   __syncthreads();

@@ -18,6 +18,11 @@
 //   warps merge (m, l, o) in shared memory.  A stream whose chunks all lie in one range is
 //   finished by that CTA; a stream cut by range edges leaves one partial per CTA in the
 //   workspace and the last of those CTAs to finish (atomic ticket, no waiting) merges them.
+//   When the plan gives every stream the same whole number C of CTAs and all the streams' C-CTA
+//   thread-block clusters are resident at once, each stream's CTAs run as one cluster instead
+//   and merge through distributed shared memory between two cluster barriers.
+// * every warp reads the row lengths and computes its CTA's range itself, so that it can start
+//   its copies before the CTA-wide barrier.
 // * each warp stages its chunks through its own ring of NSTAGE buffers.  One lane issues, per
 //   chunk, four bulk copies of contiguous bytes (K bitmap rows, V bitmap rows, K packed values,
 //   V packed values) that complete on the buffer's mbarrier; every wait is bounded in time.

@@ -243,3 +243,19 @@ def test_24_cache_cannot_have_head_keep(lib):
     st, err = _status(lib, "mustafar_append", 0x5000, 256, 100, 0x6000, C.byref(c), None, None)
     assert st == 1 and "2:4" in err, (st, err)
 
+
+
+def test_plan_queries_reject_invalid_shapes(lib):
+    # shape checks come before any device query, so they answer without a GPU
+    plan_cluster = lib.mustafar_decode_plan_cluster
+    assert plan_cluster(8, 24, 8, 128, 1024, 39, 39) == -1   # 3 q heads per kv head
+    assert plan_cluster(8, 36, 8, 128, 1024, 39, 39) == -1   # q heads not a multiple of kv heads
+    assert plan_cluster(8, 32, 8, 64, 1024, 39, 39) == -1    # head_dim other than 128
+    assert plan_cluster(8, 32, 8, 128, 0, 39, 39) == -1      # no context
+    assert plan_cluster(8, 32, 8, 128, 1024, 0, 39) == -1    # keep out of range
+    assert plan_cluster(8, 32, 8, 128, 1024, 39, 129) == -1
+    assert plan_cluster(0, 32, 8, 128, 1024, 39, 39) == -1   # no batch
+    assert plan_cluster(8, 512, 8, 128, 1024, 39, 39) == -1  # 64 q heads per kv head
+    assert lib.mustafar_decode_plan_splits(8, 8, 64, 1024, 39, 39, 0) == -1
+    with pytest.raises(M.MustafarError):
+        M.mustafar_decode_plan_cluster(8, 24, 8, 1024, 39, 39)

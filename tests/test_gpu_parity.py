@@ -256,6 +256,35 @@ def test_cache_variants_under_a_cluster_plan(kind):
     assert float(out[3].abs().max()) == 0.0 and torch.isinf(lse[3]).all()
 
 
+@pytest.mark.parametrize("splits", [0, 2])
+def test_batches_beyond_the_row_cache(splits):
+    """More than 128 batch rows: rows from 128 on are read from global memory by the range search, the
+    stream steps and the row reports (the first 128 come from the shared row cache), and the fused step
+    reads their positions from global memory too.  Ragged rows, empty rows on both sides of 128."""
+    B, Hq, Hkv, L, cap = 300, 8, 1, 100, 128
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.7, 0.5, 131)
+    seq = synth.seq_lens(B, L, True, 131)
+    seq[[5, 127, 128, 200, 299]] = 0
+    rows = (seq > 0).nonzero().flatten()
+    out, lse = _attend(q, kc, vc, seq, L, 1.0, splits)
+    o_ref, l_ref = U.oracle_attention(q[rows], U.bits(K)[rows], U.bits(V)[rows], kc.keep, vc.keep,
+                                      seq[rows].numpy(), 1.0)
+    U.assert_attn_close(out[rows.to(DEV)], o_ref, lse[rows.to(DEV)], l_ref, tag=f"{B} rows, splits {splits}")
+    empty = (seq == 0).nonzero().flatten().to(DEV)
+    assert float(out[empty].abs().max()) == 0.0 and torch.isinf(lse[empty]).all()
+    # one fused step, each row appending at its own position (an empty row at position 3)
+    pos = seq.clone()
+    pos[pos == 0] = 3
+    posd = pos.to(DEV)
+    kn, vn = synth.step_tokens(B, Hkv, D, 131, 0, DEV)
+    out, lse = M.mustafar_decode_step(q, kn, vn, posd, kc, vc, L + 1, 1.0, num_splits=splits)
+    every = torch.arange(B, device=DEV)
+    K[every, :, posd.long()] = kn
+    V[every, :, posd.long()] = vn
+    o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, (pos + 1).numpy(), 1.0)
+    U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"{B} rows, fused step, splits {splits}")
+
+
 def test_seq_len_zero_and_beyond_capacity():
     B, Hq, Hkv, L, cap = 3, 8, 2, 64, 64
     K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.5, 0.5, 21)

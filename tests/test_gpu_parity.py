@@ -133,6 +133,10 @@ def test_append_rows_at_different_positions_and_out_of_range():
     (2, 8, 2, 150, 0.25, 0.7, 2, True),    # one cache staged token by token, one in a single copy
     (2, 8, 2, 213, 0.5, 0.5, 3, True),     # keep 64 in both caches: staged in 4-token groups
     (1, 32, 2, 170, 0.0, 0.25, 0, False),  # G = 16 with both caches staged token by token
+    (2, 8, 2, 200, 0.9, 0.9, 0, True),     # keep 13: few kept values per token
+    (2, 12, 4, 129, 0.85, 0.9, 3, True),   # keeps 20 and 13, G = 3, forced splits
+    (1, 32, 2, 300, 0.9, 0.8, 0, True),    # G = 16 with keeps 13 and 26
+    (2, 8, 2, 150, 0.9, 0.7, 0, True),     # keeps 13 and 39
 ])
 def test_decode_small_cases(B, Hq, Hkv, L, sK, sV, splits, ragged):
     cap = ((L + 63) // 64) * 64
@@ -283,6 +287,26 @@ def test_batches_beyond_the_row_cache(splits):
     V[every, :, posd.long()] = vn
     o_ref, l_ref = U.oracle_attention(q, U.bits(K), U.bits(V), kc.keep, vc.keep, (pos + 1).numpy(), 1.0)
     U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"{B} rows, fused step, splits {splits}")
+
+
+def test_decode_step_with_few_kept_values():
+    """Fused steps on caches with few kept values per token (s = 0.9, keep 13), rows at their own
+    positions."""
+    B, Hq, Hkv, L, cap = 4, 32, 8, 700, 768
+    K, V, q, kc, vc, _ = _setup(B, Hq, Hkv, L, cap, 0.9, 0.9, 141)
+    pos = synth.seq_lens(B, L, True, 141)
+    posd = pos.to(DEV)
+    every = torch.arange(B, device=DEV)
+    for st in range(2):
+        qs = synth.queries(B, Hq, D, 141, DEV, step=st + 1)
+        kn, vn = synth.step_tokens(B, Hkv, D, 141, st, DEV)
+        out, lse = M.mustafar_decode_step(qs, kn, vn, posd, kc, vc, L + 2, 1.0)
+        K[every, :, posd.long()] = kn
+        V[every, :, posd.long()] = vn
+        o_ref, l_ref = U.oracle_attention(qs, U.bits(K), U.bits(V), kc.keep, vc.keep, (pos + 1).numpy(), 1.0)
+        U.assert_attn_close(out, o_ref, lse, l_ref, tag=f"keep 13, fused step {st}")
+        pos = pos + 1
+        posd = pos.to(DEV)
 
 
 def test_seq_len_zero_and_beyond_capacity():
